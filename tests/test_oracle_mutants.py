@@ -1,0 +1,92 @@
+"""Planted mistakes in the oracle must each fail at least one pin.
+
+Each case below edits a copy of ``oracle/ep_oracle.c`` (the committed source is
+never touched), builds it into a temporary library, routes the oracle through it
+and runs the pins until one fails.  A mistake that no pin catches means a pin is
+missing.  Mistakes that would write out of bounds in the mutated C code are not
+planted.
+"""
+
+import pytest
+
+import oracle
+from oracle import build as oracle_build
+import pins
+
+MUTANTS = {
+    "combine_descending_k": (
+        "for (int64_t k = 0; k < K; k++) {\n            int32_t slot = pair_slot[t * K + k];\n"
+        "            if (slot < 0)\n                continue;",
+        "for (int64_t k = K - 1; k >= 0; k--) {\n            int32_t slot = pair_slot[t * K + k];\n"
+        "            if (slot < 0)\n                continue;"),
+    "combine_sign": ("acc[h] = acc[h] + product;", "acc[h] = acc[h] - product;"),
+    "combine_ignores_weights": ("float w = topk_weights ? topk_weights[t * K + k] : 1.0f;",
+                                "float w = 1.0f;"),
+    "combine_drops_k0": ("            if (slot < 0)\n                continue;\n            float w",
+                         "            if (slot < 0 || k == 0)\n                continue;\n            float w"),
+    "combine_fused_multiply_add": (
+        "float product = w * bf16_to_f32(row[h]);\n                acc[h] = acc[h] + product;",
+        "acc[h] = fmaf(w, bf16_to_f32(row[h]), acc[h]);"),
+    "bf16_truncates": ("if (dropped > 0x8000u || (dropped == 0x8000u && (upper & 1u)))", "if (0)"),
+    "bf16_ties_away": ("if (dropped > 0x8000u || (dropped == 0x8000u && (upper & 1u)))",
+                       "if (dropped >= 0x8000u)"),
+    "e4m3_ties_up": ("if (above < below || (above == below && ((code + 1) & 1u) == 0))",
+                     "if (above <= below)"),
+    "e4m3_max_240": ("if (a >= 448.0)\n        return (uint8_t)(sign | 0x7e);",
+                     "if (a >= 240.0)\n        return (uint8_t)(sign | 0x77);"),
+    "e4m3_drops_sign_of_zero": ("uint8_t sign = signbit(v) ? 0x80 : 0x00;",
+                                "uint8_t sign = (v < 0.0f) ? 0x80 : 0x00;"),
+    "cast_fp8_max_240": ("float s = amax / 448.0f;", "float s = amax / 240.0f;"),
+    "cast_reciprocal_multiply": ("float quotient = bf16_to_f32(blk[j]) / s;",
+                                 "float quotient = bf16_to_f32(blk[j]) * (1.0f / s);"),
+    "cast_no_amax_clamp": ("if (amax < 1e-4f)\n                amax = 1e-4f;", ""),
+    "cast_amax_half_block": ("for (int j = 0; j < 128; j++) {\n                float a = fabsf(",
+                             "for (int j = 0; j < 64; j++) {\n                float a = fabsf("),
+    "layout_k_major": (
+        "for (int64_t t = 0; t < T; t++) {\n        for (int64_t k = 0; k < K; k++) {\n"
+        "            int64_t i = t * K + k;\n            int64_t e = topk_idx[i];\n            if (e < 0) {",
+        "for (int64_t k = 0; k < K; k++) {\n        for (int64_t t = 0; t < T; t++) {\n"
+        "            int64_t i = t * K + k;\n            int64_t e = topk_idx[i];\n            if (e < 0) {"),
+    "layout_unaligned_offsets": ("off[e + 1] = (int32_t)(off[e] + align_up(cnt[e], A));",
+                                 "off[e + 1] = (int32_t)(off[e] + cnt[e]);"),
+    "layout_local_expert_div": ("recv_lexp[slot] = (int32_t)(e % experts_per_rank);",
+                                "recv_lexp[slot] = (int32_t)(e / experts_per_rank);"),
+    "layout_pad_weight_one": ("recv_w[slot] = 0.0f;", "recv_w[slot] = 1.0f;"),
+    "layout_no_rank_limit": ("if (max_tokens_per_rank > 0 && T / R > max_tokens_per_rank)", "if (0)"),
+    "routing_start_exclusive": ("if (e >= local_start && e < local_end)",
+                                "if (e > local_start && e < local_end)"),
+    "dispatch_no_zero_padding": ("if (do_zero_padding)\n        for", "if (0)\n        for"),
+}
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(oracle_build.SRC) as f:
+        return f.read()
+
+
+def _run_pins():
+    for pin in pins.ALL_PINS:
+        try:
+            pin()
+        except (AssertionError, oracle.OracleError) as exc:
+            return pin.__name__, exc
+    return None, None
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, source, tmp_path):
+    old, new = MUTANTS[name]
+    assert source.count(old) == 1, "mutation anchor for %s must occur exactly once" % name
+    src = tmp_path / "mutant.c"
+    src.write_text(source.replace(old, new))
+    lib = oracle_build.build(str(src), str(tmp_path / "libmutant.so"), force=True,
+                             extra_flags=["-Wno-error", "-w"])
+    with oracle.use_library(lib):
+        caught_by, _ = _run_pins()
+    assert caught_by is not None, "no pin caught the planted mistake %r" % name
+
+
+def test_unmutated_oracle_passes_all_pins():
+    caught_by, exc = _run_pins()
+    assert caught_by is None, "%s: %s" % (caught_by, exc)
