@@ -1,0 +1,430 @@
+"""Benchmark: MoE dispatch + combine on one B200 (or N independent replicas).
+
+One step = the whole hot path over one batch: ep_layout (count + assign
+kernels), ep_dispatch (with the fused FP8 cast for the FP8 workload) and
+ep_combine, on the default workload "prefill_bf16": T = 4096 tokens,
+H = 7168 bf16, 256 experts, top-8, R = 8 virtual ranks, expert_alignment 128,
+zero padding, skewed (Zipf s = 1.2 bias) gate.  Inputs are seeded synthetic
+(workload/), resident in HBM before timing; the combine input ("expert
+outputs") is the dispatched receive buffer itself (identity experts).
+
+Timing: W warm-up steps, then K steps; before every step L2 is flushed by
+writing a 256 MiB buffer (outside the timed events); each step is timed with
+CUDA events on the launching stream, and per kernel as well.  Multi-GPU
+(torchrun): every rank runs its own replica (the path is one GPU's HBM; no
+data-path collective), the step time is the max over ranks, `value` sums the
+tokens of all ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workload  # noqa: E402
+
+METRIC = "dispatch+combine tokens/s and achieved HBM GB/s vs B200 peak (1 GPU)"
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=30)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="prefill_bf16", choices=sorted(workload.WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    return p.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def source_hash(path):
+    with open(os.path.join(ROOT, path), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel, wl):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    rec = d.get("%s@%s" % (kernel, wl))
+    if not rec or rec.get("source_sha") != source_hash(rec["source"]):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," \
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        rows = [r for r in self.rows if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# algorithmic bytes (the minimum each step must move)
+# --------------------------------------------------------------------------
+def algorithmic_bytes(cfg, cnt, A):
+    T, H, K, E = cfg["T"], cfg["H"], cfg["K"], cfg["E"]
+    N = int(cnt.sum())
+    Np = int(((cnt + A - 1) // A * A).sum())
+    pad = (Np - N) if cfg["zero_pad"] else 0
+    nb = H // 128
+    out_row = (H + 4 * nb) if cfg["fp8"] else 2 * H
+    layout_b = T * K * 8 * 2 + T * K * 4 * 2 + Np * 12 + E * 8      # idx read twice, weights, slots, maps
+    dispatch_b = T * 2 * H + (N + pad) * out_row + T * K * 4
+    combine_b = N * 2 * H + T * K * 8 + T * 2 * H
+    return dict(layout=layout_b, dispatch=dispatch_b, combine=combine_b, N=N, Np=Np, pad_rows=Np - N)
+
+
+# --------------------------------------------------------------------------
+# our implementation
+# --------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import combine_ep_layout_11_b200 as ep
+    from combine_ep_layout_11_b200 import build as lib_build
+    if rank == 0 or not os.path.exists(lib_build.LIB):
+        lib_build.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    cfg = workload.config(args.workload)
+    inp = workload.inputs(cfg)
+    T, H, K, E, R, A = cfg["T"], cfg["H"], cfg["K"], cfg["E"], cfg["R"], cfg["A"]
+    idx = torch.from_numpy(inp["topk_idx"]).to(dev)
+    w = torch.from_numpy(inp["topk_weights"]).to(dev)
+    x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+    lay = ep.Layout(T, K, E, R, A, dev, num_max_tokens_per_rank=cfg["max_tokens_per_rank"])
+    cap = lay.capacity
+    fp8 = cfg["fp8"]
+    recv = torch.empty((cap, H), dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16, device=dev)
+    recv_s = torch.empty((cap, H // 128), dtype=torch.float32, device=dev) if fp8 else None
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def dispatch():
+        if fp8:
+            ep.dispatch(lay, x, cast_to_fp8=True, do_zero_padding=cfg["zero_pad"], out=recv, out_scales=recv_s)
+        else:
+            ep.dispatch(lay, x, do_zero_padding=cfg["zero_pad"], out=recv)
+
+    # expert outputs for combine: identity experts (bf16), or seeded outputs for FP8
+    ep.layout(idx, w, E, R, A, cfg["max_tokens_per_rank"], out=lay)
+    dispatch()
+    torch.cuda.synchronize(dev)
+    if fp8:
+        y = torch.from_numpy(workload.expert_outputs(cfg, cap).view(np.int16)).to(dev).view(torch.bfloat16)
+    else:
+        y = recv.clone()
+    cnt = lay.num_recv_tokens_per_expert.cpu().numpy()
+    nbytes = algorithmic_bytes(cfg, cnt, A)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        ep.layout(idx, w, E, R, A, cfg["max_tokens_per_rank"], out=lay)
+        if evs:
+            evs[1].record(stream)
+        dispatch()
+        if evs:
+            evs[2].record(stream)
+        ep.combine(lay, y, w, out=out)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    code, flags = ep.get_status(lay)
+    assert code == 0, "device status %d (flags %d)" % (code, flags)
+    if not fp8 and cfg["drop"] == 0:   # identity experts with weights summing to 1 reproduce x
+        has = (idx >= 0).any(dim=1)
+        assert torch.equal(out[has].float(), x[has].float()), "combine(dispatch(x)) != x"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank) if (rank == 0 and not args.no_clocks) else None
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - wall0
+    if dist:
+        dist.barrier()
+    clock_info = clocks.stop() if clocks else None
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(args.steps)])
+    step_ms = per.sum(axis=1)
+    ms_per_step = float(step_ms.mean())
+    if dist:
+        tt = torch.tensor([ms_per_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_per_step = float(tt.item())
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush)
+        if dist:
+            tt = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e["ms_per_step"] = float(tt.item())
+
+    if rank != 0:
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return None
+
+    peak, peak_kind = measured_peaks()
+    k_ms = per.mean(axis=0)   # layout, dispatch, combine
+    total_bytes = nbytes["layout"] + nbytes["dispatch"] + nbytes["combine"]
+    disp_gbs = nbytes["dispatch"] / (k_ms[1] * 1e-3) / 1e9
+    value = T * world / (ms_per_step * 1e-3)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8-e4m3/bf16" if fp8 else "bf16",
+        "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
+        "config": {"workload": "%s: T=%d H=%d E=%d top-%d R=%d align=%d zero_pad=%s%s" % (
+            cfg["name"], T, H, E, K, R, A, cfg["zero_pad"], " fp8-cast" if fp8 else ""),
+            "global_batch": T * world, "parallelism": "replicas x%d (R=%d virtual ranks per GPU)" % (world, R),
+            "l2": "flushed by a 256 MiB write before every step, outside the timed events",
+            "pairs": nbytes["N"], "recv_rows": nbytes["Np"], "pad_rows": nbytes["pad_rows"],
+            "load": workload.load_stats(inp["topk_idx"], E)},
+        "hbm_gbs": round(total_bytes / (ms_per_step * 1e-3) / 1e9, 1),
+        "hbm_frac_of_measured": round(total_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+        "hbm_frac_of_nominal_8tbs": round(total_bytes / (ms_per_step * 1e-3) / 1e9 / 8000.0, 4),
+        "algorithmic_bytes_per_step": total_bytes,
+        "kernels_us": {"layout": round(k_ms[0] * 1e3, 2), "dispatch": round(k_ms[1] * 1e3, 2),
+                       "combine": round(k_ms[2] * 1e3, 2)},
+        "kernels_gbs": {"dispatch": round(disp_gbs, 1),
+                        "combine": round(nbytes["combine"] / (k_ms[2] * 1e-3) / 1e9, 1)},
+        "roofline": {"bound": "hbm", "kernel": "dispatch_cast_kernel" if fp8 else "dispatch_copy_kernel",
+                     "achieved": round(disp_gbs, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(disp_gbs / peak, 4),
+                     "traffic": ncu_traffic("dispatch_cast_kernel" if fp8 else "dispatch_copy_kernel",
+                                            cfg["name"]),
+                     "algorithmic_bytes_per_launch": nbytes["dispatch"]},
+        "gpu_launches": args.steps * 4,
+        "wall_s_timed_region": round(wall, 4),
+    }
+    if clock_info:
+        line["clocks"] = clock_info
+    if e2e:
+        line["e2e"] = {"value": round(T * world / (e2e["ms_per_step"] * 1e-3), 1), "unit": "tokens/s",
+                       "ms_per_step": round(e2e["ms_per_step"], 4),
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, inp)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush):
+    """Same step through the public API with host buffers: pinned H2D of the
+    step's inputs, the three calls, D2H of the combined output, all timed."""
+    T, H = cfg["T"], cfg["H"]
+    h_idx = torch.from_numpy(inp["topk_idx"]).pin_memory()
+    h_w = torch.from_numpy(inp["topk_weights"]).pin_memory()
+    h_x = torch.from_numpy(inp["x"].view(np.int16)).pin_memory()
+    h_out = torch.empty((T, H), dtype=torch.int16).pin_memory()
+    d_idx = torch.empty_like(h_idx, device=dev)
+    d_w = torch.empty_like(h_w, device=dev)
+    d_x = torch.empty_like(h_x, device=dev)
+    d_out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    steps = max(3, min(args.steps, 10))
+
+    def one(e0=None, e1=None):
+        if e0:
+            e0.record(stream)
+        d_idx.copy_(h_idx, non_blocking=True)
+        d_w.copy_(h_w, non_blocking=True)
+        d_x.copy_(h_x, non_blocking=True)
+        ep.layout(d_idx, d_w, cfg["E"], cfg["R"], cfg["A"], cfg["max_tokens_per_rank"], out=lay)
+        xb = d_x.view(torch.bfloat16)
+        if fp8:
+            ep.dispatch(lay, xb, cast_to_fp8=True, do_zero_padding=cfg["zero_pad"], out=recv, out_scales=recv_s)
+        else:
+            ep.dispatch(lay, xb, do_zero_padding=cfg["zero_pad"], out=recv)
+        ep.combine(lay, y, d_w, out=d_out)
+        h_out.copy_(d_out.view(torch.int16), non_blocking=True)
+        if e1:
+            e1.record(stream)
+
+    for _ in range(2):
+        flush.zero_()
+        one()
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        one(e0, e1)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    h2d = h_idx.numel() * 8 + h_w.numel() * 4 + h_x.numel() * 2
+    return {"ms_per_step": float(np.mean(ts)), "h2d": int(h2d), "d2h": int(h_out.numel() * 2)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle: the baseline leg and the reference arm
+# --------------------------------------------------------------------------
+def oracle_step_inputs(cfg, inp):
+    import oracle
+    lay = oracle.layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"],
+                        cfg["max_tokens_per_rank"])
+    y = oracle.dispatch_rows(inp["x"], lay, cfg["zero_pad"]) if not cfg["fp8"] else \
+        workload.expert_outputs(cfg, int(lay["off"][-1]))
+    return dict(inp, y=y)
+
+
+def time_oracle(cfg, inp, budget_s=10.0, min_steps=1, max_steps=None):
+    import oracle
+    full = oracle_step_inputs(cfg, inp)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.step(full, cfg)
+        n += 1
+        el = time.perf_counter() - t0
+        if (n >= min_steps and el >= budget_s) or (max_steps and n >= max_steps):
+            return n, el
+
+
+def cpu_baseline(cfg, inp):
+    n, el = time_oracle(cfg, inp, budget_s=10.0)
+    return {"value": round(cfg["T"] * n / el, 1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "%d full step(s) of the %s workload (layout, dispatch%s, combine), single-threaded C, "
+                      "%d host cores present" % (n, cfg["name"], " with cast" if cfg["fp8"] else "",
+                                                 os.cpu_count() or 0)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cfg = workload.config(args.workload)
+    inp = workload.inputs(cfg)
+    full = oracle_step_inputs(cfg, inp)
+    import oracle
+    for _ in range(args.warmup):
+        oracle.step(full, cfg)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.step(full, cfg)
+        ts.append(time.perf_counter() - t0)
+    ms = float(np.mean(ts)) * 1e3
+    v = round(cfg["T"] / (ms * 1e-3), 1)
+    return {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8-e4m3/bf16" if cfg["fp8"] else "bf16",
+            "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
+            "config": {"workload": cfg["name"], "global_batch": cfg["T"]},
+            "impl": "reference",
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": "the full %s workload per step (single-threaded C oracle)" % cfg["name"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        line = run_ours(args, rank, world, local_rank)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

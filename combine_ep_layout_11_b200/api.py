@@ -1,0 +1,197 @@
+"""Thin torch binding of the C ABI (argument marshalling only).
+
+Names follow "DeepEP 测试目标 API 系统性参考": ``layout`` derives the routing
+layout (§2.1, the V2 path that needs only topk_idx), ``dispatch`` and ``combine``
+take the layout as their handle (§2.1 / §2.2), ``cast_fp8`` is §4.2's per-token
+cast with 128-column scale blocks.  Every step runs in ``libep_b200.so`` on the
+tensors' CUDA device, on the current torch stream; torch only allocates memory.
+"""
+import ctypes
+
+import torch
+
+from . import _lib
+
+EP_OK = 0
+EP_ERR_INVALID_ARG = 1
+EP_ERR_CAPACITY = 2
+EP_ERR_BAD_EXPERT = 3
+EP_ERR_TIMEOUT = 4
+EP_ERR_CUDA = 5
+EP_ERR_UNSUPPORTED = 6
+EP_DTYPE_BF16 = 0
+EP_DTYPE_FP8_E4M3 = 1
+
+
+class EpError(RuntimeError):
+    def __init__(self, code, what):
+        msg = _lib.load().ep_status_string(code).decode()
+        super().__init__("%s: %s (status %d)" % (what, msg, code))
+        self.code = code
+
+
+def _check(code, what):
+    if code != EP_OK:
+        raise EpError(code, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def workspace_bytes(num_tokens, num_topk, num_experts, expert_alignment):
+    return int(_lib.load().ep_workspace_bytes(num_tokens, num_topk, num_experts, expert_alignment))
+
+
+def capacity_rows(num_tokens, num_topk, num_experts, expert_alignment):
+    """Receive rows that can never overflow: T*K + E*(A-1)."""
+    return int(_lib.load().ep_capacity_rows(num_tokens, num_topk, num_experts, expert_alignment))
+
+
+class Layout:
+    """The dispatch / combine handle: routing layout tensors plus the C struct.
+
+    Tensors (device): ``num_recv_tokens_per_expert`` [E], ``expert_offset`` [E+1],
+    ``pair_slot`` [T, K], ``recv_src_token`` / ``recv_weight`` /
+    ``recv_local_expert`` [capacity], ``workspace`` (bytes).
+    """
+
+    def __init__(self, num_tokens, num_topk, num_experts, num_ranks, expert_alignment, device,
+                 capacity=None, num_max_tokens_per_rank=0):
+        T, K, E, A = num_tokens, num_topk, num_experts, expert_alignment
+        if capacity is None:
+            capacity = capacity_rows(T, K, E, A)
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.num_tokens, self.num_topk, self.num_experts = T, K, E
+        self.num_ranks, self.expert_alignment = num_ranks, A
+        self.num_max_tokens_per_rank = num_max_tokens_per_rank
+        self.capacity = int(capacity)
+        self.device = dev
+        self.num_recv_tokens_per_expert = torch.empty(E, **i32)
+        self.expert_offset = torch.empty(E + 1, **i32)
+        # at least one element so the handle never carries a null pointer
+        self._pair_slot_buf = torch.empty(max(T * K, 1), **i32)
+        self.pair_slot = self._pair_slot_buf[:T * K].view(T, K)
+        n = max(self.capacity, 1)
+        self.recv_src_token = torch.empty(n, **i32)
+        self.recv_weight = torch.empty(n, dtype=torch.float32, device=dev)
+        self.recv_local_expert = torch.empty(n, **i32)
+        nbytes = workspace_bytes(T, K, E, A)
+        if nbytes == 0:
+            raise EpError(EP_ERR_INVALID_ARG, "workspace size")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        s = _lib.EpLayout()
+        s.num_recv_tokens_per_expert = self.num_recv_tokens_per_expert.data_ptr()
+        s.expert_offset = self.expert_offset.data_ptr()
+        s.pair_slot = self._pair_slot_buf.data_ptr()
+        s.recv_src_token = self.recv_src_token.data_ptr()
+        s.recv_weight = self.recv_weight.data_ptr()
+        s.recv_local_expert = self.recv_local_expert.data_ptr()
+        s.workspace = self.workspace.data_ptr()
+        s.workspace_bytes = nbytes
+        s.capacity = self.capacity
+        self.struct = s
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+    def num_recv_rows(self):
+        """Rows in use, expert_offset[E] (reads the device: synchronises)."""
+        return int(self.expert_offset[-1].item())
+
+    def rank_offsets(self):
+        """Start row of each virtual rank's receive region, [R+1] (device tensor)."""
+        El = self.num_experts // self.num_ranks
+        return self.expert_offset[::El]
+
+
+def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment=1,
+           num_max_tokens_per_rank=0, capacity=None, out=None):
+    """Compute the routing layout of ``topk_idx`` [T, K] int64 (-1 = unselected).
+
+    ``out`` may be a ``Layout`` of the same sizes to reuse its memory.
+    """
+    L = _lib.load()
+    assert topk_idx.dtype == torch.int64 and topk_idx.dim() == 2 and topk_idx.is_contiguous()
+    T, K = topk_idx.shape
+    if topk_weights is not None:
+        assert topk_weights.dtype == torch.float32 and topk_weights.shape == (T, K)
+        assert topk_weights.is_contiguous()
+    if out is not None:
+        assert (out.num_tokens, out.num_topk, out.num_experts) == (T, K, num_experts), "layout size mismatch"
+    lay = out if out is not None else Layout(T, K, num_experts, num_ranks, expert_alignment,
+                                             topk_idx.device, capacity, num_max_tokens_per_rank)
+    _check(L.ep_layout(_ptr(topk_idx), _ptr(topk_weights), T, K, num_experts, num_ranks,
+                       expert_alignment, num_max_tokens_per_rank, lay.ref(), _stream(topk_idx.device)),
+           "ep_layout")
+    return lay
+
+
+def dispatch(lay, x, x_scales=None, cast_to_fp8=False, do_zero_padding=False, out=None, out_scales=None):
+    """Scatter token rows into the receive buffer (§2.1 dispatch()).
+
+    ``x``: bf16 [T, H], or float8_e4m3fn [T, H] with ``x_scales`` fp32 [T, H/128].
+    Returns ``recv_x`` [capacity, H] (bf16, or e4m3 when the input is FP8 or
+    ``cast_to_fp8``) and, for FP8 output, ``recv_scales`` [capacity, H/128].
+    """
+    L = _lib.load()
+    assert x.dim() == 2 and x.is_contiguous() and x.shape[0] == lay.num_tokens
+    H = x.shape[1]
+    fp8_in = x.dtype == torch.float8_e4m3fn
+    assert fp8_in or x.dtype == torch.bfloat16
+    fp8_out = fp8_in or cast_to_fp8
+    cap = max(lay.capacity, 1)
+    if out is None:
+        out = torch.empty((cap, H), dtype=torch.float8_e4m3fn if fp8_out else torch.bfloat16, device=x.device)
+    if fp8_out and out_scales is None:
+        out_scales = torch.empty((cap, H // 128), dtype=torch.float32, device=x.device)
+    _check(L.ep_dispatch(lay.ref(), _ptr(x), EP_DTYPE_FP8_E4M3 if fp8_in else EP_DTYPE_BF16,
+                         _ptr(x_scales if fp8_in else None), H, int(bool(cast_to_fp8)),
+                         int(bool(do_zero_padding)), _ptr(out), _ptr(out_scales if fp8_out else None),
+                         _stream(x.device)), "ep_dispatch")
+    return (out, out_scales) if fp8_out else out
+
+
+def combine(lay, y, topk_weights=None, out=None):
+    """Weighted (or, with no weights, plain) ordered reduction back to [T, H] bf16 (§2.2)."""
+    L = _lib.load()
+    assert y.dtype == torch.bfloat16 and y.dim() == 2 and y.is_contiguous()
+    H = y.shape[1]
+    if topk_weights is not None:
+        assert topk_weights.dtype == torch.float32 and topk_weights.is_contiguous()
+    if out is None:
+        out = torch.empty((lay.num_tokens, H), dtype=torch.bfloat16, device=y.device)
+    _check(L.ep_combine(lay.ref(), _ptr(y), H, _ptr(topk_weights), _ptr(out), _stream(y.device)),
+           "ep_combine")
+    return out
+
+
+def cast_fp8(x, out=None, out_scales=None):
+    """bf16 [T, H] -> (float8_e4m3fn [T, H], fp32 scales [T, H/128]) (§4.2)."""
+    L = _lib.load()
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+    T, H = x.shape
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.float8_e4m3fn, device=x.device)
+    if out_scales is None:
+        out_scales = torch.empty((T, H // 128), dtype=torch.float32, device=x.device)
+    _check(L.ep_cast_fp8(_ptr(x), T, H, _ptr(out), _ptr(out_scales), _stream(x.device)), "ep_cast_fp8")
+    return out, out_scales
+
+
+def get_status(lay):
+    """(status code, EP_DEV_* flags) of the handle's device status word; synchronises the stream."""
+    L = _lib.load()
+    flags = ctypes.c_uint32(0)
+    code = L.ep_get_status(lay.ref(), _stream(lay.device), ctypes.byref(flags))
+    return code, flags.value
+
+
+def selftest_bounded_wait(lay, timeout_ns):
+    _check(_lib.load().ep_selftest_bounded_wait(lay.ref(), int(timeout_ns), _stream(lay.device)),
+           "ep_selftest_bounded_wait")

@@ -1,0 +1,233 @@
+// extern "C" entry points declared in include/ep_b200.h: host-side argument
+// checks, then kernel launches on the caller's stream.  No allocation, no
+// state kept between calls, no host synchronisation except ep_get_status.
+#include <limits.h>
+
+#include "ep_internal.h"
+
+namespace {
+
+constexpr uint32_t kLayoutMagic = 0x45504c31u;   // set by ep_layout on a filled handle
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int device_sms(int* sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return EP_ERR_CUDA;
+    if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return EP_ERR_CUDA;
+    return EP_OK;
+}
+
+int check_handle(const ep_layout_t* L) {
+    if (!L || L->magic != kLayoutMagic || !L->workspace || !L->pair_slot) return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+ep::WsHeader* header(const ep_layout_t* L) { return reinterpret_cast<ep::WsHeader*>(L->workspace); }
+
+}  // namespace
+
+extern "C" {
+
+int ep_version(void) { return EP_B200_VERSION; }
+
+const char* ep_status_string(int status) {
+    switch (status) {
+        case EP_OK: return "ok";
+        case EP_ERR_INVALID_ARG: return "invalid argument";
+        case EP_ERR_CAPACITY: return "capacity exceeded";
+        case EP_ERR_BAD_EXPERT: return "expert id outside [-1, num_experts)";
+        case EP_ERR_TIMEOUT: return "bounded wait ran out";
+        case EP_ERR_CUDA: return "CUDA error";
+        case EP_ERR_UNSUPPORTED: return "unsupported size";
+        default: return "unknown status";
+    }
+}
+
+size_t ep_workspace_bytes(int num_tokens, int num_topk, int num_experts, int expert_alignment) {
+    if (num_tokens < 0 || num_topk < 1 || num_experts < 1 || expert_alignment < 1) return 0;
+    return ep::ws_layout(num_tokens, num_topk, num_experts, expert_alignment).total;
+}
+
+int64_t ep_capacity_rows(int num_tokens, int num_topk, int num_experts, int expert_alignment) {
+    if (num_tokens < 0 || num_topk < 1 || num_experts < 1 || expert_alignment < 1) return 0;
+    return (int64_t)num_tokens * num_topk + (int64_t)num_experts * (expert_alignment - 1);
+}
+
+int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
+              int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
+              ep_layout_t* layout, void* stream) {
+    const int T = num_tokens, K = num_topk, E = num_experts, R = num_ranks, A = expert_alignment;
+    if (!layout) return EP_ERR_INVALID_ARG;
+    if (T < 0 || K < 1 || E < 1 || R < 1 || A < 1 || num_max_tokens_per_rank < 0) return EP_ERR_INVALID_ARG;
+    if (K > EP_MAX_TOPK || E > EP_MAX_EXPERTS) return EP_ERR_UNSUPPORTED;
+    if (E % R != 0 || T % R != 0) return EP_ERR_INVALID_ARG;
+    if ((int64_t)T * K + (int64_t)E * (A - 1) > INT_MAX) return EP_ERR_UNSUPPORTED;
+    if (layout->capacity < 0) return EP_ERR_INVALID_ARG;
+    if (layout->capacity > INT_MAX) return EP_ERR_UNSUPPORTED;
+    if (num_max_tokens_per_rank > 0 && T / R > num_max_tokens_per_rank) return EP_ERR_CAPACITY;
+    if ((T > 0 && !topk_idx) || !layout->num_recv_tokens_per_expert || !layout->expert_offset ||
+        !layout->pair_slot || !layout->recv_src_token || !layout->recv_weight || !layout->recv_local_expert ||
+        !layout->workspace)
+        return EP_ERR_INVALID_ARG;
+    if (!aligned(topk_idx, 8) || !aligned(topk_weights, 4) || !aligned(layout->num_recv_tokens_per_expert, 4) ||
+        !aligned(layout->expert_offset, 4) || !aligned(layout->pair_slot, 4) ||
+        !aligned(layout->recv_src_token, 4) || !aligned(layout->recv_weight, 4) ||
+        !aligned(layout->recv_local_expert, 4) || !aligned(layout->workspace, 256))
+        return EP_ERR_INVALID_ARG;
+    const ep::WsLayout ws = ep::ws_layout(T, K, E, A);
+    if (layout->workspace_bytes < ws.total) return EP_ERR_INVALID_ARG;
+
+    layout->num_tokens = T;
+    layout->num_topk = K;
+    layout->num_experts = E;
+    layout->num_ranks = R;
+    layout->expert_alignment = A;
+    layout->num_max_tokens_per_rank = num_max_tokens_per_rank;
+    layout->magic = kLayoutMagic;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t* wsb = reinterpret_cast<uint8_t*>(layout->workspace);
+    if (cudaMemsetAsync(wsb, 0, sizeof(ep::WsHeader), s) != cudaSuccess) return EP_ERR_CUDA;
+    if (T == 0) {
+        if (cudaMemsetAsync(layout->num_recv_tokens_per_expert, 0, (size_t)E * 4, s) != cudaSuccess ||
+            cudaMemsetAsync(layout->expert_offset, 0, (size_t)(E + 1) * 4, s) != cudaSuccess)
+            return EP_ERR_CUDA;
+        return EP_OK;
+    }
+    const ep::Chunking ch = ep::chunking(T, K, E);
+    ep::LayoutArgs a;
+    a.topk_idx = topk_idx;
+    a.topk_weights = topk_weights;
+    a.T = T; a.K = K; a.E = E; a.R = R; a.A = A;
+    a.C = ch.num_chunks;
+    a.CT = ch.chunk_tokens;
+    a.capacity = layout->capacity;
+    a.cnt = layout->num_recv_tokens_per_expert;
+    a.off = layout->expert_offset;
+    a.pair_slot = layout->pair_slot;
+    a.recv_src = layout->recv_src_token;
+    a.recv_w = layout->recv_weight;
+    a.recv_lexp = layout->recv_local_expert;
+    a.hdr = reinterpret_cast<ep::WsHeader*>(wsb);
+    a.table = reinterpret_cast<int32_t*>(wsb + ws.table_off);
+    a.padpre = reinterpret_cast<int32_t*>(wsb + ws.padpre_off);
+    a.pad_rows = reinterpret_cast<int32_t*>(wsb + ws.padrows_off);
+    return ep::launch_layout(a, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales, int hidden,
+                int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales, void* stream) {
+    int rc = check_handle(layout);
+    if (rc != EP_OK) return rc;
+    const int H = hidden, T = layout->num_tokens;
+    if (H <= 0 || (x_dtype != EP_DTYPE_BF16 && x_dtype != EP_DTYPE_FP8_E4M3)) return EP_ERR_INVALID_ARG;
+    if (cast_to_fp8 && x_dtype != EP_DTYPE_BF16) return EP_ERR_INVALID_ARG;
+    const bool fp8_in = x_dtype == EP_DTYPE_FP8_E4M3;
+    const bool fp8_out = fp8_in || cast_to_fp8;
+    if (H % 8 != 0 || (fp8_out && H % 128 != 0)) return EP_ERR_INVALID_ARG;
+    if ((T > 0 && !x) || !recv_x || (fp8_out && !recv_scales) || (fp8_in && T > 0 && !x_scales))
+        return EP_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(x_scales, 4) || !aligned(recv_scales, 16))
+        return EP_ERR_INVALID_ARG;
+    if (cast_to_fp8 && H > 16384) return EP_ERR_UNSUPPORTED;
+    if (T == 0) return EP_OK;   // no tokens, no pairs, no padding rows
+
+    const uint8_t* wsb = reinterpret_cast<const uint8_t*>(layout->workspace);
+    const ep::WsLayout ws = ep::ws_layout(T, layout->num_topk, layout->num_experts, layout->expert_alignment);
+    ep::DispatchArgs a;
+    a.x = reinterpret_cast<const uint8_t*>(x);
+    a.x_scales = fp8_in ? x_scales : nullptr;
+    a.recv = reinterpret_cast<uint8_t*>(recv_x);
+    a.recv_scales = fp8_out ? recv_scales : nullptr;
+    a.pair_slot = layout->pair_slot;
+    a.hdr = reinterpret_cast<const ep::WsHeader*>(wsb);
+    a.pad_rows = reinterpret_cast<const int32_t*>(wsb + ws.padrows_off);
+    a.status_hdr = header(layout);
+    a.T = T;
+    a.K = layout->num_topk;
+    a.H = H;
+    a.capacity = layout->capacity;
+    a.nb = fp8_out ? H / 128 : 0;
+    a.zero_pad = do_zero_padding ? 1 : 0;
+    if ((rc = device_sms(&a.sms)) != EP_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t err = cast_to_fp8 ? ep::launch_dispatch_cast(a, s) : ep::launch_dispatch_copy(a, fp8_in ? 1 : 2, s);
+    return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float* topk_weights, void* out,
+               void* stream) {
+    int rc = check_handle(layout);
+    if (rc != EP_OK) return rc;
+    const int H = hidden, T = layout->num_tokens;
+    if (H <= 0 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (T > 0 && (!y || !out)) return EP_ERR_INVALID_ARG;
+    if (!aligned(y, 16) || !aligned(out, 16) || !aligned(topk_weights, 4)) return EP_ERR_INVALID_ARG;
+    if (T == 0) return EP_OK;
+    ep::CombineArgs a;
+    a.y = reinterpret_cast<const uint16_t*>(y);
+    a.pair_slot = layout->pair_slot;
+    a.w = topk_weights;
+    a.out = reinterpret_cast<uint16_t*>(out);
+    a.T = T;
+    a.K = layout->num_topk;
+    a.H = H;
+    a.capacity = layout->capacity;
+    if ((rc = device_sms(&a.sms)) != EP_OK) return rc;
+    return ep::launch_combine(a, (cudaStream_t)stream) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+int ep_cast_fp8(const void* x, int num_tokens, int hidden, void* x_fp8, float* scales, void* stream) {
+    const int T = num_tokens, H = hidden;
+    if (T < 0 || H <= 0 || H % 128 != 0) return EP_ERR_INVALID_ARG;
+    if (H > 16384) return EP_ERR_UNSUPPORTED;
+    if (T > 0 && (!x || !x_fp8 || !scales)) return EP_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(x_fp8, 16) || !aligned(scales, 16)) return EP_ERR_INVALID_ARG;
+    if (T == 0) return EP_OK;
+    ep::DispatchArgs a;
+    a.x = reinterpret_cast<const uint8_t*>(x);
+    a.x_scales = nullptr;
+    a.recv = reinterpret_cast<uint8_t*>(x_fp8);
+    a.recv_scales = scales;
+    a.pair_slot = nullptr;   // row t -> row t
+    a.hdr = nullptr;
+    a.pad_rows = nullptr;
+    a.status_hdr = nullptr;
+    a.T = T;
+    a.K = 1;
+    a.H = H;
+    a.capacity = T;
+    a.nb = H / 128;
+    a.zero_pad = 0;
+    int rc = device_sms(&a.sms);
+    if (rc != EP_OK) return rc;
+    return ep::launch_dispatch_cast(a, (cudaStream_t)stream) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+int ep_get_status(const ep_layout_t* layout, void* stream, uint32_t* device_flags) {
+    int rc = check_handle(layout);
+    if (rc != EP_OK) return rc;
+    if (!device_flags) return EP_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t flags = 0;
+    if (cudaMemcpyAsync(&flags, &header(layout)->status, sizeof(flags), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return EP_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return EP_ERR_CUDA;
+    *device_flags = flags;
+    if (flags & EP_DEV_TIMEOUT) return EP_ERR_TIMEOUT;
+    if (flags & EP_DEV_BAD_EXPERT) return EP_ERR_BAD_EXPERT;
+    if (flags & EP_DEV_CAPACITY) return EP_ERR_CAPACITY;
+    return EP_OK;
+}
+
+int ep_selftest_bounded_wait(const ep_layout_t* layout, uint64_t timeout_ns, void* stream) {
+    int rc = check_handle(layout);
+    if (rc != EP_OK) return rc;
+    if (timeout_ns > 1000000000ull) return EP_ERR_INVALID_ARG;
+    return ep::launch_selftest_wait(header(layout), timeout_ns, (cudaStream_t)stream) == cudaSuccess
+               ? EP_OK
+               : EP_ERR_CUDA;
+}
+
+}  // extern "C"

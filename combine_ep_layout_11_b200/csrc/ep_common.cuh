@@ -1,0 +1,186 @@
+// Device helpers shared by the dispatch / combine kernels (sm_100a only):
+// inline-PTX wrappers for shared-memory barriers and TMA bulk copies, the
+// bounded wait every kernel uses, and the workspace layout that ep_layout
+// writes and ep_dispatch reads.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ep_b200.h"
+
+namespace ep {
+
+// ---------------------------------------------------------------------------
+// Device status word bits (mirrors EP_DEV_* in the public header)
+// ---------------------------------------------------------------------------
+constexpr uint32_t kDevBadExpert = EP_DEV_BAD_EXPERT;
+constexpr uint32_t kDevCapacity = EP_DEV_CAPACITY;
+constexpr uint32_t kDevTimeout = EP_DEV_TIMEOUT;
+
+// A wait on a barrier that hardware completes (a TMA load landing in shared
+// memory) gives up after this long and reports EP_DEV_TIMEOUT instead of
+// spinning forever.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// ---------------------------------------------------------------------------
+// Workspace: [0, 256) header words, then the (chunk x expert) count table,
+// the padding prefix and the list of padding rows.
+// ---------------------------------------------------------------------------
+struct WsHeader {
+    uint32_t status;     // EP_DEV_* bits
+    uint32_t ticket;     // arrival counter of the counting kernel's CTAs
+    int32_t num_pad;     // padding rows (expert_offset[E] - pairs)
+    int32_t pad0;
+};
+
+struct Chunking {
+    int num_chunks;       // C: CTAs of the counting / slot kernels
+    int chunk_tokens;     // CT: tokens per chunk
+};
+
+// Chunks of whole tokens, about 256 pairs each, at most 128 chunks, and at most
+// 32768 (chunk, expert) cells so that the whole count table fits in one CTA's
+// shared memory for the scan.
+inline Chunking chunking(int T, int K, int E) {
+    Chunking c{0, 0};
+    if (T <= 0) return c;
+    int64_t pairs = (int64_t)T * K;
+    int64_t cmax = 32768 / E;
+    if (cmax < 1) cmax = 1;
+    int64_t n = (pairs + 255) / 256;
+    if (n > 128) n = 128;
+    if (n > cmax) n = cmax;
+    if (n < 1) n = 1;
+    int64_t ct = ((int64_t)T + n - 1) / n;
+    c.chunk_tokens = (int)ct;
+    c.num_chunks = (int)(((int64_t)T + ct - 1) / ct);
+    return c;
+}
+
+struct WsLayout {
+    size_t table_off;    // int32 [C][E]: per-chunk counts, then per-chunk row bases
+    size_t padpre_off;   // int32 [E+1]: exclusive prefix of padding rows per expert
+    size_t padrows_off;  // int32 [E*(A-1)]: receive row of every padding row
+    size_t total;
+};
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WsLayout ws_layout(int T, int K, int E, int A) {
+    Chunking ch = chunking(T, K, E);
+    WsLayout w;
+    w.table_off = 256;
+    w.padpre_off = round_up(w.table_off + (size_t)ch.num_chunks * E * 4, 256);
+    w.padrows_off = round_up(w.padpre_off + ((size_t)E + 1) * 4, 256);
+    w.total = round_up(w.padrows_off + (size_t)E * (size_t)(A > 1 ? A - 1 : 0) * 4 + 4, 256);
+    return w;
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Make barrier initialisation and generic-proxy shared-memory writes visible
+// to the async proxy (the TMA engine).
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        " .reg .pred p;\n"
+        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the barrier phase with the given parity to complete; false if it
+// has not completed within limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
+// TMA bulk copy global -> shared, completion counted in bytes on `bar`.
+// (No multicast: a plain CTA-local copy.)
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// TMA bulk copy shared -> global, tracked in this thread's bulk async-group.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+                 "r"(smem_u32(smem_src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N of this thread's committed bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until at most N of this thread's committed bulk groups are incomplete.
+template <int N>
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// 16-byte streaming load that does not allocate in L1 (each row is read once).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+}  // namespace ep

@@ -1,0 +1,68 @@
+// Internal launch interface between the C ABI (ep_abi.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep_common.cuh"
+
+namespace ep {
+
+struct LayoutArgs {
+    const int64_t* topk_idx;
+    const float* topk_weights;  // nullable
+    int T, K, E, R, A;
+    int C, CT;                  // chunking
+    int64_t capacity;
+    int32_t* cnt;
+    int32_t* off;
+    int32_t* pair_slot;
+    int32_t* recv_src;
+    float* recv_w;
+    int32_t* recv_lexp;
+    WsHeader* hdr;
+    int32_t* table;
+    int32_t* padpre;
+    int32_t* pad_rows;
+};
+
+// Two kernels: per-chunk counting (its last CTA scans the count table into
+// aligned offsets and per-chunk row bases) and slot assignment.
+cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t s);
+
+struct DispatchArgs {
+    const uint8_t* x;          // token rows, row_bytes each (bf16 or e4m3)
+    const float* x_scales;     // [T][nb] for e4m3 input
+    uint8_t* recv;             // receive rows of the output type
+    float* recv_scales;        // [capacity][nb] for e4m3 output
+    const int32_t* pair_slot;  // [T*K]; nullptr: row t goes to row t (plain cast)
+    const WsHeader* hdr;       // num_pad
+    const int32_t* pad_rows;
+    WsHeader* status_hdr;      // status word
+    int T, K, H;
+    int64_t capacity;
+    int nb;                    // scales per row (H/128) when FP8 is involved
+    int zero_pad;
+    int sms;
+};
+
+// bf16 -> bf16 or e4m3 -> e4m3 row scatter through TMA bulk copies.
+cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStream_t s);
+// bf16 -> e4m3 scatter with the per-128-column cast fused in.
+cudaError_t launch_dispatch_cast(const DispatchArgs& a, cudaStream_t s);
+
+struct CombineArgs {
+    const uint16_t* y;         // bf16 [capacity][H]
+    const int32_t* pair_slot;  // [T*K]
+    const float* w;            // [T*K] or nullptr
+    uint16_t* out;             // bf16 [T][H]
+    int T, K, H;
+    int64_t capacity;
+    int sms;
+};
+
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+cudaError_t launch_selftest_wait(WsHeader* hdr, uint64_t timeout_ns, cudaStream_t s);
+
+}  // namespace ep

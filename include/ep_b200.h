@@ -1,0 +1,233 @@
+/*
+ * ep_b200.h - C ABI of the B200 (sm_100a) MoE expert-parallel dispatch /
+ * combine library, DeepEP style, with R virtual ranks held in one GPU's HBM.
+ *
+ * The operations follow "DeepEP 测试目标 API 系统性参考" (the DeepEP test-target
+ * API reference):
+ *   ep_layout    §2.1 dispatch(): the routing layout V2 derives from topk_idx
+ *                (-1 = unselected), expert_alignment, the expand layout
+ *                (do_expand: one receive row per (token, expert) pair), the
+ *                handle; §3.1: the per-expert receive counts V1 returns.
+ *   ep_dispatch  §2.1 dispatch(): rows to the owning ranks' receive regions,
+ *                same type as the input ((fp8, scales) stays (fp8, scales)),
+ *                do_zero_padding; §4.2 math.py for the fused FP8 cast.
+ *   ep_combine   §2.2 combine(): weighted reduction back to [T, hidden] bf16 in
+ *                the order the handle records; §3.2: no weights = plain sum;
+ *                §4.1 refs.py ordered_accumulate: one fixed order, so results
+ *                are bitwise reproducible.
+ *   ep_cast_fp8  §4.2 math.py per_token_cast_to_fp8, with one fp32 scale per
+ *                128-column block of a token row.
+ * The placement also matches the last stages of the Ascend full-mesh dispatch
+ * on the "URMA" tag page (count reconciliation, prefix-sum placement, reorder).
+ *
+ * Conventions for every entry point
+ *   - Memory: every array is allocated by the caller; the library never
+ *     allocates or frees memory and keeps no state between calls.  "device"
+ *     means a pointer to memory of the current CUDA device.
+ *   - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *     Every call only enqueues work on that stream and returns; results are
+ *     ready when the stream reaches them.  Nothing synchronises the host except
+ *     ep_get_status.
+ *   - Errors: host-side argument checks return a status before anything is
+ *     enqueued (EP_ERR_INVALID_ARG, EP_ERR_CAPACITY, EP_ERR_UNSUPPORTED); a
+ *     failed launch returns EP_ERR_CUDA.  Problems only the device can see
+ *     (a bad expert id, too many receive rows, a bounded wait that ran out) set
+ *     bits in the layout's device status word, read by ep_get_status; the
+ *     kernels then skip the affected writes, never write out of bounds, never
+ *     trap and never spin without limit.
+ *   - Precision: integer and byte work is exact; combine accumulates in fp32 in
+ *     ascending k with separately rounded multiply and add, then rounds to bf16
+ *     to nearest even, so results are bitwise reproducible run to run and
+ *     independent of how many tokens share a call.
+ *
+ * Layout of the receive buffers (expand layout): expert e's rows are
+ * [off[e], off[e] + cnt[e]) holding its (token, k) pairs in token-major,
+ * k-minor order, followed by align(cnt[e], A) - cnt[e] padding rows;
+ * off[e] = sum over e' < e of align(cnt[e'], A).  Virtual rank r owns experts
+ * [r*E/R, (r+1)*E/R), so its region is [off[r*E/R], off[(r+1)*E/R]) and rows
+ * are ordered by (destination rank, local expert, source token).  Token t
+ * belongs to source rank t / (T/R).
+ */
+#ifndef EP_B200_H
+#define EP_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EP_B200_VERSION 1
+
+/* Host return codes. */
+#define EP_OK 0
+#define EP_ERR_INVALID_ARG 1   /* null / misaligned pointer, bad size or shape   */
+#define EP_ERR_CAPACITY 2      /* receive rows or tokens per rank above a limit  */
+#define EP_ERR_BAD_EXPERT 3    /* (device) an expert id outside [-1, E)          */
+#define EP_ERR_TIMEOUT 4       /* (device) a bounded wait ran out                */
+#define EP_ERR_CUDA 5          /* a CUDA call failed                             */
+#define EP_ERR_UNSUPPORTED 6   /* valid arguments outside the supported range    */
+
+/* Bits of the device status word (see ep_get_status). */
+#define EP_DEV_BAD_EXPERT 0x1u
+#define EP_DEV_CAPACITY 0x2u
+#define EP_DEV_TIMEOUT 0x4u
+
+/* Element types of token rows. */
+#define EP_DTYPE_BF16 0
+#define EP_DTYPE_FP8_E4M3 1
+
+/* Supported ranges (EP_ERR_UNSUPPORTED beyond them). */
+#define EP_MAX_TOPK 32
+#define EP_MAX_EXPERTS 4096
+
+/*
+ * The handle ("handle" / EPHandle in §2.1 and §2.2): the routing layout of one
+ * batch, reused as is by ep_dispatch and ep_combine (a cached layout).
+ *
+ * The caller fills the pointer fields and `capacity` and `workspace_bytes`
+ * before ep_layout; ep_layout fills the shape fields.  All arrays are device
+ * memory owned by the caller and must stay alive while work that uses the
+ * handle is pending.
+ *   num_recv_tokens_per_expert [E]     int32  cnt[e]: pairs that chose expert e
+ *   expert_offset              [E+1]   int32  aligned exclusive prefix of cnt;
+ *                                             expert_offset[E] = rows used (Np)
+ *   pair_slot                  [T*K]   int32  receive row of pair (t, k), -1 if
+ *                                             topk_idx[t, k] == -1
+ *   recv_src_token             [capacity] int32  source token of each row, -1 on
+ *                                             padding rows
+ *   recv_weight                [capacity] fp32   topk weight of each row (1 when
+ *                                             ep_layout got no weights), 0 on padding
+ *   recv_local_expert          [capacity] int32  expert id local to the
+ *                                             destination rank (e mod E/R), -1 on padding
+ *   workspace                  ep_workspace_bytes() bytes, 256-byte aligned;
+ *                              holds the device status word and scan scratch.
+ * Rows at and beyond expert_offset[E] are not written by ep_layout.
+ */
+typedef struct ep_layout_t {
+    int32_t* num_recv_tokens_per_expert;
+    int32_t* expert_offset;
+    int32_t* pair_slot;
+    int32_t* recv_src_token;
+    float* recv_weight;
+    int32_t* recv_local_expert;
+    void* workspace;
+    uint64_t workspace_bytes;
+    int64_t capacity;
+    /* filled by ep_layout */
+    int32_t num_tokens;
+    int32_t num_topk;
+    int32_t num_experts;
+    int32_t num_ranks;
+    int32_t expert_alignment;
+    int32_t num_max_tokens_per_rank;
+    uint32_t magic;
+    uint32_t reserved;
+} ep_layout_t;
+
+/* Bytes of workspace ep_layout needs for these sizes (a pure host function). */
+size_t ep_workspace_bytes(int num_tokens, int num_topk, int num_experts, int expert_alignment);
+
+/* Worst-case receive rows: T*K + E*(A-1); a capacity of this many rows can
+ * never overflow (a pure host function). */
+int64_t ep_capacity_rows(int num_tokens, int num_topk, int num_experts, int expert_alignment);
+
+/*
+ * Routing layout (§2.1: V2 derives the layout from topk_idx; §3.1: the
+ * per-expert receive counts).
+ *   topk_idx      device int64 [T, K] row-major; -1 = unselected; NULL only if T == 0
+ *   topk_weights  device fp32 [T, K] or NULL (then recv_weight = 1 on real rows)
+ *   num_tokens T >= 0 with T % R == 0; num_topk 1 <= K <= EP_MAX_TOPK;
+ *   num_experts 1 <= E <= EP_MAX_EXPERTS with E % R == 0; num_ranks R >= 1;
+ *   expert_alignment A >= 1;
+ *   num_max_tokens_per_rank  0 = no limit; else T/R must not exceed it
+ *                             (EP_ERR_CAPACITY), as §3.3 requires of the
+ *                             per-rank dispatch budget;
+ *   layout        in: pointers, capacity, workspace; out: shape fields.
+ * Device-side: an id outside [-1, E) sets EP_DEV_BAD_EXPERT and is treated as
+ * -1; more than `capacity` rows sets EP_DEV_CAPACITY and rows past capacity are
+ * not written.  Clears the device status word first.  Deterministic: the same
+ * input gives the same bytes on every call.
+ */
+int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
+              int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
+              ep_layout_t* layout, void* stream);
+
+/*
+ * Dispatch (§2.1): for every selected pair (t, k), receive row
+ * pair_slot[t, k] := token row t.
+ *   x            device, 16-byte aligned: bf16 [T, H] if x_dtype == EP_DTYPE_BF16,
+ *                e4m3 bytes [T, H] if x_dtype == EP_DTYPE_FP8_E4M3
+ *   x_scales     device fp32 [T, H/128] for FP8 input, else ignored
+ *   hidden H     > 0; H % 8 == 0 for bf16, H % 128 == 0 whenever FP8 is involved
+ *   cast_to_fp8  1: bf16 input is cast on the way (§4.2, per 128-column block,
+ *                the same bytes ep_cast_fp8 writes) and the receive rows are FP8
+ *   do_zero_padding  1: the alignment padding rows (and their scales) are zeroed;
+ *                0: they are left untouched
+ *   recv_x       device, 16-byte aligned: [capacity, H] of the output type
+ *   recv_scales  device fp32 [capacity, H/128] when the output is FP8, else ignored
+ * Rows that no pair selects and that are not padding are left untouched.
+ */
+int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales,
+                int hidden, int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales,
+                void* stream);
+
+/*
+ * Combine (§2.2 weighted; §3.2 unweighted when topk_weights is NULL; §4.1
+ * ordered accumulation):
+ *   out[t] = bf16_rne( sum over k = 0..K-1 with pair_slot[t, k] >= 0 of
+ *                      w[t, k] * float(y[pair_slot[t, k]]) )
+ * accumulated in fp32 in ascending k from +0, each step one rounded product and
+ * one rounded sum.  A token with no selected entry gives a zero row.
+ *   y            device bf16 [capacity, H], 16-byte aligned: expert outputs in
+ *                receive order; padding rows are never read
+ *   hidden H     > 0, H % 8 == 0
+ *   topk_weights device fp32 [T, K] or NULL (unit weights)
+ *   out          device bf16 [T, H], 16-byte aligned
+ */
+int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float* topk_weights,
+               void* out, void* stream);
+
+/*
+ * FP8 cast (§4.2 per_token_cast_to_fp8 with 128-column blocks): for token t
+ * and block b, amax = max |x| over the block (clamped below at 1e-4),
+ * s = amax / 448 (fp32 division), q = e4m3(x / s) with an fp32 division,
+ * round-to-nearest-even and saturation to +-448; scales[t, b] = s.
+ * Dequantisation is float(q) * s.
+ *   x       device bf16 [T, H], 16-byte aligned, H % 128 == 0
+ *   x_fp8   device e4m3 [T, H], 16-byte aligned
+ *   scales  device fp32 [T, H/128]
+ */
+int ep_cast_fp8(const void* x, int num_tokens, int hidden, void* x_fp8, float* scales,
+                void* stream);
+
+/*
+ * Synchronises `stream`, then reads the layout's device status word into
+ * *device_flags (EP_DEV_* bits, 0 = no device-side error since the last
+ * ep_layout on this handle).  Returns EP_OK when the word is 0, else
+ * EP_ERR_TIMEOUT, EP_ERR_BAD_EXPERT or EP_ERR_CAPACITY (in that priority), or
+ * EP_ERR_CUDA if the synchronisation or the read failed.
+ */
+int ep_get_status(const ep_layout_t* layout, void* stream, uint32_t* device_flags);
+
+/*
+ * Self-test of the bounded wait every kernel uses: launches one CTA that waits
+ * on a shared-memory barrier nothing will complete, with a limit of
+ * `timeout_ns` (at most 10^9), sets EP_DEV_TIMEOUT in the layout's status word
+ * and returns.  Lets a test check on a GPU that a wait which runs out reports an
+ * error instead of hanging.
+ */
+int ep_selftest_bounded_wait(const ep_layout_t* layout, uint64_t timeout_ns, void* stream);
+
+/* Static description of a status code. */
+const char* ep_status_string(int status);
+
+/* EP_B200_VERSION of the built library. */
+int ep_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_B200_H */

@@ -1,0 +1,134 @@
+"""CPU checks of the C ABI: the library builds and loads, exports every symbol
+include/ep_b200.h declares, and its host-side checks reject bad arguments
+before anything is enqueued (no GPU needed; no compute call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ep_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from combine_ep_layout_11_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(ep_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert {"ep_layout", "ep_dispatch", "ep_combine", "ep_cast_fp8", "ep_workspace_bytes",
+            "ep_capacity_rows", "ep_get_status", "ep_status_string"} <= set(names)
+
+
+def test_every_declared_symbol_is_exported_and_bound(lib):
+    from combine_ep_layout_11_b200 import _lib
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, name
+    assert set(_lib.SIGNATURES) == set(declared_functions())
+
+
+def test_struct_size_matches_header(lib):
+    from combine_ep_layout_11_b200 import _lib
+    # 7 pointers, u64, i64, 6 x i32, 2 x u32
+    assert ctypes.sizeof(_lib.EpLayout) == 7 * 8 + 8 + 8 + 6 * 4 + 2 * 4
+
+
+def test_pure_host_functions(lib):
+    assert lib.ep_version() == 1
+    assert lib.ep_capacity_rows(4096, 8, 256, 128) == 4096 * 8 + 256 * 127
+    assert lib.ep_capacity_rows(128, 4, 16, 1) == 512
+    ws = lib.ep_workspace_bytes(4096, 8, 256, 128)
+    assert ws % 256 == 0 and ws >= 256 + 128 * 256 * 4 + 257 * 4 + 256 * 127 * 4
+    assert lib.ep_workspace_bytes(-1, 8, 256, 1) == 0
+    assert lib.ep_status_string(0) == b"ok"
+    assert lib.ep_status_string(4) == b"bounded wait ran out"
+
+
+def _handle(ws_bytes=1 << 20, magic=0):
+    from combine_ep_layout_11_b200 import _lib
+    s = _lib.EpLayout()
+    fake = 0x10000   # never dereferenced: the checks below fail before any CUDA call
+    for f in ("num_recv_tokens_per_expert", "expert_offset", "pair_slot", "recv_src_token",
+              "recv_weight", "recv_local_expert", "workspace"):
+        setattr(s, f, fake)
+    s.workspace_bytes = ws_bytes
+    s.capacity = 1000
+    s.magic = magic
+    return s
+
+
+@pytest.mark.parametrize("T,K,E,R,A,limit,expect", [
+    (8, 2, 8, 3, 1, 0, 1),       # E % R
+    (9, 2, 8, 2, 1, 0, 1),       # T % R
+    (8, 0, 8, 2, 1, 0, 1),       # K < 1
+    (8, 33, 8, 2, 1, 0, 6),      # K above EP_MAX_TOPK
+    (8, 2, 5000, 1, 1, 0, 6),    # E above EP_MAX_EXPERTS
+    (8, 2, 8, 2, 0, 0, 1),       # A < 1
+    (256, 2, 8, 2, 1, 127, 2),   # tokens per rank above the limit
+    (-1, 2, 8, 1, 1, 0, 1),      # T < 0
+])
+def test_layout_host_checks(lib, T, K, E, R, A, limit, expect):
+    s = _handle()
+    rc = lib.ep_layout(ctypes.c_void_p(0x10000), None, T, K, E, R, A, limit, ctypes.byref(s), None)
+    assert rc == expect
+
+
+def test_layout_rejects_small_or_misaligned_workspace(lib):
+    s = _handle(ws_bytes=64)
+    assert lib.ep_layout(ctypes.c_void_p(0x10000), None, 8, 2, 8, 2, 1, 0, ctypes.byref(s), None) == 1
+    s = _handle()
+    s.workspace = 0x10010
+    assert lib.ep_layout(ctypes.c_void_p(0x10000), None, 8, 2, 8, 2, 1, 0, ctypes.byref(s), None) == 1
+    s = _handle()
+    assert lib.ep_layout(None, None, 8, 2, 8, 2, 1, 0, ctypes.byref(s), None) == 1   # null topk_idx
+    assert lib.ep_layout(ctypes.c_void_p(0x10000), None, 8, 2, 8, 2, 1, 0, None, None) == 1
+
+
+def test_dispatch_combine_host_checks(lib):
+    s = _handle()                        # not filled by ep_layout: rejected
+    p = ctypes.c_void_p(0x10000)
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 256, 0, 0, p, None, None) == 1
+    assert lib.ep_combine(ctypes.byref(s), p, 256, None, p, None) == 1
+    s = _handle(magic=0x45504C31)        # a handle as ep_layout leaves it
+    s.num_tokens, s.num_topk, s.num_experts, s.num_ranks, s.expert_alignment = 8, 2, 8, 2, 1
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 100, 0, 0, p, None, None) == 1      # H % 8
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 136, 1, 0, p, p, None) == 1         # FP8: H % 128
+    assert lib.ep_dispatch(ctypes.byref(s), p, 1, None, 256, 0, 0, p, p, None) == 1         # fp8 in, no scales
+    assert lib.ep_dispatch(ctypes.byref(s), p, 1, p, 256, 1, 0, p, p, None) == 1            # cast of fp8 input
+    assert lib.ep_dispatch(ctypes.byref(s), ctypes.c_void_p(0x10008), 0, None, 256, 0, 0, p, None, None) == 1
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 32768, 1, 0, p, p, None) == 6       # cast row too large
+    assert lib.ep_combine(ctypes.byref(s), p, 100, None, p, None) == 1                      # H % 8
+    assert lib.ep_combine(ctypes.byref(s), p, 256, None, ctypes.c_void_p(0x10004), None) == 1
+    assert lib.ep_cast_fp8(p, 8, 100, p, p, None) == 1
+    assert lib.ep_cast_fp8(p, 8, 32768, p, p, None) == 6
+    flags = ctypes.c_uint32(0)
+    assert lib.ep_get_status(ctypes.byref(s), None, None) == 1
+    assert lib.ep_selftest_bounded_wait(ctypes.byref(s), 2_000_000_000, None) == 1
+
+
+def test_product_path_has_no_cpu_fallback():
+    """The package never imports the oracle and fails loudly without its library."""
+    pkg = os.path.join(ROOT, "combine_ep_layout_11_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            src = open(os.path.join(pkg, fn)).read()
+            assert "oracle" not in src and "workload" not in src, fn
+    import combine_ep_layout_11_b200._lib as L
+    saved = L._LIB_PATH, L._lib
+    try:
+        L._LIB_PATH, L._lib = "/nonexistent/libep_b200.so", None
+        with pytest.raises(ImportError):
+            L.load()
+    finally:
+        L._LIB_PATH, L._lib = saved

@@ -1,0 +1,222 @@
+"""Edge cases, device-side error reporting, determinism and batch invariance
+on the GPU, through the C ABI.
+
+Error reporting follows the library's contract: bad expert ids and receive
+overflow are reported in the device status word, never by a fault; every wait
+is bounded (the self-test makes one run out on purpose and checks the status).
+Batch invariance follows the pattern of the SGLang DeepGEMM batch-invariance
+test (rows of a batch computed alone and inside larger batches must match with
+atol = rtol = 0).
+"""
+import hashlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workload
+from gpu_util import DEV, bf16_bits, check_layout, f32_bits, fp8_bits, to_dev, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ep():
+    from combine_ep_layout_11_b200 import build
+    build.build()
+    import combine_ep_layout_11_b200 as m
+    return m
+
+
+def _full(ep, idx, w, x, E, R, A, zero_pad=True, fp8=False):
+    ref = oracle.layout(idx, w, E, R, A)
+    lay = ep.layout(to_dev(idx), None if w is None else to_dev(w), E, R, A)
+    xd = to_dev_bf16(x)
+    res = ep.dispatch(lay, xd, cast_to_fp8=fp8, do_zero_padding=zero_pad)
+    torch.cuda.synchronize()
+    assert ep.get_status(lay) == (ep.EP_OK, 0)
+    Np = check_layout(lay, ref)
+    if fp8:
+        rq, rs = oracle.cast_fp8(x)
+        assert np.array_equal(fp8_bits(res[0][:Np]), oracle.dispatch_rows(rq, ref, zero_pad)[:Np])
+        assert np.array_equal(f32_bits(res[1][:Np]), oracle.dispatch_rows(rs, ref, zero_pad)[:Np].view(np.uint32))
+    else:
+        assert np.array_equal(bf16_bits(res[:Np]), oracle.dispatch_rows(x, ref, zero_pad)[:Np])
+    if Np:
+        y = workload.expert_outputs(dict(seed=5, H=x.shape[1]), Np)
+        out = ep.combine(lay, to_dev_bf16(y), None if w is None else to_dev(w))
+        assert np.array_equal(bf16_bits(out), oracle.combine(y, ref["pair_slot"], w))
+    return lay, ref
+
+
+def _rand(T, K, E, H, seed=0, drop=0.0):
+    rng = np.random.default_rng(seed)
+    idx = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int64).reshape(T, K)
+    if drop:
+        idx[rng.random((T, K)) < drop] = -1
+    w = rng.random((T, K)).astype(np.float32)
+    x = workload.to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
+    return idx, w, x
+
+
+def test_zero_tokens(ep):
+    idx = np.zeros((0, 4), np.int64)
+    lay = ep.layout(to_dev(idx), None, 16, 2, 4)
+    recv = ep.dispatch(lay, torch.zeros((0, 256), dtype=torch.bfloat16, device=DEV), do_zero_padding=True)
+    out = ep.combine(lay, torch.zeros((4, 256), dtype=torch.bfloat16, device=DEV))
+    torch.cuda.synchronize()
+    assert out.shape == (0, 256) and recv.shape[1] == 256
+    assert lay.expert_offset.cpu().tolist() == [0] * 17
+    assert ep.get_status(lay) == (ep.EP_OK, 0)
+
+
+def test_all_unselected(ep):
+    T, K, E, H = 64, 4, 16, 256
+    idx = -np.ones((T, K), np.int64)
+    _, w, x = _rand(T, K, E, H)
+    lay, ref = _full(ep, idx, w, x, E, 2, 8)
+    out = ep.combine(lay, torch.zeros((1, H), dtype=torch.bfloat16, device=DEV), to_dev(w))
+    assert np.all(bf16_bits(out) == 0)
+
+
+@pytest.mark.parametrize("T,K,E,R,A,H", [
+    (1, 1, 1, 1, 1, 8),            # smallest everything
+    (1, 8, 256, 1, 128, 7168),     # single token
+    (7, 3, 12, 1, 5, 24),          # ragged everything, H = 24 (48-byte rows)
+    (96, 32, 64, 4, 3, 136),       # K = 32 (the maximum), H = 136
+    (130, 2, 4, 2, 128, 4096),     # few experts, heavy padding
+    (256, 8, 4096, 4, 1, 512),     # E at the maximum
+    (64, 4, 16, 16, 2, 16384),     # bf16 rows of 32 KB: two bulk segments per row
+    (4099, 8, 256, 1, 7, 7168),    # ragged chunking of a larger batch
+])
+def test_shapes_bf16(ep, T, K, E, R, A, H):
+    idx, w, x = _rand(T, K, E, H, seed=T + K, drop=0.1)
+    _full(ep, idx, w, x, E, R, A)
+
+
+@pytest.mark.parametrize("T,K,E,R,A,H", [
+    (5, 2, 8, 1, 4, 128),          # one scale per row (4-byte scale rows, plain stores)
+    (33, 8, 32, 1, 16, 640),       # 5 scales per row
+    (64, 4, 16, 2, 1, 16384),      # the largest row the cast kernel stages
+])
+def test_shapes_fp8(ep, T, K, E, R, A, H):
+    idx, w, x = _rand(T, K, E, H, seed=3 * T + K, drop=0.1)
+    _full(ep, idx, w, x, E, R, A, fp8=True)
+
+
+def test_fp8_input_passthrough(ep):
+    """(e4m3, scales) input is dispatched as is: rows and scale rows move together."""
+    T, K, E, R, A, H = 200, 8, 64, 4, 16, 1024
+    idx, w, x = _rand(T, K, E, H, seed=11)
+    q, s = oracle.cast_fp8(x)
+    ref = oracle.layout(idx, w, E, R, A)
+    lay = ep.layout(to_dev(idx), to_dev(w), E, R, A)
+    rq, rs = ep.dispatch(lay, to_dev(q).view(torch.float8_e4m3fn), x_scales=to_dev(s), do_zero_padding=True)
+    Np = int(ref["off"][-1])
+    assert np.array_equal(fp8_bits(rq[:Np]), oracle.dispatch_rows(q, ref, True)[:Np])
+    assert np.array_equal(f32_bits(rs[:Np]), oracle.dispatch_rows(s, ref, True)[:Np].view(np.uint32))
+
+
+def test_standalone_cast(ep):
+    x = np.concatenate([workload.tokens(workload.config("prefill_bf16"), rows=300),
+                        np.zeros((1, 7168), np.uint16)])
+    q, s = ep.cast_fp8(to_dev_bf16(x))
+    rq, rs = oracle.cast_fp8(x)
+    assert np.array_equal(fp8_bits(q), rq)
+    assert np.array_equal(f32_bits(s), rs.view(np.uint32))
+
+
+def test_bad_expert_reported(ep):
+    T, K, E, H = 32, 4, 16, 256
+    idx, w, x = _rand(T, K, E, H)
+    idx[3, 1] = E
+    idx[7, 0] = -5
+    lay = ep.layout(to_dev(idx), to_dev(w), E, 2, 1)
+    ep.dispatch(lay, to_dev_bf16(x))
+    code, flags = ep.get_status(lay)
+    assert code == ep.EP_ERR_BAD_EXPERT and flags & 1
+    # the bad entries are treated as unselected
+    ps = lay.pair_slot.cpu().numpy()
+    assert ps[3, 1] == -1 and ps[7, 0] == -1
+    # a later good layout on the same handle clears the status
+    idx2 = np.where(idx >= E, 0, np.maximum(idx, -1))
+    ep.layout(to_dev(idx2), to_dev(w), E, 2, 1, out=lay)
+    assert ep.get_status(lay) == (ep.EP_OK, 0)
+
+
+def test_capacity_overflow_reported(ep):
+    T, K, E, H, A = 64, 4, 16, 256, 8
+    idx, w, x = _rand(T, K, E, H)
+    lay = ep.layout(to_dev(idx), to_dev(w), E, 2, A, capacity=100)
+    recv = ep.dispatch(lay, to_dev_bf16(x), do_zero_padding=True)
+    ep.combine(lay, recv, to_dev(w))
+    code, flags = ep.get_status(lay)
+    assert code == ep.EP_ERR_CAPACITY and flags & 2
+
+
+def test_tokens_per_rank_limit(ep):
+    idx = np.zeros((256, 2), np.int64)
+    with pytest.raises(ep.EpError) as exc:
+        ep.layout(to_dev(idx), None, 8, 2, 1, num_max_tokens_per_rank=127)
+    assert exc.value.code == ep.EP_ERR_CAPACITY
+    ep.layout(to_dev(idx), None, 8, 2, 1, num_max_tokens_per_rank=128)
+
+
+def test_invalid_arguments(ep):
+    idx = to_dev(np.zeros((8, 2), np.int64))
+    for args in [(8, 3, 1), (8, 2, 0), (8, 0, 1)]:
+        with pytest.raises(ep.EpError) as exc:
+            ep.layout(idx, None, *args)
+        assert exc.value.code == ep.EP_ERR_INVALID_ARG
+    lay = ep.layout(idx, None, 8, 2, 1)
+    with pytest.raises(ep.EpError):   # H % 128 != 0 with the FP8 cast
+        ep.dispatch(lay, torch.zeros((8, 136), dtype=torch.bfloat16, device=DEV), cast_to_fp8=True)
+
+
+def test_bounded_wait_selftest(ep):
+    idx, w, x = _rand(16, 2, 8, 64)
+    lay = ep.layout(to_dev(idx), to_dev(w), 8, 2, 1)
+    ep.selftest_bounded_wait(lay, 2_000_000)       # 2 ms on a barrier nothing completes
+    code, flags = ep.get_status(lay)
+    assert code == ep.EP_ERR_TIMEOUT and flags & 4
+    _full(ep, idx, w, x, 8, 2, 1)                  # the context is still usable
+
+
+def _hash(*ts):
+    h = hashlib.sha256()
+    for t in ts:
+        h.update(t.contiguous().view(torch.uint8).cpu().numpy().tobytes())
+    return h.hexdigest()
+
+
+def test_determinism_repeated_runs(ep):
+    cfg = workload.config("prefill_bf16")
+    inp = workload.inputs(cfg)
+    idx, w, x = to_dev(inp["topk_idx"]), to_dev(inp["topk_weights"]), to_dev_bf16(inp["x"])
+    seen = set()
+    for _ in range(20):
+        lay = ep.layout(idx, w, cfg["E"], cfg["R"], cfg["A"])
+        recv = ep.dispatch(lay, x, do_zero_padding=True)
+        out = ep.combine(lay, recv, w)
+        Np = lay.num_recv_rows()
+        seen.add(_hash(lay.pair_slot, lay.recv_src_token[:Np], recv[:Np], out))
+    assert len(seen) == 1
+
+
+def test_batch_invariance(ep):
+    """Rows of the first tokens are identical whether combined in a batch of
+    1, 16, 64 or 257 tokens (the layout, and so every slot, changes with B)."""
+    T, K, E, H = 257, 8, 64, 512
+    idx, w, x = _rand(T, K, E, H, seed=21, drop=0.05)
+    outs = {}
+    for B in (1, 16, 64, 257):
+        lay = ep.layout(to_dev(idx[:B]), to_dev(w[:B]), E, 1, 4)
+        recv = ep.dispatch(lay, to_dev_bf16(x[:B]), do_zero_padding=True)
+        # a per-expert transform stands in for the experts: y = recv * (1 + lexp / 64)
+        scale = 1.0 + lay.recv_local_expert.clamp(min=0).float() / 64.0
+        y = (recv.float() * scale[:recv.shape[0], None]).to(torch.bfloat16)
+        outs[B] = bf16_bits(ep.combine(lay, y, to_dev(w[:B])))
+    for B in (16, 64, 257):
+        assert np.array_equal(outs[B][:1], outs[1])
+    assert np.array_equal(outs[257][:16], outs[16]) and np.array_equal(outs[257][:64], outs[64])

@@ -141,13 +141,23 @@ def tokens(cfg, rows=None):
 
 
 def expert_outputs(cfg, rows, seed_offset=0):
-    """Expert outputs for combine: bf16 bits [rows, H], magnitudes in [2^-7, 16)."""
+    """Expert outputs for combine: bf16 bits [rows, H], random sign and 7-bit
+    mantissa, exponent uniform in [-7, 3] (magnitudes in [2^-7, 16))."""
     g_y = np.random.Generator(np.random.PCG64(np.random.SeedSequence([cfg["seed"], 4, seed_offset])))
     H = cfg["H"]
-    sign = g_y.integers(0, 2, (rows, H), dtype=np.uint16) << np.uint16(15)
-    expo = (g_y.integers(127 - 7, 127 + 4, (rows, H), dtype=np.uint16)) << np.uint16(7)
-    mant = g_y.integers(0, 128, (rows, H), dtype=np.uint16)
-    return (sign | expo | mant).astype(np.uint16)
+    # 16 random bits per value: bit 0 sign, bits 1-7 mantissa, bits 8-15 pick
+    # the exponent (256 codes spread over the 11 exponents)
+    expo_of = ((127 - 7 + np.arange(256) * 11 // 256) << 7).astype(np.uint16)
+    out = np.empty((rows, H), np.uint16)
+    step = 8192
+    for r0 in range(0, rows, step):
+        n = min(step, rows - r0)
+        r = g_y.bit_generator.random_raw((n * H + 3) // 4).view(np.uint16)[:n * H].reshape(n, H)
+        v = expo_of[r >> np.uint16(8)]
+        v |= (r & np.uint16(1)) << np.uint16(15)
+        v |= (r >> np.uint16(1)) & np.uint16(0x7F)
+        out[r0:r0 + step] = v
+    return out
 
 
 def inputs(cfg, with_x=True):
