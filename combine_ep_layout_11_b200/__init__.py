@@ -6,9 +6,9 @@ sm_100a, declared in ``include/ep_b200.h``); this package only marshals torch
 tensors into it.  See :mod:`combine_ep_layout_11_b200.api`.
 """
 from .api import (EP_OK, EP_ERR_INVALID_ARG, EP_ERR_CAPACITY, EP_ERR_BAD_EXPERT, EP_ERR_TIMEOUT,
-                  EP_ERR_CUDA, EP_ERR_UNSUPPORTED, EpError, Layout, layout, dispatch, combine,
+                  EP_ERR_CUDA, EP_ERR_UNSUPPORTED, EpError, Layout, layout, dispatch, layout_dispatch, combine,
                   cast_fp8, get_status, capacity_rows, workspace_bytes, selftest_bounded_wait)
 
 __all__ = ["EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_CAPACITY", "EP_ERR_BAD_EXPERT", "EP_ERR_TIMEOUT",
-           "EP_ERR_CUDA", "EP_ERR_UNSUPPORTED", "EpError", "Layout", "layout", "dispatch", "combine",
+           "EP_ERR_CUDA", "EP_ERR_UNSUPPORTED", "EpError", "Layout", "layout", "dispatch", "layout_dispatch", "combine",
            "cast_fp8", "get_status", "capacity_rows", "workspace_bytes", "selftest_bounded_wait"]

@@ -84,7 +84,7 @@ class Layout:
         nbytes = workspace_bytes(T, K, E, A)
         if nbytes == 0:
             raise EpError(EP_ERR_INVALID_ARG, "workspace size")
-        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)   # zeroed before first use
         s = _lib.EpLayout()
         s.num_recv_tokens_per_expert = self.num_recv_tokens_per_expert.data_ptr()
         s.expert_offset = self.expert_offset.data_ptr()
@@ -155,6 +155,40 @@ def dispatch(lay, x, x_scales=None, cast_to_fp8=False, do_zero_padding=False, ou
                          int(bool(do_zero_padding)), _ptr(out), _ptr(out_scales if fp8_out else None),
                          _stream(x.device)), "ep_dispatch")
     return (out, out_scales) if fp8_out else out
+
+
+def layout_dispatch(topk_idx, topk_weights, x, num_experts, num_ranks, expert_alignment=1,
+                    num_max_tokens_per_rank=0, x_scales=None, cast_to_fp8=False, do_zero_padding=False,
+                    capacity=None, out_layout=None, out=None, out_scales=None):
+    """Layout and dispatch in one call (§2.1: V2's dispatch() derives the layout
+    from topk_idx).  Same results as ``layout`` then ``dispatch``; returns
+    ``(layout, recv_x)`` or ``(layout, (recv_x, recv_scales))`` for FP8 output."""
+    L = _lib.load()
+    assert topk_idx.dtype == torch.int64 and topk_idx.dim() == 2 and topk_idx.is_contiguous()
+    T, K = topk_idx.shape
+    if topk_weights is not None:
+        assert topk_weights.dtype == torch.float32 and topk_weights.shape == (T, K)
+        assert topk_weights.is_contiguous()
+    assert x.dim() == 2 and x.is_contiguous() and x.shape[0] == T
+    if out_layout is not None:
+        assert (out_layout.num_tokens, out_layout.num_topk, out_layout.num_experts) == (T, K, num_experts)
+    lay = out_layout if out_layout is not None else Layout(T, K, num_experts, num_ranks, expert_alignment,
+                                                           topk_idx.device, capacity, num_max_tokens_per_rank)
+    H = x.shape[1]
+    fp8_in = x.dtype == torch.float8_e4m3fn
+    assert fp8_in or x.dtype == torch.bfloat16
+    fp8_out = fp8_in or cast_to_fp8
+    cap = max(lay.capacity, 1)
+    if out is None:
+        out = torch.empty((cap, H), dtype=torch.float8_e4m3fn if fp8_out else torch.bfloat16, device=x.device)
+    if fp8_out and out_scales is None:
+        out_scales = torch.empty((cap, H // 128), dtype=torch.float32, device=x.device)
+    _check(L.ep_layout_dispatch(_ptr(topk_idx), _ptr(topk_weights), T, K, num_experts, num_ranks,
+                                expert_alignment, num_max_tokens_per_rank, lay.ref(), _ptr(x),
+                                EP_DTYPE_FP8_E4M3 if fp8_in else EP_DTYPE_BF16, _ptr(x_scales if fp8_in else None),
+                                H, int(bool(cast_to_fp8)), int(bool(do_zero_padding)), _ptr(out),
+                                _ptr(out_scales if fp8_out else None), _stream(x.device)), "ep_layout_dispatch")
+    return lay, ((out, out_scales) if fp8_out else out)
 
 
 def combine(lay, y, topk_weights=None, out=None):

@@ -2,6 +2,7 @@
 // checks, then kernel launches on the caller's stream.  No allocation, no
 // state kept between calls, no host synchronisation except ep_get_status.
 #include <limits.h>
+#include <stdlib.h>
 
 #include "ep_internal.h"
 
@@ -25,7 +26,113 @@ int check_handle(const ep_layout_t* L) {
 
 ep::WsHeader* header(const ep_layout_t* L) { return reinterpret_cast<ep::WsHeader*>(L->workspace); }
 
+// Argument checks of ep_layout; on success fills the handle's shape fields and
+// the kernel arguments (chunking is chosen at launch).
+int prepare_layout(const int64_t* topk_idx, const float* topk_weights, int T, int K, int E, int R, int A,
+                   int num_max_tokens_per_rank, ep_layout_t* layout, ep::LayoutArgs* a) {
+    if (!layout) return EP_ERR_INVALID_ARG;
+    if (T < 0 || K < 1 || E < 1 || R < 1 || A < 1 || num_max_tokens_per_rank < 0) return EP_ERR_INVALID_ARG;
+    if (K > EP_MAX_TOPK || E > EP_MAX_EXPERTS) return EP_ERR_UNSUPPORTED;
+    if (E % R != 0 || T % R != 0) return EP_ERR_INVALID_ARG;
+    if ((int64_t)T * K + (int64_t)E * (A - 1) > INT_MAX) return EP_ERR_UNSUPPORTED;
+    if (layout->capacity < 0) return EP_ERR_INVALID_ARG;
+    if (layout->capacity > INT_MAX) return EP_ERR_UNSUPPORTED;
+    if (num_max_tokens_per_rank > 0 && T / R > num_max_tokens_per_rank) return EP_ERR_CAPACITY;
+    if ((T > 0 && !topk_idx) || !layout->num_recv_tokens_per_expert || !layout->expert_offset ||
+        !layout->pair_slot || !layout->recv_src_token || !layout->recv_weight || !layout->recv_local_expert ||
+        !layout->workspace)
+        return EP_ERR_INVALID_ARG;
+    if (!aligned(topk_idx, 8) || !aligned(topk_weights, 4) || !aligned(layout->num_recv_tokens_per_expert, 4) ||
+        !aligned(layout->expert_offset, 4) || !aligned(layout->pair_slot, 4) ||
+        !aligned(layout->recv_src_token, 4) || !aligned(layout->recv_weight, 4) ||
+        !aligned(layout->recv_local_expert, 4) || !aligned(layout->workspace, 256))
+        return EP_ERR_INVALID_ARG;
+    const ep::WsLayout ws = ep::ws_layout(T, K, E, A);
+    if (layout->workspace_bytes < ws.total) return EP_ERR_INVALID_ARG;
+
+    layout->num_tokens = T;
+    layout->num_topk = K;
+    layout->num_experts = E;
+    layout->num_ranks = R;
+    layout->expert_alignment = A;
+    layout->num_max_tokens_per_rank = num_max_tokens_per_rank;
+    layout->magic = kLayoutMagic;
+
+    uint8_t* wsb = reinterpret_cast<uint8_t*>(layout->workspace);
+    a->topk_idx = topk_idx;
+    a->topk_weights = topk_weights;
+    a->T = T; a->K = K; a->E = E; a->R = R; a->A = A;
+    a->C = 0;
+    a->CT = 0;
+    a->capacity = layout->capacity;
+    a->cnt = layout->num_recv_tokens_per_expert;
+    a->off = layout->expert_offset;
+    a->pair_slot = layout->pair_slot;
+    a->recv_src = layout->recv_src_token;
+    a->recv_w = layout->recv_weight;
+    a->recv_lexp = layout->recv_local_expert;
+    a->hdr = reinterpret_cast<ep::WsHeader*>(wsb);
+    a->table = reinterpret_cast<int32_t*>(wsb + ws.table_off);
+    a->padpre = reinterpret_cast<int32_t*>(wsb + ws.padpre_off);
+    a->pad_rows = reinterpret_cast<int32_t*>(wsb + ws.padrows_off);
+    return EP_OK;
+}
+
+// A layout of zero tokens: no kernels, just zero counts and offsets.
+int empty_layout(ep_layout_t* layout, cudaStream_t s) {
+    if (cudaMemsetAsync(layout->workspace, 0, sizeof(ep::WsHeader), s) != cudaSuccess ||
+        cudaMemsetAsync(layout->num_recv_tokens_per_expert, 0, (size_t)layout->num_experts * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(layout->expert_offset, 0, (size_t)(layout->num_experts + 1) * 4, s) != cudaSuccess)
+        return EP_ERR_CUDA;
+    return EP_OK;
+}
+
+// Argument checks of ep_dispatch against a filled handle; fills the kernel arguments.
+int prepare_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales, int H,
+                     int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales, ep::DispatchArgs* a,
+                     int* elem_bytes) {
+    int rc = check_handle(layout);
+    if (rc != EP_OK) return rc;
+    const int T = layout->num_tokens;
+    if (H <= 0 || (x_dtype != EP_DTYPE_BF16 && x_dtype != EP_DTYPE_FP8_E4M3)) return EP_ERR_INVALID_ARG;
+    if (cast_to_fp8 && x_dtype != EP_DTYPE_BF16) return EP_ERR_INVALID_ARG;
+    const bool fp8_in = x_dtype == EP_DTYPE_FP8_E4M3;
+    const bool fp8_out = fp8_in || cast_to_fp8;
+    if (H % 8 != 0 || (fp8_out && H % 128 != 0)) return EP_ERR_INVALID_ARG;
+    if ((T > 0 && !x) || !recv_x || (fp8_out && !recv_scales) || (fp8_in && T > 0 && !x_scales))
+        return EP_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(x_scales, 4) || !aligned(recv_scales, 16))
+        return EP_ERR_INVALID_ARG;
+    if (cast_to_fp8 && H > 16384) return EP_ERR_UNSUPPORTED;
+
+    const uint8_t* wsb = reinterpret_cast<const uint8_t*>(layout->workspace);
+    const ep::WsLayout ws = ep::ws_layout(T, layout->num_topk, layout->num_experts, layout->expert_alignment);
+    a->x = reinterpret_cast<const uint8_t*>(x);
+    a->x_scales = fp8_in ? x_scales : nullptr;
+    a->recv = reinterpret_cast<uint8_t*>(recv_x);
+    a->recv_scales = fp8_out ? recv_scales : nullptr;
+    a->pair_slot = layout->pair_slot;
+    a->hdr = reinterpret_cast<const ep::WsHeader*>(wsb);
+    a->pad_rows = reinterpret_cast<const int32_t*>(wsb + ws.padrows_off);
+    a->status_hdr = header(layout);
+    a->T = T;
+    a->K = layout->num_topk;
+    a->H = H;
+    a->capacity = layout->capacity;
+    a->nb = fp8_out ? H / 128 : 0;
+    a->zero_pad = do_zero_padding ? 1 : 0;
+    *elem_bytes = fp8_in ? 1 : 2;
+    return device_sms(&a->sms);
+}
+
 }  // namespace
+
+namespace ep {
+int combine_variant() {
+    const char* v = getenv("EP_B200_COMBINE_VARIANT");
+    return (v && (v[0] == '1' || v[0] == '2')) ? v[0] - '0' : 0;
+}
+}  // namespace ep
 
 extern "C" {
 
@@ -57,102 +164,55 @@ int64_t ep_capacity_rows(int num_tokens, int num_topk, int num_experts, int expe
 int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
               int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
               ep_layout_t* layout, void* stream) {
-    const int T = num_tokens, K = num_topk, E = num_experts, R = num_ranks, A = expert_alignment;
-    if (!layout) return EP_ERR_INVALID_ARG;
-    if (T < 0 || K < 1 || E < 1 || R < 1 || A < 1 || num_max_tokens_per_rank < 0) return EP_ERR_INVALID_ARG;
-    if (K > EP_MAX_TOPK || E > EP_MAX_EXPERTS) return EP_ERR_UNSUPPORTED;
-    if (E % R != 0 || T % R != 0) return EP_ERR_INVALID_ARG;
-    if ((int64_t)T * K + (int64_t)E * (A - 1) > INT_MAX) return EP_ERR_UNSUPPORTED;
-    if (layout->capacity < 0) return EP_ERR_INVALID_ARG;
-    if (layout->capacity > INT_MAX) return EP_ERR_UNSUPPORTED;
-    if (num_max_tokens_per_rank > 0 && T / R > num_max_tokens_per_rank) return EP_ERR_CAPACITY;
-    if ((T > 0 && !topk_idx) || !layout->num_recv_tokens_per_expert || !layout->expert_offset ||
-        !layout->pair_slot || !layout->recv_src_token || !layout->recv_weight || !layout->recv_local_expert ||
-        !layout->workspace)
-        return EP_ERR_INVALID_ARG;
-    if (!aligned(topk_idx, 8) || !aligned(topk_weights, 4) || !aligned(layout->num_recv_tokens_per_expert, 4) ||
-        !aligned(layout->expert_offset, 4) || !aligned(layout->pair_slot, 4) ||
-        !aligned(layout->recv_src_token, 4) || !aligned(layout->recv_weight, 4) ||
-        !aligned(layout->recv_local_expert, 4) || !aligned(layout->workspace, 256))
-        return EP_ERR_INVALID_ARG;
-    const ep::WsLayout ws = ep::ws_layout(T, K, E, A);
-    if (layout->workspace_bytes < ws.total) return EP_ERR_INVALID_ARG;
-
-    layout->num_tokens = T;
-    layout->num_topk = K;
-    layout->num_experts = E;
-    layout->num_ranks = R;
-    layout->expert_alignment = A;
-    layout->num_max_tokens_per_rank = num_max_tokens_per_rank;
-    layout->magic = kLayoutMagic;
-
-    cudaStream_t s = (cudaStream_t)stream;
-    uint8_t* wsb = reinterpret_cast<uint8_t*>(layout->workspace);
-    if (cudaMemsetAsync(wsb, 0, sizeof(ep::WsHeader), s) != cudaSuccess) return EP_ERR_CUDA;
-    if (T == 0) {
-        if (cudaMemsetAsync(layout->num_recv_tokens_per_expert, 0, (size_t)E * 4, s) != cudaSuccess ||
-            cudaMemsetAsync(layout->expert_offset, 0, (size_t)(E + 1) * 4, s) != cudaSuccess)
-            return EP_ERR_CUDA;
-        return EP_OK;
-    }
-    const ep::Chunking ch = ep::chunking(T, K, E);
     ep::LayoutArgs a;
-    a.topk_idx = topk_idx;
-    a.topk_weights = topk_weights;
-    a.T = T; a.K = K; a.E = E; a.R = R; a.A = A;
-    a.C = ch.num_chunks;
-    a.CT = ch.chunk_tokens;
-    a.capacity = layout->capacity;
-    a.cnt = layout->num_recv_tokens_per_expert;
-    a.off = layout->expert_offset;
-    a.pair_slot = layout->pair_slot;
-    a.recv_src = layout->recv_src_token;
-    a.recv_w = layout->recv_weight;
-    a.recv_lexp = layout->recv_local_expert;
-    a.hdr = reinterpret_cast<ep::WsHeader*>(wsb);
-    a.table = reinterpret_cast<int32_t*>(wsb + ws.table_off);
-    a.padpre = reinterpret_cast<int32_t*>(wsb + ws.padpre_off);
-    a.pad_rows = reinterpret_cast<int32_t*>(wsb + ws.padrows_off);
-    return ep::launch_layout(a, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    int rc = prepare_layout(topk_idx, topk_weights, num_tokens, num_topk, num_experts, num_ranks,
+                            expert_alignment, num_max_tokens_per_rank, layout, &a);
+    if (rc != EP_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (num_tokens == 0) return empty_layout(layout, s);
+    int sms = 0;
+    if ((rc = device_sms(&sms)) != EP_OK) return rc;
+    return ep::launch_layout(a, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
 int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales, int hidden,
                 int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales, void* stream) {
-    int rc = check_handle(layout);
-    if (rc != EP_OK) return rc;
-    const int H = hidden, T = layout->num_tokens;
-    if (H <= 0 || (x_dtype != EP_DTYPE_BF16 && x_dtype != EP_DTYPE_FP8_E4M3)) return EP_ERR_INVALID_ARG;
-    if (cast_to_fp8 && x_dtype != EP_DTYPE_BF16) return EP_ERR_INVALID_ARG;
-    const bool fp8_in = x_dtype == EP_DTYPE_FP8_E4M3;
-    const bool fp8_out = fp8_in || cast_to_fp8;
-    if (H % 8 != 0 || (fp8_out && H % 128 != 0)) return EP_ERR_INVALID_ARG;
-    if ((T > 0 && !x) || !recv_x || (fp8_out && !recv_scales) || (fp8_in && T > 0 && !x_scales))
-        return EP_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(x_scales, 4) || !aligned(recv_scales, 16))
-        return EP_ERR_INVALID_ARG;
-    if (cast_to_fp8 && H > 16384) return EP_ERR_UNSUPPORTED;
-    if (T == 0) return EP_OK;   // no tokens, no pairs, no padding rows
-
-    const uint8_t* wsb = reinterpret_cast<const uint8_t*>(layout->workspace);
-    const ep::WsLayout ws = ep::ws_layout(T, layout->num_topk, layout->num_experts, layout->expert_alignment);
     ep::DispatchArgs a;
-    a.x = reinterpret_cast<const uint8_t*>(x);
-    a.x_scales = fp8_in ? x_scales : nullptr;
-    a.recv = reinterpret_cast<uint8_t*>(recv_x);
-    a.recv_scales = fp8_out ? recv_scales : nullptr;
-    a.pair_slot = layout->pair_slot;
-    a.hdr = reinterpret_cast<const ep::WsHeader*>(wsb);
-    a.pad_rows = reinterpret_cast<const int32_t*>(wsb + ws.padrows_off);
-    a.status_hdr = header(layout);
-    a.T = T;
-    a.K = layout->num_topk;
-    a.H = H;
-    a.capacity = layout->capacity;
-    a.nb = fp8_out ? H / 128 : 0;
-    a.zero_pad = do_zero_padding ? 1 : 0;
-    if ((rc = device_sms(&a.sms)) != EP_OK) return rc;
+    int elem_bytes = 0;
+    int rc = prepare_dispatch(layout, x, x_dtype, x_scales, hidden, cast_to_fp8, do_zero_padding, recv_x,
+                              recv_scales, &a, &elem_bytes);
+    if (rc != EP_OK) return rc;
+    if (layout->num_tokens == 0) return EP_OK;   // no tokens, no pairs, no padding rows
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t err = cast_to_fp8 ? ep::launch_dispatch_cast(a, s) : ep::launch_dispatch_copy(a, fp8_in ? 1 : 2, s);
+    cudaError_t err = cast_to_fp8 ? ep::launch_dispatch_cast(a, s) : ep::launch_dispatch_copy(a, elem_bytes, s);
+    return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
+                       int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
+                       ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales, int hidden,
+                       int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales, void* stream) {
+    if (!layout) return EP_ERR_INVALID_ARG;
+    ep_layout_t tmp = *layout;   // the handle changes only once every check has passed
+    ep::LayoutArgs la;
+    ep::DispatchArgs da;
+    int elem_bytes = 0;
+    int rc = prepare_layout(topk_idx, topk_weights, num_tokens, num_topk, num_experts, num_ranks,
+                            expert_alignment, num_max_tokens_per_rank, &tmp, &la);
+    if (rc != EP_OK) return rc;
+    rc = prepare_dispatch(&tmp, x, x_dtype, x_scales, hidden, cast_to_fp8, do_zero_padding, recv_x, recv_scales,
+                          &da, &elem_bytes);
+    if (rc != EP_OK) return rc;
+    *layout = tmp;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (num_tokens == 0) return empty_layout(layout, s);
+    cudaError_t err;
+    if (cast_to_fp8) {
+        err = ep::launch_layout(la, da.sms, s);
+        if (err == cudaSuccess) err = ep::launch_dispatch_cast(da, s);
+    } else {
+        err = ep::launch_layout_dispatch(la, da, elem_bytes, s);
+    }
     return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
@@ -174,6 +234,8 @@ int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float
     a.K = layout->num_topk;
     a.H = H;
     a.capacity = layout->capacity;
+    a.status = header(layout);
+    a.variant = ep::combine_variant();
     if ((rc = device_sms(&a.sms)) != EP_OK) return rc;
     return ep::launch_combine(a, (cudaStream_t)stream) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }

@@ -36,8 +36,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-template <int V>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
+template <int V, int kMinBlocks>
+__global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(CombineArgs a) {
     const int lane = threadIdx.x & 31;
     const int64_t gw = ((int64_t)blockIdx.x * kCombineThreads + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * kCombineThreads) >> 5;
@@ -47,17 +47,30 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
     const int64_t items = (int64_t)a.T * nch;
     const int K = a.K;
     const uint4* y = reinterpret_cast<const uint4*>(a.y);
+    pdl_wait();
+    pdl_launch_dependents();
 
+    // the (slot, weight) of lane k for the warp's next item is loaded while the
+    // current item is processed, so no item starts with a dependent load
+    auto fetch = [&](int64_t it, int& slot, float& w) {
+        slot = -1;
+        w = 1.0f;
+        if (it < items && lane < K) {
+            const int64_t t = it / nch;
+            slot = a.pair_slot[t * K + lane];
+            if (a.w) w = a.w[t * K + lane];
+        }
+    };
+    int next_slot;
+    float next_w;
+    fetch(gw, next_slot, next_w);
     for (int64_t it = gw; it < items; it += nw) {
         const int64_t t = it / nch;
         const int ch = (int)(it % nch);
-        int my_slot = -1;
-        float my_w = 1.0f;
-        if (lane < K) {
-            my_slot = a.pair_slot[t * K + lane];
-            if (a.w) my_w = a.w[t * K + lane];
-            if ((int64_t)my_slot >= a.capacity) my_slot = -1;
-        }
+        int my_slot = next_slot;
+        const float my_w = next_w;
+        fetch(it + nw, next_slot, next_w);
+        if ((int64_t)my_slot >= a.capacity) my_slot = -1;
         float acc[V][8];
 #pragma unroll
         for (int v = 0; v < V; ++v)
@@ -105,6 +118,131 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
     }
 }
 
+// ---------------------------------------------------------------------------
+// TMA-staged variant for K <= 8: the item is (token, 2 KB column segment).  A
+// producer warp bulk-loads the K rows' segments into a stage of a ring in
+// shared memory (one mbarrier per stage counts the bytes); four consumer warps
+// reduce the stage in ascending k, one 16-byte column per thread, and store the
+// bf16 result.  The ring keeps many row segments in flight per SM without
+// holding them in registers.
+// ---------------------------------------------------------------------------
+constexpr int kStageK = 8;
+constexpr int kSegVec = 128;                 // 16-byte columns per segment (2 KB of bf16)
+constexpr int kSegBytes = kSegVec * 16;
+constexpr int kConsumerWarps = 4;
+constexpr int kTmaThreads = 32 * (1 + kConsumerWarps);
+
+struct StageMeta {
+    float w[kStageK];
+    int32_t valid;   // bit k: row k was loaded
+    int32_t pad[7];
+};
+
+__global__ void __launch_bounds__(kTmaThreads) combine_tma_kernel(CombineArgs a, int stages) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t* ring = smem;                                                   // [stages][kStageK][kSegBytes]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * kStageK * kSegBytes);
+    uint64_t* empty = full + stages;
+    StageMeta* meta = reinterpret_cast<StageMeta*>(empty + stages);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int K = a.K, HV = a.H / 8;
+    const int nseg = (HV + kSegVec - 1) / kSegVec;
+    const int64_t items = (int64_t)a.T * nseg;
+    const int64_t G = gridDim.x, first = blockIdx.x;
+    const int64_t n = first < items ? (items - first + G - 1) / G : 0;
+    const uint32_t row_bytes = (uint32_t)a.H * 2u;
+
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // producer; the (slot, weight) of lane k for item j+1 is loaded while
+        // item j is issued, so no item waits on a dependent global load
+        auto fetch = [&](int64_t j, int32_t& slot, float& w) {
+            slot = -1;
+            w = 1.0f;
+            if (j < n && lane < K) {
+                const int64_t t = (first + j * G) / nseg;
+                slot = a.pair_slot[t * K + lane];
+                if (a.w) w = a.w[t * K + lane];
+            }
+        };
+        int32_t next_slot;
+        float next_w;
+        fetch(0, next_slot, next_w);
+        for (int64_t j = 0; j < n; ++j) {
+            const int s = (int)(j % stages);
+            int32_t slot = next_slot;
+            float w = next_w;
+            fetch(j + 1, next_slot, next_w);
+            if ((int64_t)slot >= a.capacity) slot = -1;
+            if (!mbar_wait(&empty[s], (uint32_t)(((j / stages) & 1) ^ 1))) {
+                if (lane == 0) atomicOr(&a.status->status, kDevTimeout);
+                break;
+            }
+            const int64_t item = first + j * G;
+            const int g = (int)(item % nseg);
+            const uint32_t bytes = (uint32_t)min(kSegVec, HV - g * kSegVec) * 16u;
+            const uint32_t valid = __ballot_sync(0xffffffffu, slot >= 0);
+            if (lane < kStageK) meta[s].w[lane] = w;
+            if (lane == 0) meta[s].valid = (int32_t)valid;
+            __syncwarp();   // the metadata writes are ordered before lane 0's release-arrive
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes * __popc(valid));
+            __syncwarp();
+            if (slot >= 0)
+                bulk_load(ring + ((size_t)s * kStageK + lane) * kSegBytes,
+                          a.y + (int64_t)slot * (row_bytes / 2) + (int64_t)g * kSegVec * 8, bytes, &full[s]);
+        }
+        return;
+    }
+
+    // consumers
+    const int ct = tid - 32;   // 0 .. 127: one 16-byte column of the segment
+    for (int64_t j = 0; j < n; ++j) {
+        const int s = (int)(j % stages);
+        const bool ok = mbar_wait(&full[s], (uint32_t)((j / stages) & 1));
+        if (!ok) {
+            if (ct == 0) atomicOr(&a.status->status, kDevTimeout);
+            return;
+        }
+        const int64_t item = first + j * G;
+        const int64_t t = item / nseg;
+        const int g = (int)(item % nseg);
+        const int col = g * kSegVec + ct;
+        const uint32_t valid = (uint32_t)meta[s].valid;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        if (col < HV) {
+#pragma unroll
+            for (int k = 0; k < kStageK; ++k) {
+                if (valid & (1u << k)) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(ring + ((size_t)s * kStageK + k) * kSegBytes + ct * 16);
+                    accumulate8(acc, v, meta[s].w[k]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[s])) : "memory");
+        if (col < HV) {
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]);
+            o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]);
+            o.w = pack_bf16x2(acc[6], acc[7]);
+            st_v4(reinterpret_cast<uint4*>(a.out) + t * HV + col, o);
+        }
+    }
+}
+
 __global__ void selftest_wait_kernel(WsHeader* hdr, uint64_t timeout_ns) {
     __shared__ __align__(8) uint64_t bar;
     if (threadIdx.x == 0) {
@@ -118,14 +256,24 @@ __global__ void selftest_wait_kernel(WsHeader* hdr, uint64_t timeout_ns) {
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
-    constexpr int V = 2;
+    if (a.variant == 1 && a.K <= kStageK) {
+        const int stages = 6;
+        const size_t smem = (size_t)stages * kStageK * kSegBytes + 2 * stages * 8 + stages * sizeof(StageMeta);
+        cudaError_t err =
+            cudaFuncSetAttribute(combine_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        int per_sm = 0;
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_tma_kernel, kTmaThreads, smem);
+        if (err != cudaSuccess) return err;
+        if (per_sm < 1) per_sm = 1;
+        return launch_pdl(combine_tma_kernel, dim3(a.sms * per_sm), dim3(kTmaThreads), smem, s, false, a, stages);
+    }
+    auto kernel = a.variant == 2 ? combine_kernel<1, 3> : combine_kernel<2, 2>;
     int blocks_per_sm = 0;
-    cudaError_t err =
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, combine_kernel<V>, kCombineThreads, 0);
+    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kernel, kCombineThreads, 0);
     if (err != cudaSuccess) return err;
     if (blocks_per_sm < 1) blocks_per_sm = 1;
-    combine_kernel<V><<<a.sms * blocks_per_sm, kCombineThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kernel, dim3(a.sms * blocks_per_sm), dim3(kCombineThreads), 0, s, false, a);
 }
 
 cudaError_t launch_selftest_wait(WsHeader* hdr, uint64_t timeout_ns, cudaStream_t s) {

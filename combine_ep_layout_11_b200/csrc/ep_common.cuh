@@ -28,30 +28,32 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // Workspace: [0, 256) header words, then the (chunk x expert) count table,
 // the padding prefix and the list of padding rows.
 // ---------------------------------------------------------------------------
+// `bar_count` and `pending` must be zero before the first ep_layout on a
+// workspace; every ep_layout leaves them at zero again.
 struct WsHeader {
-    uint32_t status;     // EP_DEV_* bits
-    uint32_t ticket;     // arrival counter of the counting kernel's CTAs
+    uint32_t status;     // EP_DEV_* bits of the last ep_layout and what followed it
+    uint32_t bar_count;  // grid barrier: CTAs arrived in the current generation
     int32_t num_pad;     // padding rows (expert_offset[E] - pairs)
-    int32_t pad0;
+    uint32_t pending;    // flags raised by CTAs before the barrier
+    uint32_t bar_gen;    // grid barrier generation
 };
+
+// Most chunks (CTAs of the layout kernel) a layout uses.
+constexpr int kMaxChunks = 256;
 
 struct Chunking {
     int num_chunks;       // C: CTAs of the counting / slot kernels
     int chunk_tokens;     // CT: tokens per chunk
 };
 
-// Chunks of whole tokens, about 256 pairs each, at most 128 chunks, and at most
-// 32768 (chunk, expert) cells so that the whole count table fits in one CTA's
-// shared memory for the scan.
-inline Chunking chunking(int T, int K, int E) {
+// Chunks of whole tokens, about 256 pairs each, at most `max_chunks`
+// (kMaxChunks, or fewer when the device cannot hold that many CTAs at once).
+inline Chunking chunking(int T, int K, int max_chunks = kMaxChunks) {
     Chunking c{0, 0};
     if (T <= 0) return c;
     int64_t pairs = (int64_t)T * K;
-    int64_t cmax = 32768 / E;
-    if (cmax < 1) cmax = 1;
     int64_t n = (pairs + 255) / 256;
-    if (n > 128) n = 128;
-    if (n > cmax) n = cmax;
+    if (n > max_chunks) n = max_chunks;
     if (n < 1) n = 1;
     int64_t ct = ((int64_t)T + n - 1) / n;
     c.chunk_tokens = (int)ct;
@@ -59,8 +61,10 @@ inline Chunking chunking(int T, int K, int E) {
     return c;
 }
 
+__host__ __device__ inline int round4(int x) { return (x + 3) / 4 * 4; }
+
 struct WsLayout {
-    size_t table_off;    // int32 [C][E]: per-chunk counts, then per-chunk row bases
+    size_t table_off;    // int32 [kMaxChunks][round4(E)]: per-chunk expert counts
     size_t padpre_off;   // int32 [E+1]: exclusive prefix of padding rows per expert
     size_t padrows_off;  // int32 [E*(A-1)]: receive row of every padding row
     size_t total;
@@ -69,10 +73,10 @@ struct WsLayout {
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline WsLayout ws_layout(int T, int K, int E, int A) {
-    Chunking ch = chunking(T, K, E);
+    (void)K;
     WsLayout w;
     w.table_off = 256;
-    w.padpre_off = round_up(w.table_off + (size_t)ch.num_chunks * E * 4, 256);
+    w.padpre_off = round_up(w.table_off + (T > 0 ? (size_t)kMaxChunks * round4(E) * 4 : 0), 256);
     w.padrows_off = round_up(w.padpre_off + ((size_t)E + 1) * 4, 256);
     w.total = round_up(w.padrows_off + (size_t)E * (size_t)(A > 1 ? A - 1 : 0) * 4 + 4, 256);
     return w;
@@ -163,6 +167,12 @@ __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Programmatic dependent launch: wait until the preceding grid in the stream
+// has completed and its writes are visible (a no-op when launched without the
+// attribute), and allow the next grid to be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
@@ -181,6 +191,29 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
+}
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while its predecessor in the stream finishes; it must call pdl_wait() before
+// touching global memory.
+// With `cooperative`, all CTAs of the grid are guaranteed to be resident at
+// once (needed by a grid barrier).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              bool cooperative, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = cooperative ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 }  // namespace ep

@@ -50,6 +50,8 @@ __global__ void __launch_bounds__(32) dispatch_copy_kernel(DispatchArgs a, uint3
         fence_barrier_init();
     }
     __syncwarp();
+    pdl_wait();
+    pdl_launch_dependents();
 
     const int64_t G = gridDim.x;
     const int64_t items = (int64_t)a.T * nseg;
@@ -171,6 +173,8 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
         fence_barrier_init();
     }
     __syncthreads();
+    pdl_wait();
+    pdl_launch_dependents();
 
     const int64_t G = gridDim.x;
     const int64_t first = blockIdx.x;
@@ -283,8 +287,7 @@ cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStre
     if (ctas_per_sm > 4) ctas_per_sm = 4;
     if (ctas_per_sm < 1) ctas_per_sm = 1;
     const int grid = a.sms * ctas_per_sm;
-    dispatch_copy_kernel<<<grid, 32, smem, s>>>(a, row_bytes, seg_bytes, nseg, stages);
-    return cudaGetLastError();
+    return launch_pdl(dispatch_copy_kernel, dim3(grid), dim3(32), smem, s, false, a, row_bytes, seg_bytes, nseg, stages);
 }
 
 cudaError_t launch_dispatch_cast(const DispatchArgs& a, cudaStream_t s) {
@@ -301,8 +304,7 @@ cudaError_t launch_dispatch_cast(const DispatchArgs& a, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     if (ctas_per_sm > 4) ctas_per_sm = 4;
     if (ctas_per_sm < 1) ctas_per_sm = 1;
-    dispatch_cast_kernel<<<a.sms * ctas_per_sm, kCastThreads, smem, s>>>(a, stages);
-    return cudaGetLastError();
+    return launch_pdl(dispatch_cast_kernel, dim3(a.sms * ctas_per_sm), dim3(kCastThreads), smem, s, false, a, stages);
 }
 
 }  // namespace ep

@@ -1,0 +1,171 @@
+// Layout and dispatch in one kernel, the way DeepEP V2's dispatch() derives
+// its routing layout from topk_idx inside the call ("DeepEP 测试目标 API 系统性参考"
+// §2.1 and the V1/V2 comparison table in §3.1).
+//
+// One cooperative CTA per SM, and CTA c owns layout chunk c (a run of whole
+// tokens).  Before any layout work, warp 0 starts TMA bulk loads of the
+// chunk's first token rows into a shared-memory ring, so the row reads overlap
+// the layout's latency chain (count, grid barrier, scan, slot assignment).
+// Then warp 0 walks the chunk's rows: when a row has landed, lanes k < K each
+// issue one bulk store to receive row pair_slot[t, k] (written moments before
+// by this CTA), and the freed stage is refilled.  Warp 1 meanwhile zero-fills a
+// contiguous 1/C share of all padding rows with bulk stores from a zeroed
+// segment.  The bytes moved are exactly those of ep_layout + ep_dispatch.
+#include "ep_layout_body.cuh"
+
+namespace ep {
+
+namespace {
+
+constexpr int kFusedThreads = layout_dev::kLayoutThreads;
+constexpr uint32_t kMaxSegBytes = 16384;
+
+__host__ __device__ __forceinline__ uint32_t rup(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    layout_dispatch_kernel(LayoutArgs la, DispatchArgs da, uint32_t row_bytes, uint32_t seg_bytes, int nseg,
+                           int stages, uint32_t layout_bytes) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    int32_t* lsm = reinterpret_cast<int32_t*>(smem);
+    const uint32_t stride = rup(seg_bytes, 128);
+    uint8_t* stage = smem + layout_bytes;
+    uint8_t* zero = stage + (size_t)stages * stride;
+    uint64_t* full = reinterpret_cast<uint64_t*>(zero + stride);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int K = la.K;
+    const int c = blockIdx.x;
+
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    for (uint32_t o = tid * 16u; o < stride; o += kFusedThreads * 16u)
+        *reinterpret_cast<uint4*>(zero + o) = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+    __syncthreads();
+    pdl_wait();
+    pdl_launch_dependents();
+
+    // this CTA's rows: the tokens of its layout chunk, all segments of a token in a row
+    const int64_t t0 = (int64_t)c * la.CT;
+    const int64_t t1 = min(t0 + la.CT, (int64_t)la.T);
+    const int64_t n = (t1 > t0 ? t1 - t0 : 0) * nseg;
+    auto issue = [&](int64_t j) {
+        const int64_t t = t0 + j / nseg;
+        const uint32_t off = (uint32_t)(j % nseg) * seg_bytes;
+        const uint32_t bytes = min(seg_bytes, row_bytes - off);
+        const int s = (int)(j % stages);
+        mbar_arrive_expect_tx(&full[s], bytes);
+        bulk_load(stage + (size_t)s * stride, da.x + t * row_bytes + off, bytes, &full[s]);
+    };
+    int64_t issued = n < stages ? n : stages;
+    if (tid == 0)
+        for (int64_t j = 0; j < issued; ++j) issue(j);
+
+    if (!layout_dev::layout_body(la, lsm)) {
+        // grid barrier timed out (reported): let the row loads in flight land, then stop
+        if (tid == 0)
+            for (int64_t j = 0; j < issued; ++j) mbar_wait(&full[j % stages], (uint32_t)((j / stages) & 1), 100000000ull);
+        return;
+    }
+
+    if (warp == 0) {
+        for (int64_t j = 0; j < n; ++j) {
+            const int s = (int)(j % stages);
+            if (!mbar_wait(&full[s], (uint32_t)((j / stages) & 1))) {
+                if (lane == 0) {
+                    atomicOr(&la.hdr->status, kDevTimeout);
+                    for (int64_t jj = j + 1; jj < issued; ++jj)
+                        mbar_wait(&full[jj % stages], (uint32_t)((jj / stages) & 1), 100000000ull);
+                }
+                bulk_wait_all<0>();
+                return;
+            }
+            __syncwarp();
+            const int64_t t = t0 + j / nseg;
+            const int sg = (int)(j % nseg);
+            const uint32_t off = (uint32_t)sg * seg_bytes;
+            const uint32_t bytes = min(seg_bytes, row_bytes - off);
+            int32_t slot = -1;
+            if (lane < K) {
+                slot = la.pair_slot[t * K + lane];
+                if (slot >= 0 && (int64_t)slot < la.capacity)
+                    bulk_store(da.recv + (int64_t)slot * row_bytes + off, stage + (size_t)s * stride, bytes);
+            }
+            if (da.x_scales != nullptr && sg == 0) {
+                // e4m3 input: carry the token's scale row to every destination
+                for (int k = 0; k < K; ++k) {
+                    const int32_t sk = __shfl_sync(0xffffffffu, slot, k);
+                    if (sk < 0 || (int64_t)sk >= la.capacity) continue;
+                    for (int b = lane; b < da.nb; b += 32)
+                        da.recv_scales[(int64_t)sk * da.nb + b] = da.x_scales[t * da.nb + b];
+                }
+            }
+            bulk_commit();
+            if (j >= 1 && issued < n) {          // refill the stage of row j-1
+                bulk_wait_read<1>();
+                __syncwarp();
+                if (lane == 0) issue(issued);
+                ++issued;
+            }
+        }
+        bulk_wait_all<0>();
+    } else if (warp == 1 && da.zero_pad) {
+        layout_dev::LayoutSmem L(lsm, la.E);
+        const int E = la.E;
+        const int64_t P = L.padpre[E];
+        const int64_t j0 = P * c / gridDim.x, j1 = P * (c + 1) / gridDim.x;
+        for (int64_t j = j0 + lane; j < j1; j += 32) {
+            int lo = 0, hi = E + 1;              // last e with padpre[e] <= j
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (L.padpre[mid] <= j) lo = mid + 1;
+                else hi = mid;
+            }
+            const int e = lo - 1;
+            const int64_t row = (int64_t)L.off[e] + L.cnt[e] + (j - L.padpre[e]);
+            if (row >= la.capacity) continue;
+            for (int sg = 0; sg < nseg; ++sg) {
+                const uint32_t off = (uint32_t)sg * seg_bytes;
+                bulk_store(da.recv + row * row_bytes + off, zero, min(seg_bytes, row_bytes - off));
+            }
+            if (da.recv_scales != nullptr)
+                for (int b = 0; b < da.nb; ++b) da.recv_scales[row * da.nb + b] = 0.0f;
+        }
+        bulk_commit();
+        bulk_wait_all<0>();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_layout_dispatch(LayoutArgs la, DispatchArgs da, int elem_bytes, cudaStream_t s) {
+    const uint32_t row_bytes = (uint32_t)da.H * (uint32_t)elem_bytes;
+    const int nseg = (int)((row_bytes + kMaxSegBytes - 1) / kMaxSegBytes);
+    const uint32_t seg_bytes = rup((row_bytes + nseg - 1) / nseg, 16);
+    const uint32_t stride = rup(seg_bytes, 128);
+    const uint32_t layout_bytes = rup((uint32_t)(layout_dev::layout_smem_ints(la.E) * sizeof(int32_t)), 128);
+    int max_smem = 0, dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    err = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (err != cudaSuccess) return err;
+    const size_t fixed = (size_t)layout_bytes + stride + 1024;
+    int stages = (int)(((size_t)max_smem - fixed - 8 * 16) / (stride + 8));
+    if (stages > 10) stages = 10;
+    if (stages < 2) {   // rows too large to stage beside the layout scratch: two kernels
+        cudaError_t e2 = launch_layout(la, da.sms, s);
+        return e2 == cudaSuccess ? launch_dispatch_copy(da, elem_bytes, s) : e2;
+    }
+    const size_t smem = (size_t)layout_bytes + (size_t)(stages + 1) * stride + (size_t)stages * 8;
+    err = cudaFuncSetAttribute(layout_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    // one chunk (CTA) per SM, whole tokens per chunk
+    const int64_t ct = ((int64_t)la.T + da.sms - 1) / da.sms;
+    la.CT = (int)ct;
+    la.C = (int)(((int64_t)la.T + ct - 1) / ct);
+    return launch_pdl(layout_dispatch_kernel, dim3(la.C), dim3(kFusedThreads), smem, s, true, la, da, row_bytes,
+                      seg_bytes, nseg, stages, layout_bytes);
+}
+
+}  // namespace ep

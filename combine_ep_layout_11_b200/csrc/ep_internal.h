@@ -12,7 +12,7 @@ struct LayoutArgs {
     const int64_t* topk_idx;
     const float* topk_weights;  // nullable
     int T, K, E, R, A;
-    int C, CT;                  // chunking
+    int C, CT;                  // chunking, chosen by launch_layout
     int64_t capacity;
     int32_t* cnt;
     int32_t* off;
@@ -26,9 +26,9 @@ struct LayoutArgs {
     int32_t* pad_rows;
 };
 
-// Two kernels: per-chunk counting (its last CTA scans the count table into
-// aligned offsets and per-chunk row bases) and slot assignment.
-cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t s);
+// One cooperative kernel: per-chunk counts, a grid barrier, the scans and the
+// slot assignment (see ep_layout.cu).
+cudaError_t launch_layout(LayoutArgs a, int sms, cudaStream_t s);
 
 struct DispatchArgs {
     const uint8_t* x;          // token rows, row_bytes each (bf16 or e4m3)
@@ -51,17 +51,25 @@ cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStre
 // bf16 -> e4m3 scatter with the per-128-column cast fused in.
 cudaError_t launch_dispatch_cast(const DispatchArgs& a, cudaStream_t s);
 
+// Layout and bf16 / e4m3 row scatter in one cooperative kernel (ep_fused.cu).
+cudaError_t launch_layout_dispatch(LayoutArgs la, DispatchArgs da, int elem_bytes, cudaStream_t s);
+
 struct CombineArgs {
     const uint16_t* y;         // bf16 [capacity][H]
     const int32_t* pair_slot;  // [T*K]
     const float* w;            // [T*K] or nullptr
     uint16_t* out;             // bf16 [T][H]
+    WsHeader* status;          // status word (timeouts)
     int T, K, H;
     int64_t capacity;
     int sms;
+    int variant;               // 0: register-staged loads, 1: TMA-staged ring (K <= 8)
 };
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+// Combine kernel choice (EP_B200_COMBINE_VARIANT=0|1 overrides the default).
+int combine_variant();
 
 cudaError_t launch_selftest_wait(WsHeader* hdr, uint64_t timeout_ns, cudaStream_t s);
 

@@ -101,8 +101,11 @@ extern "C" {
  *                                             ep_layout got no weights), 0 on padding
  *   recv_local_expert          [capacity] int32  expert id local to the
  *                                             destination rank (e mod E/R), -1 on padding
- *   workspace                  ep_workspace_bytes() bytes, 256-byte aligned;
+ *   workspace                  ep_workspace_bytes() bytes, 256-byte aligned,
+ *                              zero-filled by the caller before its first use
+ *                              (every later ep_layout leaves it ready again);
  *                              holds the device status word and scan scratch.
+ *                              One workspace serves one call at a time.
  * Rows at and beyond expert_offset[E] are not written by ep_layout.
  */
 typedef struct ep_layout_t {
@@ -147,8 +150,8 @@ int64_t ep_capacity_rows(int num_tokens, int num_topk, int num_experts, int expe
  *   layout        in: pointers, capacity, workspace; out: shape fields.
  * Device-side: an id outside [-1, E) sets EP_DEV_BAD_EXPERT and is treated as
  * -1; more than `capacity` rows sets EP_DEV_CAPACITY and rows past capacity are
- * not written.  Clears the device status word first.  Deterministic: the same
- * input gives the same bytes on every call.
+ * not written.  Replaces the device status word with the flags of this call.
+ * Deterministic: the same input gives the same bytes on every call.
  */
 int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
               int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
@@ -172,6 +175,19 @@ int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens
 int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales,
                 int hidden, int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales,
                 void* stream);
+
+/*
+ * Layout and dispatch in one call, as V2's dispatch() derives its layout from
+ * topk_idx itself (§2.1; §3.1's V1/V2 comparison).  Arguments and results are
+ * exactly those of ep_layout followed by ep_dispatch on the same handle; the
+ * handle is then reusable by ep_combine and by further ep_dispatch calls.  One
+ * kernel for bf16 or e4m3 input (its token-row reads overlap the layout work);
+ * with cast_to_fp8 the layout and the casting dispatch run as two kernels.
+ */
+int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
+                       int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
+                       ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales, int hidden,
+                       int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales, void* stream);
 
 /*
  * Combine (§2.2 weighted; §3.2 unweighted when topk_weights is NULL; §4.1

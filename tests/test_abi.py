@@ -95,6 +95,19 @@ def test_layout_rejects_small_or_misaligned_workspace(lib):
     assert lib.ep_layout(ctypes.c_void_p(0x10000), None, 8, 2, 8, 2, 1, 0, None, None) == 1
 
 
+def test_layout_dispatch_host_checks(lib):
+    p = ctypes.c_void_p(0x10000)
+    s = _handle()
+    # layout-side errors
+    assert lib.ep_layout_dispatch(p, None, 8, 2, 8, 3, 1, 0, ctypes.byref(s), p, 0, None, 256, 0, 0, p, None,
+                                  None) == 1
+    # dispatch-side errors leave the handle untouched
+    assert lib.ep_layout_dispatch(p, None, 8, 2, 8, 2, 1, 0, ctypes.byref(s), p, 0, None, 100, 0, 0, p, None,
+                                  None) == 1
+    assert s.magic == 0 and s.num_tokens == 0
+    assert lib.ep_layout_dispatch(p, None, 8, 2, 8, 2, 1, 0, None, p, 0, None, 256, 0, 0, p, None, None) == 1
+
+
 def test_dispatch_combine_host_checks(lib):
     s = _handle()                        # not filled by ep_layout: rejected
     p = ctypes.c_void_p(0x10000)

@@ -29,11 +29,15 @@ def ep():
     return m
 
 
-def _full(ep, idx, w, x, E, R, A, zero_pad=True, fp8=False):
+def _full(ep, idx, w, x, E, R, A, zero_pad=True, fp8=False, fused=False):
     ref = oracle.layout(idx, w, E, R, A)
-    lay = ep.layout(to_dev(idx), None if w is None else to_dev(w), E, R, A)
     xd = to_dev_bf16(x)
-    res = ep.dispatch(lay, xd, cast_to_fp8=fp8, do_zero_padding=zero_pad)
+    if fused:
+        lay, res = ep.layout_dispatch(to_dev(idx), None if w is None else to_dev(w), xd, E, R, A,
+                                      cast_to_fp8=fp8, do_zero_padding=zero_pad)
+    else:
+        lay = ep.layout(to_dev(idx), None if w is None else to_dev(w), E, R, A)
+        res = ep.dispatch(lay, xd, cast_to_fp8=fp8, do_zero_padding=zero_pad)
     torch.cuda.synchronize()
     assert ep.get_status(lay) == (ep.EP_OK, 0)
     Np = check_layout(lay, ref)
@@ -90,9 +94,10 @@ def test_all_unselected(ep):
     (64, 4, 16, 16, 2, 16384),     # bf16 rows of 32 KB: two bulk segments per row
     (4099, 8, 256, 1, 7, 7168),    # ragged chunking of a larger batch
 ])
-def test_shapes_bf16(ep, T, K, E, R, A, H):
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_shapes_bf16(ep, T, K, E, R, A, H, fused):
     idx, w, x = _rand(T, K, E, H, seed=T + K, drop=0.1)
-    _full(ep, idx, w, x, E, R, A)
+    _full(ep, idx, w, x, E, R, A, fused=fused)
 
 
 @pytest.mark.parametrize("T,K,E,R,A,H", [
@@ -100,19 +105,26 @@ def test_shapes_bf16(ep, T, K, E, R, A, H):
     (33, 8, 32, 1, 16, 640),       # 5 scales per row
     (64, 4, 16, 2, 1, 16384),      # the largest row the cast kernel stages
 ])
-def test_shapes_fp8(ep, T, K, E, R, A, H):
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_shapes_fp8(ep, T, K, E, R, A, H, fused):
     idx, w, x = _rand(T, K, E, H, seed=3 * T + K, drop=0.1)
-    _full(ep, idx, w, x, E, R, A, fp8=True)
+    _full(ep, idx, w, x, E, R, A, fp8=True, fused=fused)
 
 
-def test_fp8_input_passthrough(ep):
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_fp8_input_passthrough(ep, fused):
     """(e4m3, scales) input is dispatched as is: rows and scale rows move together."""
     T, K, E, R, A, H = 200, 8, 64, 4, 16, 1024
     idx, w, x = _rand(T, K, E, H, seed=11)
     q, s = oracle.cast_fp8(x)
     ref = oracle.layout(idx, w, E, R, A)
-    lay = ep.layout(to_dev(idx), to_dev(w), E, R, A)
-    rq, rs = ep.dispatch(lay, to_dev(q).view(torch.float8_e4m3fn), x_scales=to_dev(s), do_zero_padding=True)
+    xq = to_dev(q).view(torch.float8_e4m3fn)
+    if fused:
+        lay, (rq, rs) = ep.layout_dispatch(to_dev(idx), to_dev(w), xq, E, R, A, x_scales=to_dev(s),
+                                           do_zero_padding=True)
+    else:
+        lay = ep.layout(to_dev(idx), to_dev(w), E, R, A)
+        rq, rs = ep.dispatch(lay, xq, x_scales=to_dev(s), do_zero_padding=True)
     Np = int(ref["off"][-1])
     assert np.array_equal(fp8_bits(rq[:Np]), oracle.dispatch_rows(q, ref, True)[:Np])
     assert np.array_equal(f32_bits(rs[:Np]), oracle.dispatch_rows(s, ref, True)[:Np].view(np.uint32))
@@ -127,13 +139,17 @@ def test_standalone_cast(ep):
     assert np.array_equal(f32_bits(s), rs.view(np.uint32))
 
 
-def test_bad_expert_reported(ep):
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_bad_expert_reported(ep, fused):
     T, K, E, H = 32, 4, 16, 256
     idx, w, x = _rand(T, K, E, H)
     idx[3, 1] = E
     idx[7, 0] = -5
-    lay = ep.layout(to_dev(idx), to_dev(w), E, 2, 1)
-    ep.dispatch(lay, to_dev_bf16(x))
+    if fused:
+        lay, _ = ep.layout_dispatch(to_dev(idx), to_dev(w), to_dev_bf16(x), E, 2, 1)
+    else:
+        lay = ep.layout(to_dev(idx), to_dev(w), E, 2, 1)
+        ep.dispatch(lay, to_dev_bf16(x))
     code, flags = ep.get_status(lay)
     assert code == ep.EP_ERR_BAD_EXPERT and flags & 1
     # the bad entries are treated as unselected
@@ -145,11 +161,16 @@ def test_bad_expert_reported(ep):
     assert ep.get_status(lay) == (ep.EP_OK, 0)
 
 
-def test_capacity_overflow_reported(ep):
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_capacity_overflow_reported(ep, fused):
     T, K, E, H, A = 64, 4, 16, 256, 8
     idx, w, x = _rand(T, K, E, H)
-    lay = ep.layout(to_dev(idx), to_dev(w), E, 2, A, capacity=100)
-    recv = ep.dispatch(lay, to_dev_bf16(x), do_zero_padding=True)
+    if fused:
+        lay, recv = ep.layout_dispatch(to_dev(idx), to_dev(w), to_dev_bf16(x), E, 2, A, capacity=100,
+                                       do_zero_padding=True)
+    else:
+        lay = ep.layout(to_dev(idx), to_dev(w), E, 2, A, capacity=100)
+        recv = ep.dispatch(lay, to_dev_bf16(x), do_zero_padding=True)
     ep.combine(lay, recv, to_dev(w))
     code, flags = ep.get_status(lay)
     assert code == ep.EP_ERR_CAPACITY and flags & 2

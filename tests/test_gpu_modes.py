@@ -41,18 +41,27 @@ def _inputs(R, drop, seed):
 MODES = list(itertools.product([False, True], [1, 128], [False, True], [True, False], [0.0, 0.1], [1, 2, 8, 64]))
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
 @pytest.mark.parametrize("fp8,A,zero_pad,weighted,drop,R", MODES)
-def test_mode(ep, fp8, A, zero_pad, weighted, drop, R):
+def test_mode(ep, fp8, A, zero_pad, weighted, drop, R, fused):
     seed = hash((fp8, A, zero_pad, weighted, drop, R)) % (1 << 20)
     idx, w, x = _inputs(R, drop, seed)
     wt = w if weighted else None
     ref = oracle.layout(idx, wt, E, R, A)
-    lay = ep.layout(to_dev(idx), None if wt is None else to_dev(wt), E, R, A)
     xd = to_dev_bf16(x)
-    if fp8:
-        q, s = ep.dispatch(lay, xd, cast_to_fp8=True, do_zero_padding=zero_pad)
+    if fused:
+        lay, res = ep.layout_dispatch(to_dev(idx), None if wt is None else to_dev(wt), xd, E, R, A,
+                                      cast_to_fp8=fp8, do_zero_padding=zero_pad)
+        if fp8:
+            q, s = res
+        else:
+            recv = res
     else:
-        recv = ep.dispatch(lay, xd, do_zero_padding=zero_pad)
+        lay = ep.layout(to_dev(idx), None if wt is None else to_dev(wt), E, R, A)
+        if fp8:
+            q, s = ep.dispatch(lay, xd, cast_to_fp8=True, do_zero_padding=zero_pad)
+        else:
+            recv = ep.dispatch(lay, xd, do_zero_padding=zero_pad)
     Np = int(ref["off"][-1])
     y = workload.expert_outputs(dict(seed=seed, H=H), Np)
     out = ep.combine(lay, to_dev_bf16(y), None if wt is None else to_dev(wt))

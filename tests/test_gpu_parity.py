@@ -28,21 +28,31 @@ def ep():
     return m
 
 
-def _run(ep, name):
+def _run(ep, name, layout=True):
     cfg = workload.config(name)
     inp = workload.inputs(cfg)
     ref = oracle.layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"],
                         cfg["max_tokens_per_rank"])
     idx, w = to_dev(inp["topk_idx"]), to_dev(inp["topk_weights"])
     x = to_dev_bf16(inp["x"])
-    lay = ep.layout(idx, w, cfg["E"], cfg["R"], cfg["A"], cfg["max_tokens_per_rank"])
+    lay = ep.layout(idx, w, cfg["E"], cfg["R"], cfg["A"], cfg["max_tokens_per_rank"]) if layout else None
     return cfg, inp, ref, x, w, lay
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
 @pytest.mark.parametrize("name", NAMES)
-def test_layout_and_dispatch_bit_exact(ep, name):
-    cfg, inp, ref, x, w, lay = _run(ep, name)
-    if cfg["fp8"]:
+def test_layout_and_dispatch_bit_exact(ep, name, fused):
+    """ep_layout + ep_dispatch, and the single-call ep_layout_dispatch."""
+    cfg, inp, ref, x, w, lay = _run(ep, name, layout=not fused)
+    if fused:
+        lay, res = ep.layout_dispatch(to_dev(inp["topk_idx"]), w, x, cfg["E"], cfg["R"], cfg["A"],
+                                      cfg["max_tokens_per_rank"], cast_to_fp8=cfg["fp8"],
+                                      do_zero_padding=cfg["zero_pad"])
+        if cfg["fp8"]:
+            q, s = res
+        else:
+            recv = res
+    elif cfg["fp8"]:
         q, s = ep.dispatch(lay, x, cast_to_fp8=True, do_zero_padding=cfg["zero_pad"])
     else:
         recv = ep.dispatch(lay, x, do_zero_padding=cfg["zero_pad"])
