@@ -46,13 +46,12 @@ struct Chunking {
     int chunk_tokens;     // CT: tokens per chunk
 };
 
-// Chunks of whole tokens, about 256 pairs each, at most `max_chunks`
-// (kMaxChunks, or fewer when the device cannot hold that many CTAs at once).
-inline Chunking chunking(int T, int K, int max_chunks = kMaxChunks) {
+// Chunks of whole tokens, about `target_pairs` pairs each, at most `max_chunks`.
+inline Chunking chunking(int T, int K, int max_chunks, int target_pairs) {
     Chunking c{0, 0};
     if (T <= 0) return c;
     int64_t pairs = (int64_t)T * K;
-    int64_t n = (pairs + 255) / 256;
+    int64_t n = (pairs + target_pairs - 1) / target_pairs;
     if (n > max_chunks) n = max_chunks;
     if (n < 1) n = 1;
     int64_t ct = ((int64_t)T + n - 1) / n;

@@ -17,12 +17,12 @@ namespace ep {
 
 namespace {
 
-constexpr int kFusedThreads = layout_dev::kLayoutThreads;
 constexpr uint32_t kMaxSegBytes = 16384;
 
 __host__ __device__ __forceinline__ uint32_t rup(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__global__ void __launch_bounds__(kFusedThreads, 1)
+template <int NT>
+__global__ void __launch_bounds__(NT, 1)
     layout_dispatch_kernel(LayoutArgs la, DispatchArgs da, uint32_t row_bytes, uint32_t seg_bytes, int nseg,
                            int stages, uint32_t layout_bytes) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
         fence_barrier_init();
     }
-    for (uint32_t o = tid * 16u; o < stride; o += kFusedThreads * 16u)
+    for (uint32_t o = tid * 16u; o < stride; o += NT * 16u)
         *reinterpret_cast<uint4*>(zero + o) = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
     __syncthreads();
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     if (tid == 0)
         for (int64_t j = 0; j < issued; ++j) issue(j);
 
-    if (!layout_dev::layout_body(la, lsm)) {
+    if (!layout_dev::layout_body<NT>(la, lsm)) {
         // grid barrier timed out (reported): let the row loads in flight land, then stop
         if (tid == 0)
             for (int64_t j = 0; j < issued; ++j) mbar_wait(&full[j % stages], (uint32_t)((j / stages) & 1), 100000000ull);
@@ -137,9 +137,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     }
 }
 
-}  // namespace
-
-cudaError_t launch_layout_dispatch(LayoutArgs la, DispatchArgs da, int elem_bytes, cudaStream_t s) {
+template <int NT>
+cudaError_t launch_fused_nt(LayoutArgs la, DispatchArgs da, int elem_bytes, cudaStream_t s) {
     const uint32_t row_bytes = (uint32_t)da.H * (uint32_t)elem_bytes;
     const int nseg = (int)((row_bytes + kMaxSegBytes - 1) / kMaxSegBytes);
     const uint32_t seg_bytes = rup((row_bytes + nseg - 1) / nseg, 16);
@@ -150,22 +149,30 @@ cudaError_t launch_layout_dispatch(LayoutArgs la, DispatchArgs da, int elem_byte
     if (err != cudaSuccess) return err;
     err = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (err != cudaSuccess) return err;
-    const size_t fixed = (size_t)layout_bytes + stride + 1024;
-    int stages = (int)(((size_t)max_smem - fixed - 8 * 16) / (stride + 8));
-    if (stages > 10) stages = 10;
+    const size_t fixed = (size_t)layout_bytes + stride + 2048;
+    const int stages = (int)(((size_t)max_smem > fixed ? (size_t)max_smem - fixed : 0) / (stride + 8));
     if (stages < 2) {   // rows too large to stage beside the layout scratch: two kernels
         cudaError_t e2 = launch_layout(la, da.sms, s);
         return e2 == cudaSuccess ? launch_dispatch_copy(da, elem_bytes, s) : e2;
     }
-    const size_t smem = (size_t)layout_bytes + (size_t)(stages + 1) * stride + (size_t)stages * 8;
-    err = cudaFuncSetAttribute(layout_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int st = stages > 10 ? 10 : stages;
+    const size_t smem = (size_t)layout_bytes + (size_t)(st + 1) * stride + (size_t)st * 8;
+    err = cudaFuncSetAttribute(layout_dispatch_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     // one chunk (CTA) per SM, whole tokens per chunk
     const int64_t ct = ((int64_t)la.T + da.sms - 1) / da.sms;
     la.CT = (int)ct;
     la.C = (int)(((int64_t)la.T + ct - 1) / ct);
-    return launch_pdl(layout_dispatch_kernel, dim3(la.C), dim3(kFusedThreads), smem, s, true, la, da, row_bytes,
-                      seg_bytes, nseg, stages, layout_bytes);
+    return launch_pdl(layout_dispatch_kernel<NT>, dim3(la.C), dim3(NT), smem, s, true, la, da, row_bytes, seg_bytes,
+                      nseg, st, layout_bytes);
+}
+
+}  // namespace
+
+cudaError_t launch_layout_dispatch(LayoutArgs la, DispatchArgs da, int elem_bytes, cudaStream_t s) {
+    return layout_dev::layout_threads(la.E) == layout_dev::kWideThreads
+               ? launch_fused_nt<layout_dev::kWideThreads>(la, da, elem_bytes, s)
+               : launch_fused_nt<layout_dev::kNarrowThreads>(la, da, elem_bytes, s);
 }
 
 }  // namespace ep

@@ -3,7 +3,7 @@
 // count -> prefix-sum placement -> reorder stages of the Ascend dispatch on the
 // "URMA" tag page).
 //
-// One cooperative kernel, one CTA per chunk of whole tokens (at most 128, all
+// One cooperative kernel, one CTA per chunk of whole tokens (at most 64, all
 // resident at once):
 //   1. count: the chunk's per-expert histogram with warp-aggregated shared
 //      atomics (__match_any_sync groups lanes holding the same expert; one
@@ -28,27 +28,40 @@ namespace ep {
 
 namespace {
 
-__global__ void __launch_bounds__(layout_dev::kLayoutThreads) layout_kernel(LayoutArgs a) {
+// The layout alone uses at most this many chunks, so that the scan reads at
+// most 64 table rows (one batch of 16-byte loads per thread).
+constexpr int kLayoutChunks = 64;
+
+template <int NT>
+__global__ void __launch_bounds__(NT) layout_kernel(LayoutArgs a) {
     extern __shared__ __align__(16) int32_t sm[];
     pdl_wait();
     pdl_launch_dependents();
-    layout_dev::layout_body(a, sm);
+    layout_dev::layout_body<NT>(a, sm);
+}
+
+template <int NT>
+cudaError_t launch_layout_nt(LayoutArgs a, int sms, cudaStream_t s) {
+    const size_t smem = layout_dev::layout_smem_ints(a.E) * sizeof(int32_t);
+    cudaError_t err = cudaFuncSetAttribute(layout_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_kernel<NT>, NT, smem);
+    if (err != cudaSuccess) return err;
+    int max_chunks = sms * (per_sm > 0 ? per_sm : 1);
+    if (max_chunks > kLayoutChunks) max_chunks = kLayoutChunks;
+    const Chunking ch = chunking(a.T, a.K, max_chunks, NT);
+    a.C = ch.num_chunks;
+    a.CT = ch.chunk_tokens;
+    return launch_pdl(layout_kernel<NT>, dim3(a.C), dim3(NT), smem, s, true, a);
 }
 
 }  // namespace
 
 cudaError_t launch_layout(LayoutArgs a, int sms, cudaStream_t s) {
-    const size_t smem = layout_dev::layout_smem_ints(a.E) * sizeof(int32_t);
-    cudaError_t err = cudaFuncSetAttribute(layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_kernel, layout_dev::kLayoutThreads, smem);
-    if (err != cudaSuccess) return err;
-    const int resident = sms * (per_sm > 0 ? per_sm : 1);
-    const Chunking ch = chunking(a.T, a.K, resident < kMaxChunks ? resident : kMaxChunks);
-    a.C = ch.num_chunks;
-    a.CT = ch.chunk_tokens;
-    return launch_pdl(layout_kernel, dim3(a.C), dim3(layout_dev::kLayoutThreads), smem, s, true, a);
+    return layout_dev::layout_threads(a.E) == layout_dev::kWideThreads
+               ? launch_layout_nt<layout_dev::kWideThreads>(a, sms, s)
+               : launch_layout_nt<layout_dev::kNarrowThreads>(a, sms, s);
 }
 
 }  // namespace ep

@@ -7,42 +7,41 @@
 namespace ep {
 namespace layout_dev {
 
+// Threads per CTA: 512 for up to 1024 experts, 256 beyond (shared memory).
+constexpr int kWideThreads = 512;
+constexpr int kNarrowThreads = 256;
+constexpr int kWideMaxExperts = 1024;
+constexpr int kKeyRounds = 4;   // rounds of 32 pairs per warp whose expert ids stay in registers
 
+__host__ __device__ inline int layout_threads(int E) { return E <= kWideMaxExperts ? kWideThreads : kNarrowThreads; }
 
-constexpr int kLayoutThreads = 256;
-constexpr int kThreads = kLayoutThreads;
-constexpr int kWarps = kThreads / 32;
-constexpr int kGroups = 4;                 // thread groups over the chunk range in the scan
-constexpr int kGroupThreads = kThreads / kGroups;
+// Shared memory of layout_body, in ints: per-warp counts [warps][Ep], counts,
+// bases, offsets and padding prefix [Ep (+4)], scan partials [8 * threads].
+__host__ __device__ inline size_t layout_smem_ints(int E) {
+    const int Ep = round4(E), nt = layout_threads(E);
+    return (size_t)(nt / 32) * Ep + 4 * (size_t)Ep + 8 + 8 * (size_t)nt;
+}
+
+// Where layout_body leaves its per-chunk results in shared memory.
+struct LayoutSmem {
+    int32_t* wh;       // [warps][Ep] per-warp starting rows (after the assign: ends)
+    int32_t* cnt;      // [Ep] receive rows per expert
+    int32_t* base;     // [Ep] first row of each expert for this chunk
+    int32_t* off;      // [Ep + 4] aligned offsets, off[E] = rows used
+    int32_t* padpre;   // [Ep + 4] padding prefix, padpre[E] = padding rows
+    int32_t* part;     // [8 * threads] scan partials
+    __host__ __device__ LayoutSmem(int32_t* sm, int E) {
+        const int Ep = round4(E), nw = layout_threads(E) / 32;
+        wh = sm;
+        cnt = wh + (size_t)nw * Ep;
+        base = cnt + Ep;
+        off = base + Ep;
+        padpre = off + Ep + 4;
+        part = padpre + Ep + 4;
+    }
+};
 
 __device__ __forceinline__ int align_up_i(int x, int a) { return (x + a - 1) / a * a; }
-
-// Exclusive scan of one int per thread across the block; *total gets the sum.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, x, d);
-        if (lane >= d) x += y;
-    }
-    if (lane == 31) scratch[wid] = x;
-    __syncthreads();
-    if (wid == 0) {
-        int t = lane < kWarps ? scratch[lane] : 0;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            int y = __shfl_up_sync(0xffffffffu, t, d);
-            if (lane >= d) t += y;
-        }
-        if (lane < kWarps) scratch[lane] = t;
-    }
-    __syncthreads();
-    int prefix = (wid > 0 ? scratch[wid - 1] : 0) + x - v;
-    *total = scratch[kWarps - 1];
-    __syncthreads();
-    return prefix;
-}
 
 __device__ __forceinline__ int valid_expert(int64_t e, int E) { return (e >= 0 && e < E) ? (int)e : -1; }
 
@@ -55,14 +54,44 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Grid-wide barrier over `n` co-resident CTAs (generation counting, so it
-// needs no reset between calls).  Bounded: false if the other CTAs have not
-// all arrived within kWaitLimitNs.
-__device__ __forceinline__ bool grid_barrier(WsHeader* hdr, uint32_t n) {
+// Exclusive scan of one 64-bit value per thread across a CTA of NT threads;
+// *total gets the sum.  `scratch` holds NT / 32 values.
+template <int NT>
+__device__ __forceinline__ long long block_exclusive_scan64(long long v, long long* scratch, long long* total) {
+    constexpr int kW = NT / 32;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    long long x = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, x, d);
+        if (lane >= d) x += y;
+    }
+    if (lane == 31) scratch[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        long long t = lane < kW ? scratch[lane] : 0;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, t, d);
+            if (lane >= d) t += y;
+        }
+        if (lane < kW) scratch[lane] = t;
+    }
+    __syncthreads();
+    const long long prefix = (wid > 0 ? scratch[wid - 1] : 0) + x - v;
+    *total = scratch[kW - 1];
+    __syncthreads();
+    return prefix;
+}
+
+// Grid-wide barrier over `n` co-resident CTAs by generation counting (no reset
+// between calls).  `gen0` is the generation read (acquire) before this CTA's
+// arrival.  Bounded: false if the other CTAs have not all arrived within
+// kWaitLimitNs.
+__device__ __forceinline__ bool grid_barrier(WsHeader* hdr, uint32_t n, uint32_t gen0) {
     __shared__ int s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
-        const uint32_t gen0 = ld_acquire_u32(&hdr->bar_gen);
         __threadfence();
         const uint32_t arrived = atomicAdd(&hdr->bar_count, 1u);
         int ok = 1;
@@ -86,111 +115,161 @@ __device__ __forceinline__ bool grid_barrier(WsHeader* hdr, uint32_t n) {
     return s_ok != 0;
 }
 
-// The layout work of one CTA (chunk c = blockIdx.x of a.C co-resident CTAs of
-// kLayoutThreads threads).  `sm` holds layout_smem_ints(E) ints; on return
-// (true) it keeps LayoutSmem's arrays for this chunk.  False: the grid barrier
-// timed out (reported in the status word) and nothing past the count was written.
+// The layout work of one CTA: chunk c = blockIdx.x of a.C co-resident CTAs of
+// NT threads.  `sm` holds layout_smem_ints(E) ints; on success (true) the
+// LayoutSmem arrays hold this chunk's results.  False: the grid barrier timed
+// out (reported in the status word) and nothing past the counts was written.
+//
+//   count   warp w owns a contiguous run of the chunk's pairs; per round of 32
+//           pairs, __match_any_sync groups lanes holding the same expert and
+//           the group's lowest lane adds the group size to the warp's row
+//           wh[w][e]; the expert ids stay in registers for the assign;
+//   publish the chunk histogram (sum over warps, which also turns wh into
+//           per-warp starting offsets) is row c of table[C][Ep];
+//   barrier one bounded grid barrier;
+//   scan    thread groups sum table columns over disjoint chunk ranges with
+//           16-byte loads: the total per expert and the sum over chunks < c;
+//           one packed 64-bit block scan gives off[e] and the padding prefix;
+//   assign  rank = popc(peers & lanemask_lt) within the round, plus the warp's
+//           running offset, plus the chunk base: the stable token-major,
+//           k-minor order, equal to the sequential definition bit for bit;
+//   pads    receive-row metadata of the padding rows of experts c, c + C, ...
+template <int NT>
 __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
-    __shared__ int s_scratch[32];
+    constexpr int kW = NT / 32;
+    __shared__ long long s_scratch[kW];
+    __shared__ uint32_t s_gen0;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int c = blockIdx.x, C = a.C, E = a.E, Ep = round4(E), K = a.K;
-    int32_t* cnt_s = sm;                 // [Ep] histogram of this chunk, then totals
-    int32_t* base_s = cnt_s + Ep;        // [Ep] first row of each expert for this chunk
-    int32_t* off_s = base_s + Ep;        // [Ep + 4] aligned offsets
-    int32_t* padpre_s = off_s + Ep + 4;  // [Ep + 4] padding prefix
-    int32_t* wh = padpre_s + Ep + 4;     // [kWarps][Ep]: scan partials, then per-warp counts
+    LayoutSmem L(sm, E);
+    int32_t* my = L.wh + (size_t)w * Ep;
 
-    for (int e = tid; e < Ep; e += kThreads) cnt_s[e] = 0;
-    if (c == 0 && tid == 0) a.hdr->status = 0;
-    __syncthreads();
+    if (tid == 0) {
+        s_gen0 = ld_acquire_u32(&a.hdr->bar_gen);   // read before arriving at the barrier
+        if (c == 0) a.hdr->status = 0;
+    }
+    for (int e = lane; e < Ep; e += 32) my[e] = 0;
+    __syncwarp();
 
-    // ---- 1. count ----
+    // ---- count ----
     const int64_t p0 = (int64_t)c * a.CT * K;
     const int64_t p1 = min((int64_t)(c + 1) * a.CT, (int64_t)a.T) * K;
+    const int64_t per = ((p1 - p0 + kW - 1) / kW + 31) / 32 * 32;
+    const int64_t q0 = min(p0 + w * per, p1), q1 = min(q0 + per, p1);
     bool bad = false;
-    for (int64_t base = p0; base < p1; base += kThreads) {
-        const int64_t i = base + tid;
-        int key = -1;
-        if (i < p1) {
-            const int64_t e = a.topk_idx[i];
-            key = valid_expert(e, E);
-            bad |= (key < 0 && e != -1);
-        }
+    auto load_key = [&](int64_t i) -> int {
+        if (i >= q1) return -1;
+        const int64_t e = a.topk_idx[i];
+        const int key = valid_expert(e, E);
+        bad |= (key < 0 && e != -1);
+        return key;
+    };
+    auto count_round = [&](int key) {
         const uint32_t peers = __match_any_sync(0xffffffffu, key);
-        if (key >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cnt_s[key], __popc(peers));
-    }
+        if (key >= 0 && lane == __ffs(peers) - 1) my[key] += __popc(peers);
+        __syncwarp();
+    };
+    // the first rounds load together and keep their expert ids in registers
+    int keys[kKeyRounds];
+#pragma unroll
+    for (int r = 0; r < kKeyRounds; ++r) keys[r] = load_key(q0 + 32 * r + lane);
+#pragma unroll
+    for (int r = 0; r < kKeyRounds; ++r)
+        if (q0 + 32 * r < q1) count_round(keys[r]);
+    for (int64_t qb = q0 + 32 * kKeyRounds; qb < q1; qb += 32) count_round(load_key(qb + lane));
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&a.hdr->pending, kDevBadExpert);
     __syncthreads();
-    for (int e4 = tid; e4 < Ep / 4; e4 += kThreads)
-        reinterpret_cast<int4*>(a.table + (size_t)c * Ep)[e4] = reinterpret_cast<const int4*>(cnt_s)[e4];
+    // chunk histogram; the per-warp counts become per-warp starting offsets
+    for (int e = tid; e < Ep; e += NT) {
+        int run = 0;
+#pragma unroll
+        for (int j = 0; j < kW; ++j) {
+            const int v = L.wh[j * Ep + e];
+            L.wh[j * Ep + e] = run;
+            run += v;
+        }
+        L.cnt[e] = run;
+    }
+    __syncthreads();
+    for (int e4 = tid; e4 < Ep / 4; e4 += NT)
+        reinterpret_cast<int4*>(a.table + (size_t)c * Ep)[e4] = reinterpret_cast<const int4*>(L.cnt)[e4];
 
-    // ---- 2. grid barrier ----
-    if (!grid_barrier(a.hdr, (uint32_t)C)) {
+    // ---- barrier ----
+    if (!grid_barrier(a.hdr, (uint32_t)C, s_gen0)) {
         if (tid == 0) atomicOr(&a.hdr->status, kDevTimeout);
         return false;
     }
 
-    // ---- 3. scan ----
+    // ---- scan ----
     {
-        const int g = tid / kGroupThreads, q = tid % kGroupThreads;
-        const int c_lo = (int)((int64_t)C * g / kGroups), c_hi = (int)((int64_t)C * (g + 1) / kGroups);
-        int32_t* part_tot = wh;                 // [kGroups][Ep]
-        int32_t* part_pre = wh + kGroups * Ep;  // [kGroups][Ep]
-        for (int e4 = q; e4 < Ep / 4; e4 += kGroupThreads) {
-            int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
-            const int4* col = reinterpret_cast<const int4*>(a.table) + e4;
+        const int cols = Ep / 4;
+        int groups = NT / cols;
+        if (groups > 8) groups = 8;
+        if (groups < 1) groups = 1;
+        int32_t* part_tot = L.part;              // [groups][Ep]
+        int32_t* part_pre = L.part + 4 * NT;     // [groups][Ep]   (groups * Ep <= 4 * NT)
+        // one group: sums go straight to cnt / base (the chunk histogram in cnt
+        // is no longer needed once published); several: partials, then a sum
+        int32_t* dst_tot = groups == 1 ? L.cnt : part_tot;
+        int32_t* dst_pre = groups == 1 ? L.base : part_pre;
+        const int g = tid / cols;
+        if (g < groups) {
+            const int c_lo = (int)((int64_t)C * g / groups), c_hi = (int)((int64_t)C * (g + 1) / groups);
+            for (int q = tid % cols; q < cols; q += (cols < NT ? cols : NT)) {
+                int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
+                const int4* col = reinterpret_cast<const int4*>(a.table) + q;
 #pragma unroll 8
-            for (int cc = c_lo; cc < c_hi; ++cc) {
-                const int4 v = __ldcg(col + (size_t)cc * (Ep / 4));
-                tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
-                if (cc < c) { pre.x += v.x; pre.y += v.y; pre.z += v.z; pre.w += v.w; }
+                for (int cc = c_lo; cc < c_hi; ++cc) {
+                    const int4 v = __ldcg(col + (size_t)cc * cols);
+                    tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
+                    if (cc < c) { pre.x += v.x; pre.y += v.y; pre.z += v.z; pre.w += v.w; }
+                }
+                reinterpret_cast<int4*>(dst_tot + g * Ep)[q] = tot;
+                reinterpret_cast<int4*>(dst_pre + g * Ep)[q] = pre;
             }
-            reinterpret_cast<int4*>(part_tot + g * Ep)[e4] = tot;
-            reinterpret_cast<int4*>(part_pre + g * Ep)[e4] = pre;
         }
         __syncthreads();
-        for (int e = tid; e < E; e += kThreads) {
-            int tot = 0, pre = 0;
-#pragma unroll
-            for (int j = 0; j < kGroups; ++j) {
-                tot += part_tot[j * Ep + e];
-                pre += part_pre[j * Ep + e];
+        if (groups > 1) {
+            for (int e = tid; e < E; e += NT) {
+                int tot = 0, pre = 0;
+                for (int j = 0; j < groups; ++j) {
+                    tot += part_tot[j * Ep + e];
+                    pre += part_pre[j * Ep + e];
+                }
+                L.cnt[e] = tot;
+                L.base[e] = pre;
             }
-            cnt_s[e] = tot;
-            base_s[e] = pre;
+            __syncthreads();
         }
-        __syncthreads();
     }
-    // aligned offsets and padding prefix: each thread owns a run of experts
-    const int ipt = (E + kThreads - 1) / kThreads;
+    // aligned offsets (high word) and padding prefix (low word) in one scan;
+    // each thread owns a run of consecutive experts
+    const int ipt = (E + NT - 1) / NT;
     const int e0 = min(tid * ipt, E), e1 = min(e0 + ipt, E);
-    int loc_rows = 0, loc_pad = 0;
+    long long loc = 0;
     for (int e = e0; e < e1; ++e) {
-        const int al = align_up_i(cnt_s[e], a.A);
-        loc_rows += al;
-        loc_pad += al - cnt_s[e];
+        const int al = align_up_i(L.cnt[e], a.A);
+        loc += ((long long)al << 32) + (al - L.cnt[e]);
     }
-    int total_rows = 0, total_pad = 0;
-    int row_prefix = block_exclusive_scan(loc_rows, s_scratch, &total_rows);
-    int pad_prefix = block_exclusive_scan(loc_pad, s_scratch, &total_pad);
+    long long total = 0;
+    long long prefix = block_exclusive_scan64<NT>(loc, s_scratch, &total);
     for (int e = e0; e < e1; ++e) {
-        const int al = align_up_i(cnt_s[e], a.A);
-        off_s[e] = row_prefix;
-        padpre_s[e] = pad_prefix;
-        row_prefix += al;
-        pad_prefix += al - cnt_s[e];
+        const int al = align_up_i(L.cnt[e], a.A);
+        L.off[e] = (int)(prefix >> 32);
+        L.padpre[e] = (int)(prefix & 0xffffffffll);
+        L.base[e] += (int)(prefix >> 32);
+        prefix += ((long long)al << 32) + (al - L.cnt[e]);
     }
+    const int total_rows = (int)(total >> 32), total_pad = (int)(total & 0xffffffffll);
     if (tid == 0) {
-        off_s[E] = total_rows;
-        padpre_s[E] = total_pad;
+        L.off[E] = total_rows;
+        L.padpre[E] = total_pad;
     }
-    __syncthreads();
-    for (int e = tid; e < E; e += kThreads) base_s[e] += off_s[e];
     if (c == 0) {
-        for (int e = tid; e < E; e += kThreads) {
-            a.cnt[e] = cnt_s[e];
-            a.off[e] = off_s[e];
-            a.padpre[e] = padpre_s[e];
+        for (int e = tid; e < E; e += NT) {
+            a.cnt[e] = L.cnt[e];
+            a.off[e] = L.off[e];
+            a.padpre[e] = L.padpre[e];
         }
         if (tid == 0) {
             a.off[E] = total_rows;
@@ -201,89 +280,54 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
             if (flags) atomicOr(&a.hdr->status, flags);
         }
     }
-    for (int i = tid; i < kWarps * Ep; i += kThreads) wh[i] = 0;
     __syncthreads();
 
-    // ---- 4. assign ----
-    const int64_t n = p1 - p0;
-    const int64_t per = ((n + kWarps - 1) / kWarps + 31) / 32 * 32;
-    const int64_t q0 = min(p0 + w * per, p1), q1 = min(q0 + per, p1);
-    int32_t* my = wh + w * Ep;
-    for (int64_t qb = q0; qb < q1; qb += 32) {          // pass 1: per-warp counts
-        const int64_t i = qb + lane;
-        const int key = (i < q1) ? valid_expert(a.topk_idx[i], E) : -1;
-        const uint32_t peers = __match_any_sync(0xffffffffu, key);
-        if (key >= 0 && lane == __ffs(peers) - 1) my[key] += __popc(peers);
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += kThreads) {           // exclusive scan across warps
-        int run = 0;
-#pragma unroll
-        for (int j = 0; j < kWarps; ++j) {
-            const int v = wh[j * Ep + e];
-            wh[j * Ep + e] = run;
-            run += v;
-        }
-    }
-    __syncthreads();
-    const int El = E / a.R;
-    const uint32_t lt = lanemask_lt();
-    for (int64_t qb = q0; qb < q1; qb += 32) {          // pass 2: ranks, rows, inverse maps
-        const int64_t i = qb + lane;
-        const int key = (i < q1) ? valid_expert(a.topk_idx[i], E) : -1;
-        const uint32_t peers = __match_any_sync(0xffffffffu, key);
-        int slot = -1;
-        if (key >= 0) slot = base_s[key] + my[key] + __popc(peers & lt);
-        __syncwarp();
-        if (key >= 0 && lane == __ffs(peers) - 1) my[key] += __popc(peers);
-        __syncwarp();
-        if (i < q1) {
-            a.pair_slot[i] = slot;
-            if (slot >= 0 && (int64_t)slot < a.capacity) {
-                a.recv_src[slot] = (int32_t)(i / K);
-                a.recv_w[slot] = a.topk_weights ? a.topk_weights[i] : 1.0f;
-                a.recv_lexp[slot] = key % El;
+    // ---- assign ----
+    {
+        const int El = E / a.R;
+        const uint32_t lt = lanemask_lt();
+        auto assign_round = [&](int64_t qb, int key) {
+            const int64_t i = qb + lane;
+            const uint32_t peers = __match_any_sync(0xffffffffu, key);
+            int slot = -1;
+            if (key >= 0) slot = L.base[key] + my[key] + __popc(peers & lt);
+            __syncwarp();
+            if (key >= 0 && lane == __ffs(peers) - 1) my[key] += __popc(peers);
+            __syncwarp();
+            if (i < q1) {
+                a.pair_slot[i] = slot;
+                if (slot >= 0 && (int64_t)slot < a.capacity) {
+                    a.recv_src[slot] = (int32_t)(i / K);
+                    a.recv_w[slot] = a.topk_weights ? a.topk_weights[i] : 1.0f;
+                    a.recv_lexp[slot] = key % El;
+                }
             }
+        };
+#pragma unroll
+        for (int r = 0; r < kKeyRounds; ++r)
+            if (q0 + 32 * r < q1) assign_round(q0 + 32 * r, keys[r]);
+        for (int64_t qb = q0 + 32 * kKeyRounds; qb < q1; qb += 32) {
+            const int64_t i = qb + lane;
+            assign_round(qb, (i < q1) ? valid_expert(a.topk_idx[i], E) : -1);
         }
     }
 
-    // ---- 5. padding rows of the experts e = c, c + C, ... ----
+    // ---- padding rows of the experts e = c, c + C, ... ----
     for (int e = c; e < E; e += C) {
-        const int r0 = off_s[e] + cnt_s[e], r1 = off_s[e + 1];
-        const int pp = padpre_s[e];
-        for (int r = r0 + tid; r < r1; r += kThreads) {
-            a.pad_rows[pp + (r - r0)] = r;
-            if ((int64_t)r < a.capacity) {
-                a.recv_src[r] = -1;
-                a.recv_w[r] = 0.0f;
-                a.recv_lexp[r] = -1;
+        const int r0 = L.off[e] + L.cnt[e], r1 = L.off[e + 1];
+        const int pp = L.padpre[e];
+        for (int row = r0 + tid; row < r1; row += NT) {
+            a.pad_rows[pp + (row - r0)] = row;
+            if ((int64_t)row < a.capacity) {
+                a.recv_src[row] = -1;
+                a.recv_w[row] = 0.0f;
+                a.recv_lexp[row] = -1;
             }
         }
     }
     __syncthreads();
     return true;
 }
-
-// Shared memory of layout_body, in ints.
-__host__ __device__ inline size_t layout_smem_ints(int E) {
-    const int Ep = round4(E);
-    return (size_t)2 * Ep + 2 * ((size_t)Ep + 4) + (size_t)kWarps * Ep;
-}
-
-// Where layout_body leaves its per-chunk results in shared memory.
-struct LayoutSmem {
-    int32_t* cnt;      // [E] receive rows per expert
-    int32_t* base;     // [E] first row of each expert for this chunk
-    int32_t* off;      // [E+1] aligned offsets
-    int32_t* padpre;   // [E+1] padding prefix
-    __device__ LayoutSmem(int32_t* sm, int E) {
-        const int Ep = round4(E);
-        cnt = sm;
-        base = sm + Ep;
-        off = base + Ep;
-        padpre = off + Ep + 4;
-    }
-};
 
 }  // namespace layout_dev
 }  // namespace ep
