@@ -40,6 +40,7 @@ SIGNATURES = {
     "ep_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "ep_capacity_rows": (_i64, [_i, _i, _i, _i]),
     "ep_layout": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp]),
+    "ep_layout_no_alloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp]),
     "ep_dispatch": (_i, [_LP, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp]),
     "ep_layout_dispatch": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp]),
     "ep_combine": (_i, [_LP, _vp, _i, _vp, _vp, _vp]),

@@ -218,6 +218,38 @@ int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float
 int ep_cast_fp8(const void* x, int num_tokens, int hidden, void* x_fp8, float* scales,
                 void* stream);
 
+/* Size of the library-owned workspace behind ep_layout_no_alloc. */
+#define EP_NO_ALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+/*
+ * ep_layout for callers that cannot allocate device memory themselves: a plain
+ * C host program that links this library but owns no device allocator, or a
+ * process whose device memory is entirely reserved by another framework's pool
+ * that it cannot extend, so it has no buffer to offer as the workspace.  (The
+ * pages have no counterpart; this is an addition of this library.)
+ *
+ * Same arguments, checks and results as ep_layout, except that layout->workspace
+ * and layout->workspace_bytes are ignored on entry: the call uses a fixed 4 MiB
+ * array in the library's own device memory (EP_NO_ALLOC_SCRATCH_BYTES), and on
+ * success stores that array's device address in the handle, so ep_dispatch,
+ * ep_combine and ep_get_status work on the handle as usual.  The caller still
+ * provides every input and output array.  It calls no cudaMalloc or cudaFree.
+ *
+ *   - Sizes whose workspace (ep_workspace_bytes) exceeds 4 MiB are rejected
+ *     with EP_ERR_UNSUPPORTED, before anything is enqueued.
+ *   - Every GPU that loads the library holds the 4 MiB until the process exits.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (each call clears the words that must start at zero).  Calls
+ *     whose work overlaps on the GPU - from other streams or threads, or a
+ *     dispatch or combine of an older handle still pending - race on it.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current (cudaGetSymbolAddress) and caches it; make that first call
+ *     before any stream capture.
+ */
+int ep_layout_no_alloc(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
+                       int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
+                       ep_layout_t* layout, void* stream);
+
 /*
  * Synchronises `stream`, then reads the layout's device status word into
  * *device_flags (EP_DEV_* bits, 0 = no device-side error since the last
