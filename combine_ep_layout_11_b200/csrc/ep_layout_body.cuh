@@ -53,6 +53,16 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t atom_add_release_u32(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 
 // Exclusive scan of one 64-bit value per thread across a CTA of NT threads;
 // *total gets the sum.  `scratch` holds NT / 32 values.
@@ -85,19 +95,21 @@ __device__ __forceinline__ long long block_exclusive_scan64(long long v, long lo
 }
 
 // Grid-wide barrier over `n` co-resident CTAs by generation counting (no reset
-// between calls).  `gen0` is the generation read (acquire) before this CTA's
-// arrival.  Bounded: false if the other CTAs have not all arrived within
-// kWaitLimitNs.
+// between calls).  `gen0` is the generation read before this CTA's arrival
+// (every arrival of this generation happens after that read, so the value
+// cannot have moved on yet).  The CTA's writes are ordered before thread 0's
+// release arrival by __syncthreads; the last arriver publishes the new
+// generation with a release store; the others acquire it.  Bounded: false if
+// the other CTAs have not all arrived within kWaitLimitNs.
 __device__ __forceinline__ bool grid_barrier(WsHeader* hdr, uint32_t n, uint32_t gen0) {
     __shared__ int s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        const uint32_t arrived = atomicAdd(&hdr->bar_count, 1u);
+        const uint32_t arrived = atom_add_release_u32(&hdr->bar_count, 1u);
         int ok = 1;
         if (arrived == n - 1) {
             hdr->bar_count = 0;
-            __threadfence();
             st_release_u32(&hdr->bar_gen, gen0 + 1);
         } else {
             const uint64_t t0 = globaltimer_ns();
@@ -108,7 +120,6 @@ __device__ __forceinline__ bool grid_barrier(WsHeader* hdr, uint32_t n, uint32_t
                 }
             }
         }
-        __threadfence();
         s_ok = ok;
     }
     __syncthreads();
@@ -145,7 +156,7 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     int32_t* my = L.wh + (size_t)w * Ep;
 
     if (tid == 0) {
-        s_gen0 = ld_acquire_u32(&a.hdr->bar_gen);   // read before arriving at the barrier
+        s_gen0 = ld_relaxed_u32(&a.hdr->bar_gen);   // read before arriving at the barrier
         if (c == 0) a.hdr->status = 0;
     }
     for (int e = lane; e < Ep; e += 32) my[e] = 0;
@@ -275,9 +286,6 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
             a.off[E] = total_rows;
             a.padpre[E] = total_pad;
             a.hdr->num_pad = total_pad;
-            uint32_t flags = atomicExch(&a.hdr->pending, 0u);
-            if ((int64_t)total_rows > a.capacity) flags |= kDevCapacity;
-            if (flags) atomicOr(&a.hdr->status, flags);
         }
     }
     __syncthreads();
@@ -324,6 +332,11 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
                 a.recv_lexp[row] = -1;
             }
         }
+    }
+    if (c == 0 && tid == 0) {   // fold the flags of this call into the status word
+        uint32_t flags = atomicExch(&a.hdr->pending, 0u);
+        if ((int64_t)total_rows > a.capacity) flags |= kDevCapacity;
+        if (flags) atomicOr(&a.hdr->status, flags);
     }
     __syncthreads();
     return true;
