@@ -82,6 +82,25 @@ def ncu_traffic(kernel, wl):
 
 
 # --------------------------------------------------------------------------
+# multi-rank host logic: every rank runs its own replica
+# --------------------------------------------------------------------------
+def max_over_ranks(x, dist, device):
+    """The max of a per-rank value over all ranks (step times are taken as the
+    slowest rank's); the identity on one rank."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, ms_per_step):
+    """Whole-job tokens/s: the tokens of all ranks over the (max) step time."""
+    return tokens_per_rank * world / (ms_per_step * 1e-3)
+
+
+# --------------------------------------------------------------------------
 # clocks sampled during the timed region
 # --------------------------------------------------------------------------
 class ClockSampler:
@@ -243,7 +262,7 @@ def run_ours(args, rank, world, local_rank):
     if dist:
         dist.barrier()
     clock_info = clocks.stop() if clocks else None
-    ms_per_step = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    ms_per_step = max_over_ranks(np.mean([e[0].elapsed_time(e[1]) for e in evs]), dist, dev)
     # per-kernel breakdown: the same K steps again with events between the kernels
     evk = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     for i in range(args.steps):
@@ -251,18 +270,11 @@ def run_ours(args, rank, world, local_rank):
         step(evk[i])
     torch.cuda.synchronize(dev)
     per = np.array([[evk[i][j].elapsed_time(evk[i][j + 1]) for j in range(3)] for i in range(args.steps)])
-    if dist:
-        tt = torch.tensor([ms_per_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_per_step = float(tt.item())
 
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush)
-        if dist:
-            tt = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e["ms_per_step"] = float(tt.item())
+        e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dist, dev)
 
     if rank != 0:
         if dist:
@@ -284,7 +296,7 @@ def run_ours(args, rank, world, local_rank):
     kernels_us["combine"] = round(k_ms[2] * 1e3, 2)
     kernels_us["note"] = "second pass with events between the calls"
     disp_gbs = top_bytes / (top_ms * 1e-3) / 1e9
-    value = T * world / (ms_per_step * 1e-3)
+    value = job_throughput(T, world, ms_per_step)
     line = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -322,7 +334,7 @@ def run_ours(args, rank, world, local_rank):
     if clock_info:
         line["clocks"] = clock_info
     if e2e:
-        line["e2e"] = {"value": round(T * world / (e2e["ms_per_step"] * 1e-3), 1), "unit": "tokens/s",
+        line["e2e"] = {"value": round(job_throughput(T, world, e2e["ms_per_step"]), 1), "unit": "tokens/s",
                        "ms_per_step": round(e2e["ms_per_step"], 4),
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
     if world == 1 and not args.no_cpu_baseline:

@@ -1,0 +1,77 @@
+"""The N > 1 path of bench.py, on the CPU with world-size-2 `gloo` processes.
+
+With several GPUs every rank runs its own replica of the single-GPU path (there
+is no data-path collective); the process group only provides the barrier and
+the max over ranks of the step time, and the job throughput sums the tokens of
+all ranks.  These host-side pieces are exercised here without a GPU."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % port, rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        step_ms = [0.25, 0.40][rank]                 # rank 1 is the slower one
+        m = bench.max_over_ranks(step_ms, dist, "cpu")
+        value = bench.job_throughput(4096, world, m)
+        dist.barrier()
+        out.put((rank, m, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_job_throughput_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    mp.start_processes(_worker, args=(2, port, q), nprocs=2, join=True, start_method="spawn")
+    got = sorted(q.get(timeout=30) for _ in range(2))
+    for rank, m, value in got:
+        assert m == pytest.approx(0.40)                          # every rank sees the slowest rank's time
+        assert value == pytest.approx(2 * 4096 / 0.40e-3)       # tokens of both ranks over that time
+
+
+def test_single_rank_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(0.3, None, "cpu") == pytest.approx(0.3)
+    assert bench.job_throughput(100, 1, 1.0) == pytest.approx(1e5)
+
+
+@pytest.mark.slow
+def test_reference_arm_under_torchrun_prints_one_line():
+    """`bench.py --impl reference` launched as 2 ranks: rank 0 alone times the
+    CPU oracle and prints the one JSON line; the other rank exits 0."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1", "--gpus", "2"]
+    res = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300,
+                         env=dict(os.environ, OMP_NUM_THREADS="1"))
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [json.loads(l) for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["n_gpus"] == 2 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
