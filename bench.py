@@ -62,21 +62,28 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
-def source_hash(path):
-    with open(os.path.join(ROOT, path), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel, wl):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+    """DRAM bytes (read + write) per launch from the committed ncu capture
+    (profiles/traffic.json), if it was taken on the current kernel sources;
+    else None."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return None
     rec = d.get("%s@%s" % (kernel, wl))
-    if not rec or rec.get("source_sha") != source_hash(rec["source"]):
+    try:
+        if not rec or rec.get("source_sha") != source_hash(rec["sources"]):
+            return None
+    except OSError:
         return None
     return rec.get("dram_bytes_per_launch")
 
