@@ -1,8 +1,8 @@
 """Benchmark: MoE dispatch + combine on one B200 (or N independent replicas).
 
-One step = the whole hot path over one batch: ep_layout (count + assign
-kernels), ep_dispatch (with the fused FP8 cast for the FP8 workload) and
-ep_combine, on the default workload "prefill_bf16": T = 4096 tokens,
+One step = the whole hot path over one batch: ep_layout (one kernel),
+ep_dispatch (with the fused FP8 cast for the FP8 workload) and ep_combine, on
+the default workload "prefill_bf16": T = 4096 tokens,
 H = 7168 bf16, 256 experts, top-8, R = 8 virtual ranks, expert_alignment 128,
 zero padding, skewed (Zipf s = 1.2 bias) gate.  Inputs are seeded synthetic
 (workload/), resident in HBM before timing; the combine input ("expert
@@ -48,8 +48,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
-    p.add_argument("--separate", action="store_true",
-                   help="ep_layout + ep_dispatch as two calls instead of the single ep_layout_dispatch")
+    p.add_argument("--fused", action="store_true",
+                   help="the single ep_layout_dispatch call instead of ep_layout + ep_dispatch")
     return p.parse_args()
 
 
@@ -222,7 +222,7 @@ def run_ours(args, rank, world, local_rank):
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        if args.separate:
+        if not args.fused:
             ep.layout(idx, w, E, R, A, cfg["max_tokens_per_rank"], out=lay)
             if evs:
                 evs[1].record(stream)
@@ -292,7 +292,7 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind = measured_peaks()
     k_ms = per.mean(axis=0)   # layout, dispatch, combine (fused: layout+dispatch, -, combine)
     total_bytes = nbytes["layout"] + nbytes["dispatch"] + nbytes["combine"]
-    if args.separate:
+    if not args.fused:
         top_kernel = "dispatch_cast_kernel" if fp8 else "dispatch_copy_kernel"
         top_bytes, top_ms = nbytes["dispatch"], k_ms[1]
         kernels_us = {"layout": round(k_ms[0] * 1e3, 2), "dispatch": round(k_ms[1] * 1e3, 2)}
@@ -335,7 +335,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": round(disp_gbs / peak, 4),
                      "traffic": ncu_traffic(top_kernel, cfg["name"]),
                      "algorithmic_bytes_per_launch": top_bytes},
-        "gpu_launches": args.steps * (2 if (not args.separate and not fp8) else 3),
+        "gpu_launches": args.steps * (2 if (args.fused and not fp8) else 3),
         "wall_s_timed_region": round(wall, 4),
     }
     if clock_info:
@@ -374,9 +374,13 @@ def run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush):
         d_w.copy_(h_w, non_blocking=True)
         d_x.copy_(h_x, non_blocking=True)
         xb = d_x.view(torch.bfloat16)
-        ep.layout_dispatch(d_idx, d_w, xb, cfg["E"], cfg["R"], cfg["A"], cfg["max_tokens_per_rank"],
-                           cast_to_fp8=fp8, do_zero_padding=cfg["zero_pad"], out_layout=lay, out=recv,
-                           out_scales=recv_s)
+        if args.fused:
+            ep.layout_dispatch(d_idx, d_w, xb, cfg["E"], cfg["R"], cfg["A"], cfg["max_tokens_per_rank"],
+                               cast_to_fp8=fp8, do_zero_padding=cfg["zero_pad"], out_layout=lay, out=recv,
+                               out_scales=recv_s)
+        else:
+            ep.layout(d_idx, d_w, cfg["E"], cfg["R"], cfg["A"], cfg["max_tokens_per_rank"], out=lay)
+            ep.dispatch(lay, xb, cast_to_fp8=fp8, do_zero_padding=cfg["zero_pad"], out=recv, out_scales=recv_s)
         ep.combine(lay, y, d_w, out=d_out)
         h_out.copy_(d_out.view(torch.int16), non_blocking=True)
         if e1:

@@ -2,7 +2,6 @@
 // checks, then kernel launches on the caller's stream.  No allocation, no
 // state kept between calls, no host synchronisation except ep_get_status.
 #include <limits.h>
-#include <stdlib.h>
 
 #include "ep_internal.h"
 
@@ -127,13 +126,6 @@ int prepare_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, cons
 
 }  // namespace
 
-namespace ep {
-int combine_variant() {
-    const char* v = getenv("EP_B200_COMBINE_VARIANT");
-    return (v && (v[0] == '1' || v[0] == '2')) ? v[0] - '0' : 0;
-}
-}  // namespace ep
-
 extern "C" {
 
 int ep_version(void) { return EP_B200_VERSION; }
@@ -235,7 +227,6 @@ int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float
     a.H = H;
     a.capacity = layout->capacity;
     a.status = header(layout);
-    a.variant = ep::combine_variant();
     if ((rc = device_sms(&a.sms)) != EP_OK) return rc;
     return ep::launch_combine(a, (cudaStream_t)stream) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }

@@ -8,8 +8,9 @@
 // in fp32 from +0, every step __fmul_rn then __fadd_rn (never contracted into
 // an FMA), so the result is the same bits whatever the launch shape.  The
 // kernel is bound by HBM reads: K rows of 2H bytes in, one row out per token.
-// A work item is (token, 32*V 16-byte columns); a warp issues all K row loads
-// of its item before accumulating, so each lane keeps 8*V loads in flight.
+// A work item is (token, 32*V 16-byte columns); a warp issues the loads of KB
+// rows of its item together before summing them, so each lane keeps KB*V
+// loads in flight, and every row is read in contiguous 32*V*16-byte pieces.
 // Padding rows are never read.
 #include <cuda_bf16.h>
 
@@ -20,7 +21,6 @@ namespace ep {
 namespace {
 
 constexpr int kCombineThreads = 256;
-constexpr int kKBatch = 8;
 
 __device__ __forceinline__ void accumulate8(float (&acc)[8], uint4 v, float w) {
     const uint32_t u[4] = {v.x, v.y, v.z, v.w};
@@ -36,7 +36,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-template <int V, int kMinBlocks>
+// V: 16-byte columns per lane per row (a row segment of V * 512 bytes per
+// item); KB: rows whose loads are issued together before they are summed.
+template <int V, int kMinBlocks, int KB>
 __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(CombineArgs a) {
     const int lane = threadIdx.x & 31;
     const int64_t gw = ((int64_t)blockIdx.x * kCombineThreads + threadIdx.x) >> 5;
@@ -77,10 +79,10 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[v][i] = 0.0f;
 
-        for (int k0 = 0; k0 < K; k0 += kKBatch) {
-            uint4 rows[kKBatch][V];
+        for (int k0 = 0; k0 < K; k0 += KB) {
+            uint4 rows[KB][V];
 #pragma unroll
-            for (int kk = 0; kk < kKBatch; ++kk) {
+            for (int kk = 0; kk < KB; ++kk) {
                 const int k = k0 + kk;
                 const int slot = __shfl_sync(0xffffffffu, my_slot, k & 31);
                 const bool use = (k < K) && slot >= 0;
@@ -92,7 +94,7 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
                 }
             }
 #pragma unroll
-            for (int kk = 0; kk < kKBatch; ++kk) {
+            for (int kk = 0; kk < KB; ++kk) {
                 const int k = k0 + kk;
                 const int slot = __shfl_sync(0xffffffffu, my_slot, k & 31);
                 const float w = __shfl_sync(0xffffffffu, my_w, k & 31);
@@ -118,131 +120,6 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
     }
 }
 
-// ---------------------------------------------------------------------------
-// TMA-staged variant for K <= 8: the item is (token, 2 KB column segment).  A
-// producer warp bulk-loads the K rows' segments into a stage of a ring in
-// shared memory (one mbarrier per stage counts the bytes); four consumer warps
-// reduce the stage in ascending k, one 16-byte column per thread, and store the
-// bf16 result.  The ring keeps many row segments in flight per SM without
-// holding them in registers.
-// ---------------------------------------------------------------------------
-constexpr int kStageK = 8;
-constexpr int kSegVec = 128;                 // 16-byte columns per segment (2 KB of bf16)
-constexpr int kSegBytes = kSegVec * 16;
-constexpr int kConsumerWarps = 4;
-constexpr int kTmaThreads = 32 * (1 + kConsumerWarps);
-
-struct StageMeta {
-    float w[kStageK];
-    int32_t valid;   // bit k: row k was loaded
-    int32_t pad[7];
-};
-
-__global__ void __launch_bounds__(kTmaThreads) combine_tma_kernel(CombineArgs a, int stages) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t* ring = smem;                                                   // [stages][kStageK][kSegBytes]
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * kStageK * kSegBytes);
-    uint64_t* empty = full + stages;
-    StageMeta* meta = reinterpret_cast<StageMeta*>(empty + stages);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int K = a.K, HV = a.H / 8;
-    const int nseg = (HV + kSegVec - 1) / kSegVec;
-    const int64_t items = (int64_t)a.T * nseg;
-    const int64_t G = gridDim.x, first = blockIdx.x;
-    const int64_t n = first < items ? (items - first + G - 1) / G : 0;
-    const uint32_t row_bytes = (uint32_t)a.H * 2u;
-
-    if (tid == 0) {
-        for (int s = 0; s < stages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        fence_barrier_init();
-    }
-    __syncthreads();
-    pdl_wait();
-    pdl_launch_dependents();
-
-    if (warp == 0) {
-        // producer; the (slot, weight) of lane k for item j+1 is loaded while
-        // item j is issued, so no item waits on a dependent global load
-        auto fetch = [&](int64_t j, int32_t& slot, float& w) {
-            slot = -1;
-            w = 1.0f;
-            if (j < n && lane < K) {
-                const int64_t t = (first + j * G) / nseg;
-                slot = a.pair_slot[t * K + lane];
-                if (a.w) w = a.w[t * K + lane];
-            }
-        };
-        int32_t next_slot;
-        float next_w;
-        fetch(0, next_slot, next_w);
-        for (int64_t j = 0; j < n; ++j) {
-            const int s = (int)(j % stages);
-            int32_t slot = next_slot;
-            float w = next_w;
-            fetch(j + 1, next_slot, next_w);
-            if ((int64_t)slot >= a.capacity) slot = -1;
-            if (!mbar_wait(&empty[s], (uint32_t)(((j / stages) & 1) ^ 1))) {
-                if (lane == 0) atomicOr(&a.status->status, kDevTimeout);
-                break;
-            }
-            const int64_t item = first + j * G;
-            const int g = (int)(item % nseg);
-            const uint32_t bytes = (uint32_t)min(kSegVec, HV - g * kSegVec) * 16u;
-            const uint32_t valid = __ballot_sync(0xffffffffu, slot >= 0);
-            if (lane < kStageK) meta[s].w[lane] = w;
-            if (lane == 0) meta[s].valid = (int32_t)valid;
-            __syncwarp();   // the metadata writes are ordered before lane 0's release-arrive
-            if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes * __popc(valid));
-            __syncwarp();
-            if (slot >= 0)
-                bulk_load(ring + ((size_t)s * kStageK + lane) * kSegBytes,
-                          a.y + (int64_t)slot * (row_bytes / 2) + (int64_t)g * kSegVec * 8, bytes, &full[s]);
-        }
-        return;
-    }
-
-    // consumers
-    const int ct = tid - 32;   // 0 .. 127: one 16-byte column of the segment
-    for (int64_t j = 0; j < n; ++j) {
-        const int s = (int)(j % stages);
-        const bool ok = mbar_wait(&full[s], (uint32_t)((j / stages) & 1));
-        if (!ok) {
-            if (ct == 0) atomicOr(&a.status->status, kDevTimeout);
-            return;
-        }
-        const int64_t item = first + j * G;
-        const int64_t t = item / nseg;
-        const int g = (int)(item % nseg);
-        const int col = g * kSegVec + ct;
-        const uint32_t valid = (uint32_t)meta[s].valid;
-        float acc[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-        if (col < HV) {
-#pragma unroll
-            for (int k = 0; k < kStageK; ++k) {
-                if (valid & (1u << k)) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(ring + ((size_t)s * kStageK + k) * kSegBytes + ct * 16);
-                    accumulate8(acc, v, meta[s].w[k]);
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[s])) : "memory");
-        if (col < HV) {
-            uint4 o;
-            o.x = pack_bf16x2(acc[0], acc[1]);
-            o.y = pack_bf16x2(acc[2], acc[3]);
-            o.z = pack_bf16x2(acc[4], acc[5]);
-            o.w = pack_bf16x2(acc[6], acc[7]);
-            st_v4(reinterpret_cast<uint4*>(a.out) + t * HV + col, o);
-        }
-    }
-}
-
 __global__ void selftest_wait_kernel(WsHeader* hdr, uint64_t timeout_ns) {
     __shared__ __align__(8) uint64_t bar;
     if (threadIdx.x == 0) {
@@ -256,19 +133,10 @@ __global__ void selftest_wait_kernel(WsHeader* hdr, uint64_t timeout_ns) {
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
-    if (a.variant == 1 && a.K <= kStageK) {
-        const int stages = 6;
-        const size_t smem = (size_t)stages * kStageK * kSegBytes + 2 * stages * 8 + stages * sizeof(StageMeta);
-        cudaError_t err =
-            cudaFuncSetAttribute(combine_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-        int per_sm = 0;
-        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_tma_kernel, kTmaThreads, smem);
-        if (err != cudaSuccess) return err;
-        if (per_sm < 1) per_sm = 1;
-        return launch_pdl(combine_tma_kernel, dim3(a.sms * per_sm), dim3(kTmaThreads), smem, s, false, a, stages);
-    }
-    auto kernel = a.variant == 2 ? combine_kernel<1, 3> : combine_kernel<2, 2>;
+    // items of 2 KB per row, rows loaded 4 at a time: contiguous 2 KB reads per
+    // row keep DRAM pages open (measured faster than 1 KB items with 8 rows in
+    // flight, and than staging the rows through shared memory with TMA)
+    auto kernel = combine_kernel<4, 2, 4>;
     int blocks_per_sm = 0;
     cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kernel, kCombineThreads, 0);
     if (err != cudaSuccess) return err;

@@ -63,13 +63,10 @@ struct CombineArgs {
     int T, K, H;
     int64_t capacity;
     int sms;
-    int variant;               // 0: register-staged loads, 1: TMA-staged ring (K <= 8)
 };
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 
-// Combine kernel choice (EP_B200_COMBINE_VARIANT=0|1 overrides the default).
-int combine_variant();
 
 cudaError_t launch_selftest_wait(WsHeader* hdr, uint64_t timeout_ns, cudaStream_t s);
 
