@@ -71,7 +71,9 @@ def _load(path):
     L.orc_dequant_fp8.restype = None
     L.orc_dequant_fp8.argtypes = [vp, vp, i64, i64, vp]
     L.orc_combine.restype = None
-    L.orc_combine.argtypes = [vp, i64, vp, vp, i64, i64, vp]
+    L.orc_combine.argtypes = [vp, i64, vp, vp, i64, i64, vp, vp, vp]
+    L.orc_accumulate_recv_stats.restype = None
+    L.orc_accumulate_recv_stats.argtypes = [vp, i64, vp]
     L.orc_routing_table.restype = i32
     L.orc_routing_table.argtypes = [vp, i64, vp, i64, i64, i64, i64, i64,
                                     vp, vp, vp, vp, vp, vp, vp, vp]
@@ -181,12 +183,13 @@ def dequant_fp8(q, scales):
     return out
 
 
-def combine(y_bf16, pair_slot, topk_weights):
+def combine(y_bf16, pair_slot, topk_weights, bias0=None, bias1=None):
     """Ordered weighted reduction ([API] §2.2, §3.2, §4.1): bf16 [T, H].
 
     ``y_bf16`` holds the expert outputs, one bf16 row per receive row (uint16
     bits, [rows, H]); ``pair_slot`` [T, K] names the row of each pair; NULL
-    (None) weights mean unit weights.
+    (None) weights mean unit weights; ``bias0`` / ``bias1`` (bf16 bits [T, H])
+    are the optional output bias, the sum's starting value.
     """
     y_bf16 = np.ascontiguousarray(y_bf16, dtype=np.uint16)
     pair_slot = np.ascontiguousarray(pair_slot, dtype=np.int32)
@@ -197,9 +200,24 @@ def combine(y_bf16, pair_slot, topk_weights):
     if topk_weights is not None:
         topk_weights = np.ascontiguousarray(topk_weights, dtype=np.float32)
         assert topk_weights.shape == (T, K)
+    biases = []
+    for b in (bias0, bias1):
+        if b is not None:
+            b = np.ascontiguousarray(b, dtype=np.uint16)
+            assert b.shape == (T, H)
+        biases.append(b)
     out = np.zeros((T, H), np.uint16)
-    lib().orc_combine(_p(y_bf16), H, _p(pair_slot), _p(topk_weights), T, K, _p(out))
+    lib().orc_combine(_p(y_bf16), H, _p(pair_slot), _p(topk_weights), T, K, _p(biases[0]), _p(biases[1]),
+                      _p(out))
     return out
+
+
+def accumulate_recv_stats(stats, cnt):
+    """cumulative_local_expert_recv_stats ([API] §2.1, §3.3): stats += cnt (int32)."""
+    stats = np.array(stats, dtype=np.int32, copy=True)
+    cnt = np.ascontiguousarray(cnt, dtype=np.int32)
+    lib().orc_accumulate_recv_stats(_p(cnt), cnt.size, _p(stats))
+    return stats
 
 
 def routing_table(gate_indices, gate_weights, num_tokens, top_k, local_start, local_end):
@@ -266,5 +284,5 @@ def step(inp, cfg):
         recv = (dispatch_rows(q, lay, cfg["zero_pad"]), dispatch_rows(s, lay, cfg["zero_pad"]))
     else:
         recv = dispatch_rows(inp["x"], lay, cfg["zero_pad"])
-    out = combine(inp["y"], lay["pair_slot"], inp["topk_weights"])
+    out = combine(inp["y"], lay["pair_slot"], inp["topk_weights"], inp.get("bias0"), inp.get("bias1"))
     return lay, recv, out

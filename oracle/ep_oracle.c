@@ -26,7 +26,8 @@
  *  - amax is clamped below at 1e-4 so an all-zero block gets a finite scale;
  *  - the quotient x / scale is one correctly rounded binary32 division and the
  *    E4M3 conversion rounds to nearest-even and saturates to +-448;
- *  - combine starts from 0, skips -1 entries, and for k = 0..K-1 in order does
+ *  - combine starts from 0 (or from the output bias: bias0, plus bias1 as one
+ *    rounded sum), skips -1 entries, and for k = 0..K-1 in order does
  *    acc = acc + (w * y) with two binary32 roundings (no fused multiply-add),
  *    then rounds acc to bf16 to nearest-even; NULL weights mean w = 1;
  *  - the source rank of token t is t / (T / R); expert e lives on rank e / (E / R).
@@ -308,18 +309,27 @@ void orc_dequant_fp8(const uint8_t* q, const float* scales, int64_t T, int64_t H
 /* Combine: ordered weighted reduction          [API] §2.2, §3.2, §4.1 */
 /* ------------------------------------------------------------------ */
 
-/* out[t] = bf16( sum over k = 0..K-1 with pair_slot[t, k] >= 0 of w[t, k] * y[slot] )
- * accumulated in binary32 in ascending k, starting from 0.  Each step is one
+/* out[t] = bf16( init[t] + sum over k = 0..K-1 with pair_slot[t, k] >= 0 of w[t, k] * y[slot] )
+ * accumulated in binary32 in ascending k.  The starting value init[t] is 0,
+ * or the output bias ([API] §2.2 combine() bias, §4.1 refs.combine
+ * initial_value): float(bias0[t]), and with a second bias
+ * float(bias0[t]) + float(bias1[t]) as one rounded sum.  Each term is one
  * rounded product followed by one rounded sum.  NULL weights: w = 1. */
 void orc_combine(const uint16_t* y, int64_t H, const int32_t* pair_slot,
-                 const float* topk_weights, int64_t T, int64_t K, uint16_t* out)
+                 const float* topk_weights, int64_t T, int64_t K,
+                 const uint16_t* bias0, const uint16_t* bias1, uint16_t* out)
 {
     float* acc = (float*)malloc((size_t)(H > 0 ? H : 1) * sizeof(float));
     if (!acc)
         return;
     for (int64_t t = 0; t < T; t++) {
-        for (int64_t h = 0; h < H; h++)
+        for (int64_t h = 0; h < H; h++) {
             acc[h] = 0.0f;
+            if (bias0)
+                acc[h] = bf16_to_f32(bias0[t * H + h]);
+            if (bias1)
+                acc[h] = acc[h] + bf16_to_f32(bias1[t * H + h]);
+        }
         for (int64_t k = 0; k < K; k++) {
             int32_t slot = pair_slot[t * K + k];
             if (slot < 0)
@@ -335,6 +345,15 @@ void orc_combine(const uint16_t* y, int64_t H, const int32_t* pair_slot,
             out[t * H + h] = f32_to_bf16_rne(acc[h]);
     }
     free(acc);
+}
+
+/* Running per-expert receive counts across calls ([API] §2.1 and §3.3:
+ * cumulative_local_expert_recv_stats; rank r's local experts are entries
+ * [r*E/R, (r+1)*E/R)): stats[e] += cnt[e]. */
+void orc_accumulate_recv_stats(const int32_t* cnt, int64_t E, int32_t* stats)
+{
+    for (int64_t e = 0; e < E; e++)
+        stats[e] += cnt[e];
 }
 
 /* ------------------------------------------------------------------ */

@@ -391,29 +391,42 @@ def pin_combine_golden():
         y = np.array(case["y_bits"], np.uint16)
         ps = np.array(case["pair_slot"], np.int32)
         w = None if case["weights"] is None else np.array(case["weights"], np.float32)
-        out = oracle.combine(y, ps, w)
+        b0 = np.array(case["bias0_bits"], np.uint16) if "bias0_bits" in case else None
+        b1 = np.array(case["bias1_bits"], np.uint16) if "bias1_bits" in case else None
+        out = oracle.combine(y, ps, w, b0, b1)
         assert out.tolist() == case["out_bits"], case["name"]
+
+
+def _rand_bf16(rng, shape, lo=-60, hi=60):
+    """Random signs and mantissas, exponents in [lo, hi]: no overflow, no subnormals."""
+    return ((rng.integers(0, 2, shape, dtype=np.uint16) << 15)
+            | (rng.integers(127 + lo, 127 + hi + 1, shape, dtype=np.uint16) << 7)
+            | rng.integers(0, 128, shape, dtype=np.uint16)).astype(np.uint16)
 
 
 def pin_combine_fp64_bound(seed=13):
     rng = np.random.default_rng(seed)
-    for (T, K, rows, H, weighted) in [(64, 8, 300, 64, True), (32, 4, 50, 40, False), (16, 1, 16, 8, True)]:
+    for (T, K, rows, H, weighted, nbias) in [(64, 8, 300, 64, True, 0), (32, 4, 50, 40, False, 0),
+                                             (16, 1, 16, 8, True, 0), (48, 8, 200, 32, True, 1),
+                                             (24, 4, 80, 16, False, 2)]:
         # random signs and mantissas, exponents in [-60, 60]: no overflow, no subnormal products
-        y = ((rng.integers(0, 2, (rows, H), dtype=np.uint16) << 15)
-             | (rng.integers(127 - 60, 127 + 61, (rows, H), dtype=np.uint16) << 7)
-             | rng.integers(0, 128, (rows, H), dtype=np.uint16)).astype(np.uint16)
+        y = _rand_bf16(rng, (rows, H))
         ps = rng.integers(-1, rows, (T, K)).astype(np.int32)
         w = (rng.standard_normal((T, K)) * 2).astype(np.float32) if weighted else None
-        out = oracle.combine(y, ps, w)
+        biases = [_rand_bf16(rng, (T, H)) for _ in range(nbias)] + [None] * (2 - nbias)
+        out = oracle.combine(y, ps, w, biases[0], biases[1])
         yf = oracle.bf16_to_f32(y).astype(np.float64)
         wf = np.ones((T, K)) if w is None else w.astype(np.float64)
         sel = ps >= 0
         terms = np.where(sel[:, :, None], wf[:, :, None] * yf[np.maximum(ps, 0)], 0.0)
-        exact = terms.sum(axis=1)
-        mag = np.abs(terms).sum(axis=1)
+        bsum = sum(oracle.bf16_to_f32(b).astype(np.float64) for b in biases if b is not None)
+        exact = terms.sum(axis=1) + bsum
+        mag = np.abs(terms).sum(axis=1) + sum(np.abs(oracle.bf16_to_f32(b).astype(np.float64))
+                                              for b in biases if b is not None)
         got = oracle.bf16_to_f32(out).astype(np.float64)
         u = 2.0 ** -24
-        gamma = 2 * K * u / (1 - 2 * K * u)
+        n = 2 * K + nbias                 # K products, K + nbias - 1 additions, at most
+        gamma = n * u / (1 - n * u)
         bound = 2.0 ** -8 * np.abs(exact) * (1 + gamma) + (1 + 2.0 ** -8) * gamma * mag + 1e-40
         assert np.all(np.abs(got - exact) <= bound)
 
@@ -448,10 +461,25 @@ def pin_combine_permutation():
     assert np.array_equal(oracle.combine(y, ps, None), y[ps[:, 0]])
 
 
+def pin_recv_stats():
+    """cumulative_local_expert_recv_stats over two calls = the two histograms summed."""
+    rng = np.random.default_rng(23)
+    E = 16
+    stats = rng.integers(0, 100, E).astype(np.int32)
+    start = stats.copy()
+    seen = np.zeros(E, np.int64)
+    for _ in range(2):
+        idx = rng.integers(-1, E, (40, 4)).astype(np.int64)
+        lay = oracle.layout(idx, None, E, 4, 8)
+        stats = oracle.accumulate_recv_stats(stats, lay["cnt"])
+        seen += np.bincount(idx[idx >= 0], minlength=E)
+    assert np.array_equal(stats, start + seen)
+
+
 ALL_PINS = [
     pin_layout_exhaustive, pin_layout_random, pin_layout_invariants_workloads, pin_layout_errors,
     pin_routing_table_golden, pin_dispatch_rows, pin_e4m3_decode_table, pin_e4m3_encode_vs_torch,
     pin_e4m3_saturation, pin_fp8_golden_block, pin_cast_vs_torch, pin_cast_roundtrip,
     pin_bf16_rounding, pin_combine_golden, pin_combine_fp64_bound, pin_combine_identity,
-    pin_combine_permutation,
+    pin_combine_permutation, pin_recv_stats,
 ]

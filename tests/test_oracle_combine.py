@@ -21,3 +21,7 @@ def test_combine_identity_experts_reproduce_x():
 
 def test_combine_k1_is_permutation():
     pins.pin_combine_permutation()
+
+
+def test_recv_stats_accumulate_over_calls():
+    pins.pin_recv_stats()

@@ -1,6 +1,6 @@
 """Planted mistakes in the oracle must each fail at least one pin.
 
-Each case below edits a copy of ``oracle/ep_oracle.c`` (the committed source is
+Each case below makes one or more edits to a copy of ``oracle/ep_oracle.c`` (the committed source is
 never touched), builds it into a temporary library, routes the oracle through it
 and runs the pins until one fails.  A mistake that no pin catches means a pin is
 missing.  Mistakes that would write out of bounds in the mutated C code are not
@@ -27,6 +27,15 @@ MUTANTS = {
     "combine_fused_multiply_add": (
         "float product = w * bf16_to_f32(row[h]);\n                acc[h] = acc[h] + product;",
         "acc[h] = fmaf(w, bf16_to_f32(row[h]), acc[h]);"),
+    "combine_ignores_bias0": ("acc[h] = bf16_to_f32(bias0[t * H + h]);", "acc[h] = 0.0f;"),
+    "combine_ignores_bias1": ("acc[h] = acc[h] + bf16_to_f32(bias1[t * H + h]);", "acc[h] = acc[h];"),
+    "combine_bias_added_last": [
+        ("            if (bias0)\n                acc[h] = bf16_to_f32(bias0[t * H + h]);\n"
+         "            if (bias1)\n                acc[h] = acc[h] + bf16_to_f32(bias1[t * H + h]);\n", ""),
+        ("            out[t * H + h] = f32_to_bf16_rne(acc[h]);",
+         "            out[t * H + h] = f32_to_bf16_rne(acc[h] + (bias0 ? bf16_to_f32(bias0[t * H + h]) : 0.0f)\n"
+         "                                             + (bias1 ? bf16_to_f32(bias1[t * H + h]) : 0.0f));")],
+    "stats_overwrite": ("stats[e] += cnt[e];", "stats[e] = cnt[e];"),
     "bf16_truncates": ("if (dropped > 0x8000u || (dropped == 0x8000u && (upper & 1u)))", "if (0)"),
     "bf16_ties_away": ("if (dropped > 0x8000u || (dropped == 0x8000u && (upper & 1u)))",
                        "if (dropped >= 0x8000u)"),
@@ -76,10 +85,15 @@ def _run_pins():
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_planted_mistake(name, source, tmp_path):
-    old, new = MUTANTS[name]
-    assert source.count(old) == 1, "mutation anchor for %s must occur exactly once" % name
+    edits = MUTANTS[name]
+    if isinstance(edits, tuple):
+        edits = [edits]
+    mutated = source
+    for old, new in edits:
+        assert mutated.count(old) == 1, "mutation anchor for %s must occur exactly once" % name
+        mutated = mutated.replace(old, new)
     src = tmp_path / "mutant.c"
-    src.write_text(source.replace(old, new))
+    src.write_text(mutated)
     lib = oracle_build.build(str(src), str(tmp_path / "libmutant.so"), force=True,
                              extra_flags=["-Wno-error", "-w"])
     with oracle.use_library(lib):
