@@ -67,9 +67,13 @@ def _load(path):
     L.orc_dispatch_rows.restype = None
     L.orc_dispatch_rows.argtypes = [vp, i64, i64, i64, vp, vp, vp, i64, i32, vp]
     L.orc_cast_fp8.restype = None
-    L.orc_cast_fp8.argtypes = [vp, i64, i64, vp, vp]
+    L.orc_cast_fp8.argtypes = [vp, i64, i64, i64, ctypes.c_int, vp, vp]
     L.orc_dequant_fp8.restype = None
-    L.orc_dequant_fp8.argtypes = [vp, vp, i64, i64, vp]
+    L.orc_dequant_fp8.argtypes = [vp, vp, i64, i64, i64, vp]
+    L.orc_ue8m0_encode.restype = ctypes.c_int
+    L.orc_ue8m0_encode.argtypes = [vp, i64, vp]
+    L.orc_ue8m0_decode.restype = None
+    L.orc_ue8m0_decode.argtypes = [vp, i64, vp]
     L.orc_combine.restype = None
     L.orc_combine.argtypes = [vp, i64, vp, vp, i64, i64, vp, vp, vp]
     L.orc_accumulate_recv_stats.restype = None
@@ -162,24 +166,63 @@ def dispatch_rows(x_rows, lay, do_zero_padding, fill=0xA5):
     return recv.view(x_rows.dtype).reshape((cap,) + tail)
 
 
-def cast_fp8(x_bf16):
-    """Per-128-column-block E4M3 cast ([API] §4.2): returns (q uint8 [T, H], scales f32 [T, H/128])."""
+def cast_fp8(x_bf16, per_row=False, round_scale=False):
+    """E4M3 cast ([API] §4.2): returns (q uint8 [T, H], scales f32 [T, H/128]).
+
+    ``per_row``: one scale per token row ([T, 1]) as §4.2's per_token_cast_to_fp8
+    prints it, instead of one per 128-column block.  ``round_scale``: each
+    scale rounded up to a power of two ([API] §3.3 round_scale)."""
     x_bf16 = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     T, H = x_bf16.shape
     assert H % 128 == 0, "FP8 cast needs H % 128 == 0"
+    group = H if per_row else 128
     q = np.zeros((T, H), np.uint8)
-    s = np.zeros((T, H // 128), np.float32)
-    lib().orc_cast_fp8(_p(x_bf16), T, H, _p(q), _p(s))
+    s = np.zeros((T, H // group), np.float32)
+    lib().orc_cast_fp8(_p(x_bf16), T, H, group, int(bool(round_scale)), _p(q), _p(s))
     return q, s
 
 
 def dequant_fp8(q, scales):
-    """Dequantisation ([API] §4.2): float(q) * scale in binary32."""
+    """Dequantisation ([API] §4.2): float(q) * scale in binary32; the group
+    width is H / scales.shape[1] (128, or H for per-row scales)."""
     q = np.ascontiguousarray(q, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.float32)
     T, H = q.shape
+    group = H // scales.shape[1] if scales.ndim == 2 else H
     out = np.zeros((T, H), np.float32)
-    lib().orc_dequant_fp8(_p(q), _p(scales), T, H, _p(out))
+    lib().orc_dequant_fp8(_p(q), _p(scales), T, H, group, _p(out))
+    return out
+
+
+def ue8m0_encode(scales):
+    """Power-of-two fp32 scales as UE8M0 bytes ([API] §3.3 use_ue8m0): 2^k -> k + 127."""
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    out = np.zeros(scales.shape, np.uint8)
+    rc = lib().orc_ue8m0_encode(_p(scales), scales.size, _p(out))
+    if rc != 0:
+        raise OracleError(rc, "UE8M0 needs power-of-two scales")
+    return out
+
+
+def ue8m0_decode(b):
+    """UE8M0 bytes to fp32: b -> 2^(b - 127)."""
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    out = np.zeros(b.shape, np.float32)
+    lib().orc_ue8m0_decode(_p(b), b.size, _p(out))
+    return out
+
+
+def scales_col_major(scales):
+    """TMA-aligned column-major placement of row-major scales [rows, G]
+    ([API] §2.1 use_tma_aligned_col_major_sf): entry (r, g) goes to g * ld + r
+    with ld = rows rounded up to 16 bytes of elements; returns [G, ld], the
+    padding entries zero."""
+    scales = np.asarray(scales)
+    rows, G = scales.shape
+    per16 = 16 // scales.dtype.itemsize
+    ld = (rows + per16 - 1) // per16 * per16
+    out = np.zeros((G, ld), scales.dtype)
+    out[:, :rows] = scales.T
     return out
 
 

@@ -22,7 +22,9 @@
  *         reconciliation, prefix-sum placement and output reordering.
  *
  * Readings where the pages are silent (all listed in the design notes):
- *  - scales are per 128-column block of a token row, fp32, row-major [T, H/128];
+ *  - scales are per 128-column block of a token row, fp32, row-major [T, H/128]
+ *    (per row, [T], as a variant); round_scale rounds a scale up to a power
+ *    of two; UE8M0 stores such a scale as its biased exponent byte;
  *  - amax is clamped below at 1e-4 so an all-zero block gets a finite scale;
  *  - the quotient x / scale is one correctly rounded binary32 division and the
  *    E4M3 conversion rounds to nearest-even and saturates to +-448;
@@ -264,19 +266,37 @@ void orc_dispatch_rows(const uint8_t* x, int64_t row_bytes, int64_t T, int64_t K
 /* FP8 cast                                     [API] §4.2              */
 /* ------------------------------------------------------------------ */
 
-/* For each token t and each block b of 128 columns:
- *   amax = max |x[t, 128b .. 128b+127]|, clamped below at 1e-4
- *   s    = amax / 448                     (binary32 division)
- *   q[j] = e4m3(x[t, j] / s)              (binary32 division, RNE, saturating)
- *   scales[t, b] = s                                                     */
-void orc_cast_fp8(const uint16_t* x, int64_t T, int64_t H, uint8_t* q, float* scales)
+/* Smallest power of two >= s, for a positive normal s: the round_scale option
+ * ([API] §3.3 low_latency_dispatch: round_scale rounds the scale to a power of
+ * two; reading: upwards, so that |x / s| <= 448 still holds and nothing
+ * saturates).  frexpf writes s = m * 2^e with m in [0.5, 1); s is itself a
+ * power of two exactly when m == 0.5. */
+static float pow2_ceil(float s)
 {
-    int64_t nb = H / 128;
+    int e;
+    float m = frexpf(s, &e);
+    if (m == 0.5f)
+        return s;
+    return ldexpf(1.0f, e);
+}
+
+/* For each token t and each group g of `group` columns (group = 128: one scale
+ * per 128-column block; group = H: one scale per row, [API] §4.2
+ * per_token_cast_to_fp8):
+ *   amax = max |x[t, g*group .. g*group + group - 1]|, clamped below at 1e-4
+ *   s    = amax / 448                     (binary32 division)
+ *   s    = pow2_ceil(s)                   (only with round_pow2)
+ *   q[j] = e4m3(x[t, j] / s)              (binary32 division, RNE, saturating)
+ *   scales[t, g] = s                      (row-major [T, H / group])        */
+void orc_cast_fp8(const uint16_t* x, int64_t T, int64_t H, int64_t group, int round_pow2, uint8_t* q,
+                  float* scales)
+{
+    int64_t ng = H / group;
     for (int64_t t = 0; t < T; t++) {
-        for (int64_t b = 0; b < nb; b++) {
-            const uint16_t* blk = x + t * H + b * 128;
+        for (int64_t g = 0; g < ng; g++) {
+            const uint16_t* blk = x + t * H + g * group;
             float amax = 0.0f;
-            for (int j = 0; j < 128; j++) {
+            for (int64_t j = 0; j < group; j++) {
                 float a = fabsf(bf16_to_f32(blk[j]));
                 if (a > amax)
                     amax = a;
@@ -284,23 +304,49 @@ void orc_cast_fp8(const uint16_t* x, int64_t T, int64_t H, uint8_t* q, float* sc
             if (amax < 1e-4f)
                 amax = 1e-4f;
             float s = amax / 448.0f;
-            scales[t * nb + b] = s;
-            for (int j = 0; j < 128; j++) {
+            if (round_pow2)
+                s = pow2_ceil(s);
+            scales[t * ng + g] = s;
+            for (int64_t j = 0; j < group; j++) {
                 float quotient = bf16_to_f32(blk[j]) / s;
-                q[t * H + b * 128 + j] = orc_e4m3_encode(quotient);
+                q[t * H + g * group + j] = orc_e4m3_encode(quotient);
             }
         }
     }
 }
 
-/* Dequantisation: value = float(q) * s, one binary32 multiplication. */
-void orc_dequant_fp8(const uint8_t* q, const float* scales, int64_t T, int64_t H, float* out)
+/* UE8M0 ([API] §3.3 use_ue8m0): an unsigned 8-bit exponent, value 2^(b - 127),
+ * no sign and no mantissa.  A power-of-two scale s = 2^k is stored as
+ * b = k + 127; frexpf gives s = 0.5 * 2^e, so k = e - 1.  Returns ORC_OK, or
+ * ORC_ERR_INVALID_ARG if some s is not a power of two in [2^-127, 2^127]. */
+int orc_ue8m0_encode(const float* s, int64_t n, uint8_t* out)
 {
-    int64_t nb = H / 128;
+    for (int64_t i = 0; i < n; i++) {
+        int e;
+        float m = frexpf(s[i], &e);
+        if (m != 0.5f || e - 1 < -127 || e - 1 > 127)
+            return ORC_ERR_INVALID_ARG;
+        out[i] = (uint8_t)(e - 1 + 127);
+    }
+    return ORC_OK;
+}
+
+/* value of a UE8M0 byte: 2^(b - 127) (b = 255 is not produced by the cast). */
+void orc_ue8m0_decode(const uint8_t* b, int64_t n, float* out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = ldexpf(1.0f, (int)b[i] - 127);
+}
+
+/* Dequantisation: value = float(q) * s, one binary32 multiplication, with the
+ * scale of the value's group (group = 128 or H, as in orc_cast_fp8). */
+void orc_dequant_fp8(const uint8_t* q, const float* scales, int64_t T, int64_t H, int64_t group, float* out)
+{
+    int64_t ng = H / group;
     for (int64_t t = 0; t < T; t++)
         for (int64_t j = 0; j < H; j++) {
             float v = orc_e4m3_decode(q[t * H + j]);
-            float s = scales[t * nb + j / 128];
+            float s = scales[t * ng + j / group];
             out[t * H + j] = v * s;
         }
 }

@@ -371,6 +371,111 @@ def pin_cast_roundtrip():
     assert np.all(qb[amax >= 1e-4] == 448.0)
 
 
+def _torch_cast_variant(xb, per_row, round_scale):
+    """The pages' formula through torch, with the group width and the
+    power-of-two rounding of the scale written with torch's log2 / ceil / exp2."""
+    T, H = xb.shape
+    g = H if per_row else 128
+    xf = torch.from_numpy(oracle.bf16_to_f32(xb).reshape(T, H // g, g))
+    amax = xf.abs().amax(dim=2).clamp_min(1e-4)
+    s = amax / 448.0
+    if round_scale:
+        s = torch.exp2(torch.ceil(torch.log2(s.double()))).float()
+    q = (xf / s.unsqueeze(2)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return q.reshape(T, H).numpy(), s.numpy()
+
+
+def _variant_inputs():
+    xb = cast_test_inputs()
+    # blocks whose amax / 448 is exactly a power of two (amax = 1.75 * 2^j)
+    rng = np.random.default_rng(29)
+    x5 = (rng.uniform(-1, 1, (16, 1024)) * 1.75).astype(np.float32)
+    x5[:, ::128] = np.float32(1.75) * np.exp2(rng.integers(-20, 20, (16, 8))).astype(np.float32)
+    return np.concatenate([xb, workload.to_bf16_bits(x5)])
+
+
+def pin_cast_variants_vs_torch():
+    xb = _variant_inputs()
+    for per_row in (False, True):
+        for round_scale in (False, True):
+            q, s = oracle.cast_fp8(xb, per_row=per_row, round_scale=round_scale)
+            tq, ts = _torch_cast_variant(xb, per_row, round_scale)
+            assert np.array_equal(s.view(np.uint32), ts.view(np.uint32)), (per_row, round_scale)
+            assert np.array_equal(q, tq), (per_row, round_scale)
+
+
+def pin_round_scale_properties():
+    """A rounded scale is a power of two, not below amax / 448 and below twice it."""
+    xb = _variant_inputs()
+    for per_row in (False, True):
+        _, s0 = oracle.cast_fp8(xb, per_row=per_row)
+        _, s1 = oracle.cast_fp8(xb, per_row=per_row, round_scale=True)
+        m, _ = np.frexp(s1.astype(np.float64))
+        assert np.all(m == 0.5)
+        assert np.all(s1 >= s0) and np.all(s1.astype(np.float64) / 2 < s0)
+
+
+def pin_fp8_variants_golden():
+    g = _golden("fp8_variants_example.json")
+    x = np.zeros((1, g["H"]), np.float32)
+    x[0, :len(g["block0_values"])] = g["block0_values"]
+    x[0, 128:128 + len(g["block1_values"])] = g["block1_values"]
+    xb = workload.to_bf16_bits(x)
+    assert np.array_equal(oracle.bf16_to_f32(xb), x), "golden values must be bf16-exact"
+    n0, n1 = len(g["block0_values"]), len(g["block1_values"])
+    q, s = oracle.cast_fp8(xb, round_scale=True)
+    assert q[0, :n0].tolist() == g["block_round"]["block0_codes"]
+    assert q[0, 128:128 + n1].tolist() == g["block_round"]["block1_codes"]
+    assert s[0].tolist() == g["block_round"]["scales"]
+    assert oracle.ue8m0_encode(s)[0].tolist() == g["block_round"]["ue8m0"]
+    q, s = oracle.cast_fp8(xb, per_row=True, round_scale=True)
+    assert s.shape == (1, 1) and float(s[0, 0]) == g["row_round"]["scale"]
+    assert q[0, :n0].tolist() == g["block_round"]["block0_codes"]
+    assert q[0, 128:128 + n1].tolist() == g["row_round"]["block1_codes"]
+    assert int(oracle.ue8m0_encode(s)[0, 0]) == g["row_round"]["ue8m0"]
+
+
+def pin_ue8m0():
+    b = np.arange(255, dtype=np.uint8)
+    v = oracle.ue8m0_decode(b)
+    assert np.array_equal(v.astype(np.float64), np.exp2(b.astype(np.float64) - 127))
+    assert np.array_equal(oracle.ue8m0_encode(v), b)
+    for bad in (3.0, 0.75, 1.5 * 2.0 ** -20):
+        try:
+            oracle.ue8m0_encode(np.array([bad], np.float32))
+        except oracle.OracleError:
+            continue
+        raise AssertionError("UE8M0 accepted a scale that is not a power of two: %r" % bad)
+
+
+def pin_cast_variants_roundtrip():
+    xb = _variant_inputs()
+    T, H = xb.shape
+    x = oracle.bf16_to_f32(xb).astype(np.float64)
+    for per_row in (False, True):
+        for round_scale in (False, True):
+            q, s = oracle.cast_fp8(xb, per_row=per_row, round_scale=round_scale)
+            d = oracle.dequant_fp8(q, s).astype(np.float64)
+            sb = np.repeat(s.astype(np.float64), H // s.shape[1], axis=1)
+            bound = np.maximum(np.abs(x) * 2.0 ** -4, sb * 2.0 ** -10) * (1 + 2.0 ** -18) + sb * 2.0 ** -30
+            assert np.all(np.abs(d - x) <= bound), (per_row, round_scale)
+            assert np.all(np.abs(oracle.e4m3_decode(q)) <= 448.0)
+
+
+def pin_scales_col_major():
+    rng = np.random.default_rng(31)
+    for rows, G, dt in [(1, 1, np.float32), (5, 3, np.float32), (8, 56, np.float32), (17, 2, np.uint8),
+                        (32, 7, np.uint8)]:
+        sc = rng.integers(1, 200, (rows, G)).astype(dt)
+        cm = oracle.scales_col_major(sc)
+        per16 = 16 // np.dtype(dt).itemsize
+        assert cm.shape[0] == G and cm.shape[1] % per16 == 0 and rows <= cm.shape[1] < rows + per16
+        flat = cm.reshape(-1)
+        for r in range(rows):
+            for g in range(G):
+                assert flat[g * cm.shape[1] + r] == sc[r, g]
+
+
 def pin_bf16_rounding():
     rng = np.random.default_rng(9)
     u = rng.integers(0, 1 << 32, 400000, dtype=np.uint64).astype(np.uint32)
@@ -482,4 +587,6 @@ ALL_PINS = [
     pin_e4m3_saturation, pin_fp8_golden_block, pin_cast_vs_torch, pin_cast_roundtrip,
     pin_bf16_rounding, pin_combine_golden, pin_combine_fp64_bound, pin_combine_identity,
     pin_combine_permutation, pin_recv_stats,
+    pin_cast_variants_vs_torch, pin_round_scale_properties, pin_fp8_variants_golden, pin_ue8m0,
+    pin_cast_variants_roundtrip, pin_scales_col_major,
 ]

@@ -49,8 +49,14 @@ MUTANTS = {
     "cast_reciprocal_multiply": ("float quotient = bf16_to_f32(blk[j]) / s;",
                                  "float quotient = bf16_to_f32(blk[j]) * (1.0f / s);"),
     "cast_no_amax_clamp": ("if (amax < 1e-4f)\n                amax = 1e-4f;", ""),
-    "cast_amax_half_block": ("for (int j = 0; j < 128; j++) {\n                float a = fabsf(",
-                             "for (int j = 0; j < 64; j++) {\n                float a = fabsf("),
+    "cast_amax_half_block": ("for (int64_t j = 0; j < group; j++) {\n                float a = fabsf(",
+                             "for (int64_t j = 0; j < group / 2; j++) {\n                float a = fabsf("),
+    "cast_row_amax_first_block": ("for (int64_t j = 0; j < group; j++) {\n                float a = fabsf(",
+                                  "for (int64_t j = 0; j < 128; j++) {\n                float a = fabsf("),
+    "pow2_rounds_down": ("    return ldexpf(1.0f, e);\n}", "    return ldexpf(1.0f, e - 1);\n}"),
+    "pow2_doubles_exact_powers": ("    if (m == 0.5f)\n        return s;\n", ""),
+    "pow2_ignored": ("            if (round_pow2)\n                s = pow2_ceil(s);\n", ""),
+    "ue8m0_off_by_one": ("out[i] = (uint8_t)(e - 1 + 127);", "out[i] = (uint8_t)(e + 127);"),
     "layout_k_major": (
         "for (int64_t t = 0; t < T; t++) {\n        for (int64_t k = 0; k < K; k++) {\n"
         "            int64_t i = t * K + k;\n            int64_t e = topk_idx[i];\n            if (e < 0) {",
