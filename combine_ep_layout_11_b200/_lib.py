@@ -30,6 +30,7 @@ class EpLayout(ctypes.Structure):
         ("num_max_tokens_per_rank", ctypes.c_int32),
         ("magic", ctypes.c_uint32),
         ("reserved", ctypes.c_uint32),
+        ("cumulative_local_expert_recv_stats", ctypes.c_void_p),
     ]
 
 
@@ -43,7 +44,7 @@ SIGNATURES = {
     "ep_layout_no_alloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp]),
     "ep_dispatch": (_i, [_LP, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp]),
     "ep_layout_dispatch": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp]),
-    "ep_combine": (_i, [_LP, _vp, _i, _vp, _vp, _vp]),
+    "ep_combine": (_i, [_LP, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "ep_cast_fp8": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "ep_get_status": (_i, [_LP, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "ep_selftest_bounded_wait": (_i, [_LP, _u64, _vp]),

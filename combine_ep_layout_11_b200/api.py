@@ -96,6 +96,7 @@ class Layout:
         s.workspace_bytes = nbytes
         s.capacity = self.capacity
         self.struct = s
+        self.cumulative_local_expert_recv_stats = None
 
     def ref(self):
         return ctypes.byref(self.struct)
@@ -110,11 +111,22 @@ class Layout:
         return self.expert_offset[::El]
 
 
+def _set_recv_stats(lay, stats):
+    """Point the handle at the caller's running per-expert receive counts (or at none)."""
+    if stats is not None:
+        assert stats.dtype == torch.int32 and stats.is_contiguous() and stats.numel() == lay.num_experts
+        assert stats.device == lay.device
+    lay.cumulative_local_expert_recv_stats = stats       # kept alive with the handle
+    lay.struct.cumulative_local_expert_recv_stats = _ptr(stats)
+
+
 def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment=1,
-           num_max_tokens_per_rank=0, capacity=None, out=None):
+           num_max_tokens_per_rank=0, capacity=None, out=None, cumulative_local_expert_recv_stats=None):
     """Compute the routing layout of ``topk_idx`` [T, K] int64 (-1 = unselected).
 
     ``out`` may be a ``Layout`` of the same sizes to reuse its memory.
+    ``cumulative_local_expert_recv_stats``: int32 [E] on the device or None;
+    when given, this call's per-expert receive counts are added to it (§2.1).
     """
     L = _lib.load()
     assert topk_idx.dtype == torch.int64 and topk_idx.dim() == 2 and topk_idx.is_contiguous()
@@ -126,6 +138,7 @@ def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment=1,
         assert (out.num_tokens, out.num_topk, out.num_experts) == (T, K, num_experts), "layout size mismatch"
     lay = out if out is not None else Layout(T, K, num_experts, num_ranks, expert_alignment,
                                              topk_idx.device, capacity, num_max_tokens_per_rank)
+    _set_recv_stats(lay, cumulative_local_expert_recv_stats)
     _check(L.ep_layout(_ptr(topk_idx), _ptr(topk_weights), T, K, num_experts, num_ranks,
                        expert_alignment, num_max_tokens_per_rank, lay.ref(), _stream(topk_idx.device)),
            "ep_layout")
@@ -159,7 +172,8 @@ def dispatch(lay, x, x_scales=None, cast_to_fp8=False, do_zero_padding=False, ou
 
 def layout_dispatch(topk_idx, topk_weights, x, num_experts, num_ranks, expert_alignment=1,
                     num_max_tokens_per_rank=0, x_scales=None, cast_to_fp8=False, do_zero_padding=False,
-                    capacity=None, out_layout=None, out=None, out_scales=None):
+                    capacity=None, out_layout=None, out=None, out_scales=None,
+                    cumulative_local_expert_recv_stats=None):
     """Layout and dispatch in one call (§2.1: V2's dispatch() derives the layout
     from topk_idx).  Same results as ``layout`` then ``dispatch``; returns
     ``(layout, recv_x)`` or ``(layout, (recv_x, recv_scales))`` for FP8 output."""
@@ -174,6 +188,7 @@ def layout_dispatch(topk_idx, topk_weights, x, num_experts, num_ranks, expert_al
         assert (out_layout.num_tokens, out_layout.num_topk, out_layout.num_experts) == (T, K, num_experts)
     lay = out_layout if out_layout is not None else Layout(T, K, num_experts, num_ranks, expert_alignment,
                                                            topk_idx.device, capacity, num_max_tokens_per_rank)
+    _set_recv_stats(lay, cumulative_local_expert_recv_stats)
     H = x.shape[1]
     fp8_in = x.dtype == torch.float8_e4m3fn
     assert fp8_in or x.dtype == torch.bfloat16
@@ -191,17 +206,31 @@ def layout_dispatch(topk_idx, topk_weights, x, num_experts, num_ranks, expert_al
     return lay, ((out, out_scales) if fp8_out else out)
 
 
-def combine(lay, y, topk_weights=None, out=None):
-    """Weighted (or, with no weights, plain) ordered reduction back to [T, H] bf16 (§2.2)."""
+def combine(lay, y, topk_weights=None, bias=None, out=None):
+    """Weighted (or, with no weights, plain) ordered reduction back to [T, H] bf16 (§2.2).
+
+    ``bias``: None, a bf16 [T, H] tensor, or a pair of them (§2.2 combine():
+    0, 1 or 2 output biases); the fp32 sum starts from bias0 (+ bias1).
+    """
     L = _lib.load()
     assert y.dtype == torch.bfloat16 and y.dim() == 2 and y.is_contiguous()
     H = y.shape[1]
     if topk_weights is not None:
         assert topk_weights.dtype == torch.float32 and topk_weights.is_contiguous()
+    if bias is None:
+        biases = (None, None)
+    elif isinstance(bias, torch.Tensor):
+        biases = (bias, None)
+    else:
+        assert len(bias) == 2, "bias is a tensor or a pair of tensors"
+        biases = tuple(bias)
+    for b in biases:
+        if b is not None:
+            assert b.dtype == torch.bfloat16 and b.is_contiguous() and b.shape == (lay.num_tokens, H)
     if out is None:
         out = torch.empty((lay.num_tokens, H), dtype=torch.bfloat16, device=y.device)
-    _check(L.ep_combine(lay.ref(), _ptr(y), H, _ptr(topk_weights), _ptr(out), _stream(y.device)),
-           "ep_combine")
+    _check(L.ep_combine(lay.ref(), _ptr(y), H, _ptr(topk_weights), _ptr(biases[0]), _ptr(biases[1]),
+                        _ptr(out), _stream(y.device)), "ep_combine")
     return out
 
 

@@ -44,7 +44,8 @@ int prepare_layout(const int64_t* topk_idx, const float* topk_weights, int T, in
     if (!aligned(topk_idx, 8) || !aligned(topk_weights, 4) || !aligned(layout->num_recv_tokens_per_expert, 4) ||
         !aligned(layout->expert_offset, 4) || !aligned(layout->pair_slot, 4) ||
         !aligned(layout->recv_src_token, 4) || !aligned(layout->recv_weight, 4) ||
-        !aligned(layout->recv_local_expert, 4) || !aligned(layout->workspace, 256))
+        !aligned(layout->recv_local_expert, 4) || !aligned(layout->workspace, 256) ||
+        !aligned(layout->cumulative_local_expert_recv_stats, 4))
         return EP_ERR_INVALID_ARG;
     const ep::WsLayout ws = ep::ws_layout(T, K, E, A);
     if (layout->workspace_bytes < ws.total) return EP_ERR_INVALID_ARG;
@@ -74,6 +75,7 @@ int prepare_layout(const int64_t* topk_idx, const float* topk_weights, int T, in
     a->table = reinterpret_cast<int32_t*>(wsb + ws.table_off);
     a->padpre = reinterpret_cast<int32_t*>(wsb + ws.padpre_off);
     a->pad_rows = reinterpret_cast<int32_t*>(wsb + ws.padrows_off);
+    a->stats = layout->cumulative_local_expert_recv_stats;
     return EP_OK;
 }
 
@@ -208,19 +210,24 @@ int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int n
     return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
-int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float* topk_weights, void* out,
-               void* stream) {
+int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float* topk_weights, const void* bias0,
+               const void* bias1, void* out, void* stream) {
     int rc = check_handle(layout);
     if (rc != EP_OK) return rc;
     const int H = hidden, T = layout->num_tokens;
     if (H <= 0 || H % 8 != 0) return EP_ERR_INVALID_ARG;
     if (T > 0 && (!y || !out)) return EP_ERR_INVALID_ARG;
-    if (!aligned(y, 16) || !aligned(out, 16) || !aligned(topk_weights, 4)) return EP_ERR_INVALID_ARG;
+    if (bias1 && !bias0) return EP_ERR_INVALID_ARG;
+    if (!aligned(y, 16) || !aligned(out, 16) || !aligned(topk_weights, 4) || !aligned(bias0, 16) ||
+        !aligned(bias1, 16))
+        return EP_ERR_INVALID_ARG;
     if (T == 0) return EP_OK;
     ep::CombineArgs a;
     a.y = reinterpret_cast<const uint16_t*>(y);
     a.pair_slot = layout->pair_slot;
     a.w = topk_weights;
+    a.bias0 = reinterpret_cast<const uint16_t*>(bias0);
+    a.bias1 = reinterpret_cast<const uint16_t*>(bias1);
     a.out = reinterpret_cast<uint16_t*>(out);
     a.T = T;
     a.K = layout->num_topk;

@@ -3,10 +3,12 @@
 // §3.2 Buffer.combine() plain sum when no weights are given, §4.1 refs.py
 // ordered_accumulate: one fixed accumulation order for bitwise determinism).
 //
-//   out[t] = bf16_rne( sum_{k ascending, pair_slot[t,k] >= 0} w[t,k] * y[pair_slot[t,k]] )
+//   out[t] = bf16_rne( init[t] + sum_{k ascending, pair_slot[t,k] >= 0} w[t,k] * y[pair_slot[t,k]] )
 //
-// in fp32 from +0, every step __fmul_rn then __fadd_rn (never contracted into
-// an FMA), so the result is the same bits whatever the launch shape.  The
+// in fp32, every step __fmul_rn then __fadd_rn (never contracted into an FMA),
+// so the result is the same bits whatever the launch shape.  init[t] is +0, or
+// the output bias of §2.2 combine() (bias0, or bias0 + bias1 rounded once),
+// the initial value of the reference accumulation in §4.1.  The
 // kernel is bound by HBM reads: K rows of 2H bytes in, one row out per token.
 // A work item is (token, 32*V 16-byte columns); a warp issues the loads of KB
 // rows of its item together before summing them, so each lane keeps KB*V
@@ -31,14 +33,30 @@ __device__ __forceinline__ void accumulate8(float (&acc)[8], uint4 v, float w) {
     }
 }
 
+// acc := float(b0), then acc := acc + float(b1) (one rounded sum) when two biases
+__device__ __forceinline__ void init_bias8(float (&acc)[8], uint4 b0, uint4 b1, bool two) {
+    const uint32_t u[4] = {b0.x, b0.y, b0.z, b0.w};
+    const uint32_t p[4] = {b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = __uint_as_float(u[i] << 16);
+        acc[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+        if (two) {
+            acc[2 * i] = __fadd_rn(acc[2 * i], __uint_as_float(p[i] << 16));
+            acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __uint_as_float(p[i] & 0xffff0000u));
+        }
+    }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&p);
 }
 
 // V: 16-byte columns per lane per row (a row segment of V * 512 bytes per
-// item); KB: rows whose loads are issued together before they are summed.
-template <int V, int kMinBlocks, int KB>
+// item); KB: rows whose loads are issued together before they are summed;
+// kBias: the sum starts from the output bias (a.bias0 is set).
+template <int V, int kMinBlocks, int KB, bool kBias>
 __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(CombineArgs a) {
     const int lane = threadIdx.x & 31;
     const int64_t gw = ((int64_t)blockIdx.x * kCombineThreads + threadIdx.x) >> 5;
@@ -79,6 +97,21 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[v][i] = 0.0f;
 
+        // the biases of this item, loaded before the first batch of rows and
+        // folded in after that batch is in flight
+        uint4 b0[V], b1[V];
+        if (kBias) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                const int col = ch * per_item + v * 32 + lane;
+                const bool in = col < HV;
+                b0[v] = in ? ld_stream_v4(reinterpret_cast<const uint4*>(a.bias0) + t * HV + col)
+                           : make_uint4(0, 0, 0, 0);
+                b1[v] = (in && a.bias1) ? ld_stream_v4(reinterpret_cast<const uint4*>(a.bias1) + t * HV + col)
+                                        : make_uint4(0, 0, 0, 0);
+            }
+        }
+
         for (int k0 = 0; k0 < K; k0 += KB) {
             uint4 rows[KB][V];
 #pragma unroll
@@ -92,6 +125,10 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
                     rows[kk][v] = (use && col < HV) ? ld_stream_v4(y + (int64_t)slot * HV + col)
                                                     : make_uint4(0, 0, 0, 0);
                 }
+            }
+            if (kBias && k0 == 0) {
+#pragma unroll
+                for (int v = 0; v < V; ++v) init_bias8(acc[v], b0[v], b1[v], a.bias1 != nullptr);
             }
 #pragma unroll
             for (int kk = 0; kk < KB; ++kk) {
@@ -135,8 +172,9 @@ __global__ void selftest_wait_kernel(WsHeader* hdr, uint64_t timeout_ns) {
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
     // items of 2 KB per row, rows loaded 4 at a time: contiguous 2 KB reads per
     // row keep DRAM pages open (measured faster than 1 KB items with 8 rows in
-    // flight, and than staging the rows through shared memory with TMA)
-    auto kernel = combine_kernel<4, 2, 4>;
+    // flight, and than staging the rows through shared memory with TMA); with
+    // a bias, 2 rows at a time keep the bias registers from spilling
+    auto kernel = a.bias0 ? combine_kernel<4, 2, 2, true> : combine_kernel<4, 2, 4, false>;
     int blocks_per_sm = 0;
     cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kernel, kCombineThreads, 0);
     if (err != cudaSuccess) return err;

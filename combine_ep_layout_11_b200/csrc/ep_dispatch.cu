@@ -20,7 +20,7 @@ namespace ep {
 namespace {
 
 constexpr uint32_t kMaxSegBytes = 16384;   // one bulk copy per row segment
-constexpr int kCastThreads = 128;
+constexpr int kCastThreads = 256;
 
 __host__ __device__ __forceinline__ uint32_t round_up_u32(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
@@ -293,7 +293,7 @@ cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStre
 cudaError_t launch_dispatch_cast(const DispatchArgs& a, cudaStream_t s) {
     const uint32_t in_stride = round_up_u32(2u * a.H, 128);
     const uint32_t out_stride = round_up_u32((uint32_t)a.H + 4u * a.nb, 128);
-    const int stages = 2;
+    const int stages = 3;   // H <= 16384: at most 130 KB of stages
     const size_t smem = (size_t)stages * in_stride + 2 * (size_t)out_stride + (size_t)stages * 8 +
                         (size_t)stages * 32 * 4;
     cudaError_t err =

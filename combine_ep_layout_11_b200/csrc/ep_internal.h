@@ -24,6 +24,7 @@ struct LayoutArgs {
     int32_t* table;
     int32_t* padpre;
     int32_t* pad_rows;
+    int32_t* stats;             // [E] running receive counts, nullable
 };
 
 // One cooperative kernel: per-chunk counts, a grid barrier, the scans and the
@@ -58,6 +59,8 @@ struct CombineArgs {
     const uint16_t* y;         // bf16 [capacity][H]
     const int32_t* pair_slot;  // [T*K]
     const float* w;            // [T*K] or nullptr
+    const uint16_t* bias0;     // bf16 [T][H] or nullptr
+    const uint16_t* bias1;     // bf16 [T][H] or nullptr (only with bias0)
     uint16_t* out;             // bf16 [T][H]
     WsHeader* status;          // status word (timeouts)
     int T, K, H;

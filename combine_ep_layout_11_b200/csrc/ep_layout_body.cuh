@@ -279,6 +279,7 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     if (c == 0) {
         for (int e = tid; e < E; e += NT) {
             a.cnt[e] = L.cnt[e];
+            if (a.stats) a.stats[e] += L.cnt[e];
             a.off[e] = L.off[e];
             a.padpre[e] = L.padpre[e];
         }

@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define EP_B200_VERSION 1
+#define EP_B200_VERSION 2
 
 /* Host return codes. */
 #define EP_OK 0
@@ -106,6 +106,13 @@ extern "C" {
  *                              (every later ep_layout leaves it ready again);
  *                              holds the device status word and scan scratch.
  *                              One workspace serves one call at a time.
+ *   cumulative_local_expert_recv_stats [E] int32 or NULL (§2.1 dispatch() and
+ *                              §3.3 low_latency_dispatch() argument of that
+ *                              name): a running per-expert receive count owned
+ *                              by the caller; when set, every ep_layout adds
+ *                              cnt[e] to entry e (virtual rank r's local
+ *                              experts are entries [r*E/R, (r+1)*E/R)).  Not
+ *                              cleared by the library.
  * Rows at and beyond expert_offset[E] are not written by ep_layout.
  */
 typedef struct ep_layout_t {
@@ -127,6 +134,7 @@ typedef struct ep_layout_t {
     int32_t num_max_tokens_per_rank;
     uint32_t magic;
     uint32_t reserved;
+    int32_t* cumulative_local_expert_recv_stats;   /* optional, see above */
 } ep_layout_t;
 
 /* Bytes of workspace ep_layout needs for these sizes (a pure host function). */
@@ -190,20 +198,25 @@ int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int n
                        int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales, void* stream);
 
 /*
- * Combine (§2.2 weighted; §3.2 unweighted when topk_weights is NULL; §4.1
- * ordered accumulation):
- *   out[t] = bf16_rne( sum over k = 0..K-1 with pair_slot[t, k] >= 0 of
- *                      w[t, k] * float(y[pair_slot[t, k]]) )
- * accumulated in fp32 in ascending k from +0, each step one rounded product and
- * one rounded sum.  A token with no selected entry gives a zero row.
+ * Combine (§2.2 weighted, with 0, 1 or 2 output biases; §3.2 unweighted when
+ * topk_weights is NULL; §4.1 ordered accumulation and its initial value):
+ *   out[t] = bf16_rne( init[t] + sum over k = 0..K-1 with pair_slot[t, k] >= 0
+ *                      of w[t, k] * float(y[pair_slot[t, k]]) )
+ * accumulated in fp32 in ascending k, each step one rounded product and one
+ * rounded sum.  init[t] is +0 without bias, float(bias0[t]) with one bias, and
+ * the rounded sum float(bias0[t]) + float(bias1[t]) with two.  A token with no
+ * selected entry gives bf16(init[t]).
  *   y            device bf16 [capacity, H], 16-byte aligned: expert outputs in
  *                receive order; padding rows are never read
  *   hidden H     > 0, H % 8 == 0
  *   topk_weights device fp32 [T, K] or NULL (unit weights)
- *   out          device bf16 [T, H], 16-byte aligned
+ *   bias0, bias1 device bf16 [T, H], 16-byte aligned, or NULL; bias1 without
+ *                bias0 is EP_ERR_INVALID_ARG
+ *   out          device bf16 [T, H], 16-byte aligned; may not alias y, and may
+ *                alias a bias only if it is that very array
  */
 int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float* topk_weights,
-               void* out, void* stream);
+               const void* bias0, const void* bias1, void* out, void* stream);
 
 /*
  * FP8 cast (§4.2 per_token_cast_to_fp8 with 128-column blocks): for token t

@@ -40,12 +40,13 @@ def test_every_declared_symbol_is_exported_and_bound(lib):
 
 def test_struct_size_matches_header(lib):
     from combine_ep_layout_11_b200 import _lib
-    # 7 pointers, u64, i64, 6 x i32, 2 x u32
-    assert ctypes.sizeof(_lib.EpLayout) == 7 * 8 + 8 + 8 + 6 * 4 + 2 * 4
+    # 7 pointers, u64, i64, 6 x i32, 2 x u32, the optional stats pointer
+    assert ctypes.sizeof(_lib.EpLayout) == 7 * 8 + 8 + 8 + 6 * 4 + 2 * 4 + 8
+    assert _lib.EpLayout.cumulative_local_expert_recv_stats.offset == 104
 
 
 def test_pure_host_functions(lib):
-    assert lib.ep_version() == 1
+    assert lib.ep_version() == 2
     assert lib.ep_capacity_rows(4096, 8, 256, 128) == 4096 * 8 + 256 * 127
     assert lib.ep_capacity_rows(128, 4, 16, 1) == 512
     ws = lib.ep_workspace_bytes(4096, 8, 256, 128)
@@ -84,6 +85,12 @@ def test_layout_host_checks(lib, T, K, E, R, A, limit, expect):
     assert rc == expect
 
 
+def test_layout_rejects_misaligned_recv_stats(lib):
+    s = _handle()
+    s.cumulative_local_expert_recv_stats = 0x10002
+    assert lib.ep_layout(ctypes.c_void_p(0x10000), None, 8, 2, 8, 2, 1, 0, ctypes.byref(s), None) == 1
+
+
 def test_layout_rejects_small_or_misaligned_workspace(lib):
     s = _handle(ws_bytes=64)
     assert lib.ep_layout(ctypes.c_void_p(0x10000), None, 8, 2, 8, 2, 1, 0, ctypes.byref(s), None) == 1
@@ -112,7 +119,7 @@ def test_dispatch_combine_host_checks(lib):
     s = _handle()                        # not filled by ep_layout: rejected
     p = ctypes.c_void_p(0x10000)
     assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 256, 0, 0, p, None, None) == 1
-    assert lib.ep_combine(ctypes.byref(s), p, 256, None, p, None) == 1
+    assert lib.ep_combine(ctypes.byref(s), p, 256, None, None, None, p, None) == 1
     s = _handle(magic=0x45504C31)        # a handle as ep_layout leaves it
     s.num_tokens, s.num_topk, s.num_experts, s.num_ranks, s.expert_alignment = 8, 2, 8, 2, 1
     assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 100, 0, 0, p, None, None) == 1      # H % 8
@@ -121,8 +128,11 @@ def test_dispatch_combine_host_checks(lib):
     assert lib.ep_dispatch(ctypes.byref(s), p, 1, p, 256, 1, 0, p, p, None) == 1            # cast of fp8 input
     assert lib.ep_dispatch(ctypes.byref(s), ctypes.c_void_p(0x10008), 0, None, 256, 0, 0, p, None, None) == 1
     assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 32768, 1, 0, p, p, None) == 6       # cast row too large
-    assert lib.ep_combine(ctypes.byref(s), p, 100, None, p, None) == 1                      # H % 8
-    assert lib.ep_combine(ctypes.byref(s), p, 256, None, ctypes.c_void_p(0x10004), None) == 1
+    assert lib.ep_combine(ctypes.byref(s), p, 100, None, None, None, p, None) == 1          # H % 8
+    assert lib.ep_combine(ctypes.byref(s), p, 256, None, None, None, ctypes.c_void_p(0x10004), None) == 1
+    assert lib.ep_combine(ctypes.byref(s), p, 256, None, None, p, p, None) == 1             # bias1 alone
+    assert lib.ep_combine(ctypes.byref(s), p, 256, None, ctypes.c_void_p(0x10008), None, p, None) == 1
+    assert lib.ep_combine(ctypes.byref(s), p, 256, None, p, ctypes.c_void_p(0x10002), p, None) == 1
     assert lib.ep_cast_fp8(p, 8, 100, p, p, None) == 1
     assert lib.ep_cast_fp8(p, 8, 32768, p, p, None) == 6
     flags = ctypes.c_uint32(0)

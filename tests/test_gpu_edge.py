@@ -241,3 +241,68 @@ def test_batch_invariance(ep):
     for B in (16, 64, 257):
         assert np.array_equal(outs[B][:1], outs[1])
     assert np.array_equal(outs[257][:16], outs[16]) and np.array_equal(outs[257][:64], outs[64])
+
+
+def test_recv_stats_accumulate_over_calls(ep):
+    """cumulative_local_expert_recv_stats (§2.1, §3.3): each layout adds its
+    per-expert counts; a call without the tensor, or with no tokens, adds nothing."""
+    T, K, E, R, A, H = 256, 8, 64, 4, 8, 128
+    stats0 = np.arange(E, dtype=np.int32) * 1000
+    stats = to_dev(stats0)
+    expect = stats0
+    lay = None
+    for seed in (1, 2, 3):
+        idx, w, x = _rand(T, K, E, H, seed=seed, drop=0.1)
+        ref = oracle.layout(idx, w, E, R, A)
+        lay = ep.layout(to_dev(idx), to_dev(w), E, R, A, out=lay, cumulative_local_expert_recv_stats=stats)
+        expect = oracle.accumulate_recv_stats(expect, ref["cnt"])
+    lay, _ = ep.layout_dispatch(to_dev(idx), to_dev(w), to_dev_bf16(x), E, R, A, out_layout=lay,
+                                cumulative_local_expert_recv_stats=stats)
+    expect = oracle.accumulate_recv_stats(expect, ref["cnt"])
+    ep.layout(to_dev(idx), to_dev(w), E, R, A, out=lay)                     # no stats: unchanged
+    ep.layout(to_dev(np.zeros((0, K), np.int64)), None, E, R, A, cumulative_local_expert_recv_stats=stats)
+    torch.cuda.synchronize()
+    assert np.array_equal(stats.cpu().numpy(), expect)
+
+
+@pytest.mark.parametrize("T,K,E,H,num_bias", [(64, 4, 16, 24, 1), (64, 4, 16, 24, 2), (33, 32, 64, 1032, 2),
+                                              (5, 1, 4, 8, 1)])
+def test_combine_bias_shapes(ep, T, K, E, H, num_bias):
+    """Bias with ragged rows (H = 24, 1032: rows not a multiple of the 2 KB item),
+    K at its maximum, all-unselected tokens (out = bf16(bias0 [+ bias1]))."""
+    idx, w, _ = _rand(T, K, E, H, seed=T * K, drop=0.2)
+    idx[:3] = -1
+    lay = ep.layout(to_dev(idx), to_dev(w), E, 1, 2)
+    ref = oracle.layout(idx, w, E, 1, 2)
+    Np = int(ref["off"][-1])
+    cfg = dict(seed=T + K + H, H=H)
+    y = workload.expert_outputs(cfg, max(Np, 1))
+    biases = [workload.expert_outputs(cfg, T, seed_offset=1 + i) for i in range(num_bias)]
+    dev_b = [to_dev_bf16(b) for b in biases]
+    out = ep.combine(lay, to_dev_bf16(y), to_dev(w), bias=dev_b[0] if num_bias == 1 else tuple(dev_b))
+    exp = oracle.combine(y, ref["pair_slot"], w, *(biases + [None] * (2 - num_bias)))
+    assert np.array_equal(bf16_bits(out), exp)
+
+
+def test_combine_in_place_over_bias(ep):
+    """out may be bias0 itself: every element reads its bias before it is written."""
+    T, K, E, H = 128, 8, 32, 7168
+    idx, w, _ = _rand(T, K, E, H, seed=5, drop=0.1)
+    lay = ep.layout(to_dev(idx), to_dev(w), E, 2, 1)
+    ref = oracle.layout(idx, w, E, 2, 1)
+    cfg = dict(seed=77, H=H)
+    y = workload.expert_outputs(cfg, int(ref["off"][-1]))
+    b0 = workload.expert_outputs(cfg, T, seed_offset=1)
+    d_b0 = to_dev_bf16(b0)
+    out = ep.combine(lay, to_dev_bf16(y), to_dev(w), bias=d_b0, out=d_b0)
+    assert out.data_ptr() == d_b0.data_ptr()
+    assert np.array_equal(bf16_bits(out), oracle.combine(y, ref["pair_slot"], w, b0, None))
+
+
+def test_combine_second_bias_alone_rejected(ep):
+    idx, w, _ = _rand(16, 2, 8, 64)
+    lay = ep.layout(to_dev(idx), to_dev(w), 8, 2, 1)
+    b = torch.zeros((16, 64), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ep.EpError) as exc:
+        ep.combine(lay, torch.zeros((64, 64), dtype=torch.bfloat16, device=DEV), bias=(None, b))
+    assert exc.value.code == ep.EP_ERR_INVALID_ARG

@@ -91,6 +91,22 @@ def test_combine_vs_oracle(ep, name):
     assert exact == 1.0, "combine is within tolerance but not bit-exact (%.6f equal)" % exact
 
 
+@pytest.mark.parametrize("num_bias", [1, 2])
+@pytest.mark.parametrize("name", ["prefill_bf16", "decode"])
+def test_combine_with_bias_vs_oracle(ep, name, num_bias):
+    """§2.2 combine() bias: the sum starts at bias0 (+ bias1), bit-exact with the oracle."""
+    cfg, inp, ref, x, w, lay = _run(ep, name)
+    Np = int(ref["off"][-1])
+    y_host = workload.expert_outputs(cfg, Np)
+    biases = [workload.expert_outputs(cfg, cfg["T"], seed_offset=1 + i) for i in range(num_bias)]
+    dev_b = [to_dev_bf16(b) for b in biases]
+    out = ep.combine(lay, to_dev_bf16(y_host), w, bias=dev_b[0] if num_bias == 1 else tuple(dev_b))
+    got = bf16_bits(out)
+    exp = oracle.combine(y_host, ref["pair_slot"], inp["topk_weights"], *(biases + [None] * (2 - num_bias)))
+    exact = assert_combine_close(got, exp)
+    assert exact == 1.0, "combine is within tolerance but not bit-exact (%.6f equal)" % exact
+
+
 @pytest.mark.parametrize("name", ["prefill_bf16", "decode", "large_prefill"])
 def test_identity_experts_reproduce_x(ep, name):
     """combine(dispatch(x)) with weights renormalised over the selected entries is x."""
