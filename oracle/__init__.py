@@ -70,6 +70,8 @@ def _load(path):
     L.orc_cast_fp8.argtypes = [vp, i64, i64, i64, ctypes.c_int, vp, vp]
     L.orc_dequant_fp8.restype = None
     L.orc_dequant_fp8.argtypes = [vp, vp, i64, i64, i64, vp]
+    L.orc_rank_layout.restype = ctypes.c_int
+    L.orc_rank_layout.argtypes = [vp, vp, i64, i64, i64, i64, i64, i64] + [vp] * 9
     L.orc_ue8m0_encode.restype = ctypes.c_int
     L.orc_ue8m0_encode.argtypes = [vp, i64, vp]
     L.orc_ue8m0_decode.restype = None
@@ -142,6 +144,47 @@ def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment,
     return dict(cnt=cnt, off=off, pair_slot=pair_slot, recv_src=recv_src[:capacity],
                 recv_w=recv_w[:capacity], recv_lexp=recv_lexp[:capacity],
                 num_experts=E, num_ranks=int(num_ranks), expert_alignment=int(expert_alignment),
+                capacity=int(capacity))
+
+
+def rank_layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment=1, capacity=None):
+    """Per-token-per-rank layout ([API] §2.1 with do_expand off; §3.1's V1
+    quantities): one receive row per (token, rank) the token reaches.
+
+    Returns a dict with ``num_tokens_per_rank`` [R], ``rank_off`` [R+1],
+    ``is_token_in_rank`` bool [T, R], ``token_slot`` [T, R],
+    ``num_tokens_per_expert`` / ``num_recv_tokens_per_expert`` (aligned) [E],
+    ``recv_src`` [capacity], ``recv_topk_idx`` int64 / ``recv_topk_weights``
+    [capacity, K]; plus ``pair_slot`` / ``cnt`` / ``off`` aliases of
+    token_slot / num_tokens_per_rank / rank_off so that ``dispatch_rows`` and
+    ``combine`` (with K = R and unit weights) serve this form too.
+    """
+    topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int64)
+    T, K = topk_idx.shape
+    E, R = int(num_experts), int(num_ranks)
+    if topk_weights is not None:
+        topk_weights = np.ascontiguousarray(topk_weights, dtype=np.float32)
+        assert topk_weights.shape == (T, K)
+    if capacity is None:
+        capacity = T * R
+    n_rank = np.zeros(R, np.int32)
+    rank_off = np.zeros(R + 1, np.int32)
+    in_rank = np.zeros((T, R), np.uint8)
+    token_slot = np.full((T, R), -1, np.int32)
+    n_exp = np.zeros(E, np.int32)
+    n_recv = np.zeros(E, np.int32)
+    recv_src = np.full(max(capacity, 1), -1, np.int32)
+    recv_idx = np.full((max(capacity, 1), K), -1, np.int64)
+    recv_w = np.zeros((max(capacity, 1), K), np.float32)
+    rc = lib().orc_rank_layout(_p(topk_idx), _p(topk_weights), T, K, E, R, int(expert_alignment), int(capacity),
+                               _p(n_rank), _p(rank_off), _p(in_rank), _p(token_slot), _p(n_exp), _p(n_recv),
+                               _p(recv_src), _p(recv_idx), _p(recv_w))
+    if rc != OK:
+        raise OracleError(rc, "rank layout")
+    return dict(num_tokens_per_rank=n_rank, rank_off=rank_off, is_token_in_rank=in_rank.astype(bool),
+                token_slot=token_slot, num_tokens_per_expert=n_exp, num_recv_tokens_per_expert=n_recv,
+                recv_src=recv_src[:capacity], recv_topk_idx=recv_idx[:capacity], recv_topk_weights=recv_w[:capacity],
+                pair_slot=token_slot, cnt=n_rank, off=rank_off, num_experts=R, num_ranks=R,
                 capacity=int(capacity))
 
 

@@ -239,6 +239,88 @@ int orc_layout(const int64_t* topk_idx, const float* topk_weights,
 }
 
 /* ------------------------------------------------------------------ */
+/* Per-token-per-rank layout                    [API] §2.1, §3.1, §3.2  */
+/* ------------------------------------------------------------------ */
+
+/* The default receive form of dispatch (do_expand off, [API] §2.1): one
+ * receive row per (token, destination rank) that the token reaches, with the
+ * V1 layout quantities of [API] §3.1 (num_tokens_per_rank, is_token_in_rank,
+ * num_tokens_per_expert) and the V1 receive outputs (recv_topk_idx,
+ * recv_topk_weights, num_recv_tokens_per_expert_list).
+ *  is_token_in_rank[t, r]   1 if some k has topk_idx[t, k] on rank r (e / (E/R) == r)
+ *  num_tokens_per_rank[r]   number of tokens with is_token_in_rank[t, r]
+ *  rank_off[r]              sum over r' < r of num_tokens_per_rank[r']; rank_off[R] = rows used
+ *  token_slot[t, r]         receive row of (t, r), -1 if the token does not reach r
+ *  num_tokens_per_expert[e] number of pairs (t, k) that chose e
+ *  num_recv_per_expert[e]   align(num_tokens_per_expert[e], A) (the aligned list of §3.1)
+ *  recv_src[row]            source token of the row
+ *  recv_topk_idx[row, k]    topk_idx[t, k] - r*(E/R) if that expert is on the row's rank r, else -1
+ *  recv_topk_w[row, k]      topk_weights[t, k] (1 without weights) for those entries, else 0
+ * Rows of rank r are [rank_off[r], rank_off[r+1]) in ascending token order
+ * (so by source rank, then token).  No padding rows. */
+int orc_rank_layout(const int64_t* topk_idx, const float* topk_weights, int64_t T, int64_t K, int64_t E,
+                    int64_t R, int64_t A, int64_t capacity, int32_t* num_tokens_per_rank, int32_t* rank_off,
+                    uint8_t* is_token_in_rank, int32_t* token_slot, int32_t* num_tokens_per_expert,
+                    int32_t* num_recv_per_expert, int32_t* recv_src, int64_t* recv_topk_idx, float* recv_topk_w)
+{
+    if (T < 0 || K < 1 || E < 1 || R < 1 || A < 1 || E % R != 0 || T % R != 0)
+        return ORC_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < T * K; i++)
+        if (topk_idx[i] < -1 || topk_idx[i] >= E)
+            return ORC_ERR_BAD_EXPERT;
+    int64_t experts_per_rank = E / R;
+
+    for (int64_t e = 0; e < E; e++)
+        num_tokens_per_expert[e] = 0;
+    for (int64_t i = 0; i < T * K; i++)
+        if (topk_idx[i] >= 0)
+            num_tokens_per_expert[topk_idx[i]] += 1;
+    for (int64_t e = 0; e < E; e++)
+        num_recv_per_expert[e] = (int32_t)align_up(num_tokens_per_expert[e], A);
+
+    for (int64_t t = 0; t < T; t++)
+        for (int64_t r = 0; r < R; r++) {
+            uint8_t in = 0;
+            for (int64_t k = 0; k < K; k++) {
+                int64_t e = topk_idx[t * K + k];
+                if (e >= 0 && e / experts_per_rank == r)
+                    in = 1;
+            }
+            is_token_in_rank[t * R + r] = in;
+        }
+    for (int64_t r = 0; r < R; r++) {
+        num_tokens_per_rank[r] = 0;
+        for (int64_t t = 0; t < T; t++)
+            num_tokens_per_rank[r] += is_token_in_rank[t * R + r];
+    }
+    rank_off[0] = 0;
+    for (int64_t r = 0; r < R; r++)
+        rank_off[r + 1] = rank_off[r] + num_tokens_per_rank[r];
+    if (rank_off[R] > capacity)
+        return ORC_ERR_CAPACITY;
+
+    for (int64_t r = 0; r < R; r++) {
+        int64_t row = rank_off[r];
+        for (int64_t t = 0; t < T; t++) {
+            if (!is_token_in_rank[t * R + r]) {
+                token_slot[t * R + r] = -1;
+                continue;
+            }
+            token_slot[t * R + r] = (int32_t)row;
+            recv_src[row] = (int32_t)t;
+            for (int64_t k = 0; k < K; k++) {
+                int64_t e = topk_idx[t * K + k];
+                int local = e >= 0 && e / experts_per_rank == r;
+                recv_topk_idx[row * K + k] = local ? e - r * experts_per_rank : -1;
+                recv_topk_w[row * K + k] = local ? (topk_weights ? topk_weights[t * K + k] : 1.0f) : 0.0f;
+            }
+            row += 1;
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* Dispatch: row scatter                        [API] §2.1              */
 /* ------------------------------------------------------------------ */
 

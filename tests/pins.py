@@ -581,6 +581,107 @@ def pin_recv_stats():
     assert np.array_equal(stats, start + seen)
 
 
+def _rank_layout_numpy(idx, w, E, R, A):
+    """The per-token-per-rank layout restated with numpy set operations."""
+    T, K = idx.shape
+    El = E // R
+    dest = np.where(idx >= 0, idx // El, -1)
+    in_rank = (dest[:, :, None] == np.arange(R)[None, None, :]).any(axis=1)
+    tokens = [np.nonzero(in_rank[:, r])[0] for r in range(R)]
+    n_rank = np.array([len(tk) for tk in tokens], np.int32)
+    rank_off = np.concatenate([[0], np.cumsum(n_rank)]).astype(np.int32)
+    token_slot = np.full((T, R), -1, np.int32)
+    for r in range(R):
+        token_slot[tokens[r], r] = rank_off[r] + np.arange(len(tokens[r]))
+    src = np.concatenate(tokens + [np.zeros(0, np.int64)]).astype(np.int32)
+    row_rank = np.repeat(np.arange(R), n_rank)
+    local = dest[src] == row_rank[:, None]
+    ridx = np.where(local, idx[src] - row_rank[:, None] * El, -1)
+    ww = np.ones((T, K), np.float32) if w is None else w
+    rw = np.where(local, ww[src], 0).astype(np.float32)
+    n_exp = np.bincount(idx[idx >= 0], minlength=E).astype(np.int32)
+    n_recv = ((n_exp + A - 1) // A * A).astype(np.int32)
+    return dict(is_token_in_rank=in_rank, num_tokens_per_rank=n_rank, rank_off=rank_off, token_slot=token_slot,
+                recv_src=src, recv_topk_idx=ridx, recv_topk_weights=rw, num_tokens_per_expert=n_exp,
+                num_recv_tokens_per_expert=n_recv)
+
+
+def pin_rank_layout_vs_numpy(n=120, seed=37):
+    rng = np.random.default_rng(seed)
+    for i in range(n):
+        R = int(rng.choice([1, 2, 4, 8]))
+        E = R * int(rng.integers(1, 5))
+        T = R * int(rng.integers(0, 9))
+        K = int(rng.integers(1, 6))
+        A = int(rng.integers(1, 4))
+        idx = rng.integers(-1, E, (T, K)).astype(np.int64)
+        w = rng.random((T, K)).astype(np.float32) if i % 2 else None
+        got = oracle.rank_layout(idx, w, E, R, A)
+        exp = _rank_layout_numpy(idx, w, E, R, A)
+        rows = int(exp["rank_off"][-1])
+        for key in ("is_token_in_rank", "num_tokens_per_rank", "rank_off", "token_slot",
+                    "num_tokens_per_expert", "num_recv_tokens_per_expert"):
+            assert np.array_equal(got[key], exp[key]), key
+        assert np.array_equal(got["recv_src"][:rows], exp["recv_src"])
+        assert np.array_equal(got["recv_topk_idx"][:rows], exp["recv_topk_idx"])
+        assert np.array_equal(got["recv_topk_weights"][:rows].view(np.uint32),
+                              exp["recv_topk_weights"].view(np.uint32))
+
+
+def pin_rank_layout_golden():
+    g = _golden("rank_layout_example.json")
+    d = oracle.rank_layout(np.array(g["topk_idx"], np.int64), np.array(g["topk_weights"], np.float32),
+                           g["E"], g["R"], g["A"])
+    rows = sum(g["num_tokens_per_rank"])
+    for key in ("num_tokens_per_rank", "token_slot", "num_tokens_per_expert", "num_recv_tokens_per_expert"):
+        assert d[key].tolist() == g[key], key
+    assert d["is_token_in_rank"].astype(int).tolist() == g["is_token_in_rank"]
+    assert d["recv_src"][:rows].tolist() == g["recv_src"]
+    assert d["recv_topk_idx"][:rows].tolist() == g["recv_topk_idx"]
+    assert d["recv_topk_weights"][:rows].tolist() == g["recv_topk_weights"]
+
+
+def pin_rank_layout_matches_expand():
+    """Same routing, both forms: per-expert counts agree with the expand layout,
+    and the local entries of rank r's rows are exactly the pairs the expand
+    layout puts in rank r's region."""
+    for name in ("tiny", "prefill_bf16"):
+        cfg = workload.config(name)
+        idx, w = workload.routing(cfg)
+        E, R, A = cfg["E"], cfg["R"], cfg["A"]
+        ex = oracle.layout(idx, w, E, R, A)
+        rk = oracle.rank_layout(idx, w, E, R, A)
+        assert np.array_equal(rk["num_tokens_per_expert"], ex["cnt"])
+        assert np.array_equal(rk["num_recv_tokens_per_expert"], np.diff(ex["off"]))
+        El = E // R
+        for r in range(R):
+            lo, hi = rk["rank_off"][r], rk["rank_off"][r + 1]
+            ri = rk["recv_topk_idx"][lo:hi]
+            pairs = int((ri >= 0).sum())
+            assert pairs == int(ex["cnt"][r * El:(r + 1) * El].sum())
+
+
+def pin_rank_combine_identity():
+    """Rank-level combine (§3.2: plain sum over the reached ranks, K = R, unit
+    weights): expert outputs equal to x on each token's first rank and 0 on
+    the others reproduce x."""
+    rng = np.random.default_rng(41)
+    T, K, E, R, H = 48, 4, 16, 4, 64
+    idx = rng.integers(-1, E, (T, K)).astype(np.int64)
+    idx[0] = -1
+    x = workload.to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
+    rk = oracle.rank_layout(idx, None, E, R, 1)
+    y = np.zeros((rk["capacity"], H), np.uint16)
+    for t in range(T):
+        slots = rk["token_slot"][t][rk["token_slot"][t] >= 0]
+        if slots.size:
+            y[slots[0]] = x[t]
+    out = oracle.combine(y, rk["token_slot"], None)
+    has = rk["is_token_in_rank"].any(axis=1)
+    expect = np.where(x == 0x8000, np.uint16(0), x)
+    assert np.array_equal(out[has], expect[has]) and np.all(out[~has] == 0)
+
+
 ALL_PINS = [
     pin_layout_exhaustive, pin_layout_random, pin_layout_invariants_workloads, pin_layout_errors,
     pin_routing_table_golden, pin_dispatch_rows, pin_e4m3_decode_table, pin_e4m3_encode_vs_torch,
@@ -589,4 +690,5 @@ ALL_PINS = [
     pin_combine_permutation, pin_recv_stats,
     pin_cast_variants_vs_torch, pin_round_scale_properties, pin_fp8_variants_golden, pin_ue8m0,
     pin_cast_variants_roundtrip, pin_scales_col_major,
+    pin_rank_layout_vs_numpy, pin_rank_layout_golden, pin_rank_layout_matches_expand, pin_rank_combine_identity,
 ]

@@ -36,6 +36,18 @@ MUTANTS = {
          "            out[t * H + h] = f32_to_bf16_rne(acc[h] + (bias0 ? bf16_to_f32(bias0[t * H + h]) : 0.0f)\n"
          "                                             + (bias1 ? bf16_to_f32(bias1[t * H + h]) : 0.0f));")],
     "stats_overwrite": ("stats[e] += cnt[e];", "stats[e] = cnt[e];"),
+    "rank_rows_descending_token": (
+        "        for (int64_t t = 0; t < T; t++) {\n            if (!is_token_in_rank[t * R + r]) {",
+        "        for (int64_t t = T - 1; t >= 0; t--) {\n            if (!is_token_in_rank[t * R + r]) {"),
+    "rank_global_expert_ids": ("recv_topk_idx[row * K + k] = local ? e - r * experts_per_rank : -1;",
+                               "recv_topk_idx[row * K + k] = local ? e : -1;"),
+    "rank_remote_weights_kept": (
+        "recv_topk_w[row * K + k] = local ? (topk_weights ? topk_weights[t * K + k] : 1.0f) : 0.0f;",
+        "recv_topk_w[row * K + k] = topk_weights ? topk_weights[t * K + k] : 1.0f;"),
+    "rank_by_modulo": ("if (e >= 0 && e / experts_per_rank == r)\n                    in = 1;",
+                       "if (e >= 0 && e % R == r)\n                    in = 1;"),
+    "rank_list_unaligned": ("num_recv_per_expert[e] = (int32_t)align_up(num_tokens_per_expert[e], A);",
+                            "num_recv_per_expert[e] = num_tokens_per_expert[e];"),
     "bf16_truncates": ("if (dropped > 0x8000u || (dropped == 0x8000u && (upper & 1u)))", "if (0)"),
     "bf16_ties_away": ("if (dropped > 0x8000u || (dropped == 0x8000u && (upper & 1u)))",
                        "if (dropped >= 0x8000u)"),
