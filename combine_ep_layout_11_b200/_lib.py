@@ -42,10 +42,12 @@ SIGNATURES = {
     "ep_capacity_rows": (_i64, [_i, _i, _i, _i]),
     "ep_layout": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp]),
     "ep_layout_no_alloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp]),
-    "ep_dispatch": (_i, [_LP, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp]),
-    "ep_layout_dispatch": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp]),
+    "ep_scale_bytes": (_i64, [_i64, _i, _i]),
+    "ep_dispatch": (_i, [_LP, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "ep_layout_dispatch": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp,
+                                _vp]),
     "ep_combine": (_i, [_LP, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
-    "ep_cast_fp8": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "ep_cast_fp8": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "ep_get_status": (_i, [_LP, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "ep_selftest_bounded_wait": (_i, [_LP, _u64, _vp]),
     "ep_status_string": (ctypes.c_char_p, [_i]),

@@ -3,8 +3,10 @@
 Names follow "DeepEP 测试目标 API 系统性参考": ``layout`` derives the routing
 layout (§2.1, the V2 path that needs only topk_idx), ``dispatch`` and ``combine``
 take the layout as their handle (§2.1 / §2.2), ``cast_fp8`` is §4.2's per-token
-cast with 128-column scale blocks.  Every step runs in ``libep_b200.so`` on the
-tensors' CUDA device, on the current torch stream; torch only allocates memory.
+cast with 128-column scale blocks (or the scale variants of §3.3 and §2.1:
+per-row, ``round_scale``, ``use_ue8m0``, ``use_tma_aligned_col_major_sf``).
+Every step runs in ``libep_b200.so`` on the tensors' CUDA device, on the
+current torch stream; torch only allocates memory.
 """
 import ctypes
 
@@ -21,6 +23,31 @@ EP_ERR_CUDA = 5
 EP_ERR_UNSUPPORTED = 6
 EP_DTYPE_BF16 = 0
 EP_DTYPE_FP8_E4M3 = 1
+EP_SF_PER_ROW = 0x1
+EP_SF_POW2 = 0x2
+EP_SF_UE8M0 = 0x4
+EP_SF_COL_MAJOR = 0x8
+
+
+def scale_format(per_token=False, round_scale=False, use_ue8m0=False, use_tma_aligned_col_major_sf=False):
+    """EP_SF_* bits from the pages' option names (UE8M0 implies round_scale)."""
+    return ((EP_SF_PER_ROW if per_token else 0) | (EP_SF_POW2 if (round_scale or use_ue8m0) else 0)
+            | (EP_SF_UE8M0 if use_ue8m0 else 0) | (EP_SF_COL_MAJOR if use_tma_aligned_col_major_sf else 0))
+
+
+def scale_tensor(rows, hidden, fmt, device):
+    """An uninitialised scale array for ``rows`` FP8 rows in format ``fmt``, as a
+    logical [rows, groups] view: fp32 or uint8 (UE8M0) elements, row-major, or
+    column-major with the leading dimension padded to 16 bytes (stride (1, ld))."""
+    nbytes = int(_lib.load().ep_scale_bytes(rows, hidden, fmt))
+    if nbytes < 0:
+        raise EpError(EP_ERR_INVALID_ARG, "scale format")
+    groups = 1 if fmt & EP_SF_PER_ROW else hidden // 128
+    dtype = torch.uint8 if fmt & EP_SF_UE8M0 else torch.float32
+    if fmt & EP_SF_COL_MAJOR:
+        ld = nbytes // (groups * dtype.itemsize) if groups else 0
+        return torch.empty((groups, max(ld, 1)), dtype=dtype, device=device).t()[:rows]
+    return torch.empty((rows, groups), dtype=dtype, device=device)
 
 
 class EpError(RuntimeError):
@@ -145,12 +172,15 @@ def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment=1,
     return lay
 
 
-def dispatch(lay, x, x_scales=None, cast_to_fp8=False, do_zero_padding=False, out=None, out_scales=None):
+def dispatch(lay, x, x_scales=None, cast_to_fp8=False, do_zero_padding=False, out=None, out_scales=None,
+             scale_fmt=0):
     """Scatter token rows into the receive buffer (§2.1 dispatch()).
 
     ``x``: bf16 [T, H], or float8_e4m3fn [T, H] with ``x_scales`` fp32 [T, H/128].
     Returns ``recv_x`` [capacity, H] (bf16, or e4m3 when the input is FP8 or
-    ``cast_to_fp8``) and, for FP8 output, ``recv_scales`` [capacity, H/128].
+    ``cast_to_fp8``) and, for FP8 output, ``recv_scales`` [capacity, groups]
+    (fp32 per 128-column block unless ``scale_fmt``, EP_SF_* bits from
+    ``scale_format()``, asks for another form of the cast's scales).
     """
     L = _lib.load()
     assert x.dim() == 2 and x.is_contiguous() and x.shape[0] == lay.num_tokens
@@ -162,9 +192,9 @@ def dispatch(lay, x, x_scales=None, cast_to_fp8=False, do_zero_padding=False, ou
     if out is None:
         out = torch.empty((cap, H), dtype=torch.float8_e4m3fn if fp8_out else torch.bfloat16, device=x.device)
     if fp8_out and out_scales is None:
-        out_scales = torch.empty((cap, H // 128), dtype=torch.float32, device=x.device)
+        out_scales = scale_tensor(cap, H, scale_fmt, x.device)
     _check(L.ep_dispatch(lay.ref(), _ptr(x), EP_DTYPE_FP8_E4M3 if fp8_in else EP_DTYPE_BF16,
-                         _ptr(x_scales if fp8_in else None), H, int(bool(cast_to_fp8)),
+                         _ptr(x_scales if fp8_in else None), H, int(bool(cast_to_fp8)), int(scale_fmt),
                          int(bool(do_zero_padding)), _ptr(out), _ptr(out_scales if fp8_out else None),
                          _stream(x.device)), "ep_dispatch")
     return (out, out_scales) if fp8_out else out
@@ -173,7 +203,7 @@ def dispatch(lay, x, x_scales=None, cast_to_fp8=False, do_zero_padding=False, ou
 def layout_dispatch(topk_idx, topk_weights, x, num_experts, num_ranks, expert_alignment=1,
                     num_max_tokens_per_rank=0, x_scales=None, cast_to_fp8=False, do_zero_padding=False,
                     capacity=None, out_layout=None, out=None, out_scales=None,
-                    cumulative_local_expert_recv_stats=None):
+                    cumulative_local_expert_recv_stats=None, scale_fmt=0):
     """Layout and dispatch in one call (§2.1: V2's dispatch() derives the layout
     from topk_idx).  Same results as ``layout`` then ``dispatch``; returns
     ``(layout, recv_x)`` or ``(layout, (recv_x, recv_scales))`` for FP8 output."""
@@ -197,11 +227,11 @@ def layout_dispatch(topk_idx, topk_weights, x, num_experts, num_ranks, expert_al
     if out is None:
         out = torch.empty((cap, H), dtype=torch.float8_e4m3fn if fp8_out else torch.bfloat16, device=x.device)
     if fp8_out and out_scales is None:
-        out_scales = torch.empty((cap, H // 128), dtype=torch.float32, device=x.device)
+        out_scales = scale_tensor(cap, H, scale_fmt, x.device)
     _check(L.ep_layout_dispatch(_ptr(topk_idx), _ptr(topk_weights), T, K, num_experts, num_ranks,
                                 expert_alignment, num_max_tokens_per_rank, lay.ref(), _ptr(x),
                                 EP_DTYPE_FP8_E4M3 if fp8_in else EP_DTYPE_BF16, _ptr(x_scales if fp8_in else None),
-                                H, int(bool(cast_to_fp8)), int(bool(do_zero_padding)), _ptr(out),
+                                H, int(bool(cast_to_fp8)), int(scale_fmt), int(bool(do_zero_padding)), _ptr(out),
                                 _ptr(out_scales if fp8_out else None), _stream(x.device)), "ep_layout_dispatch")
     return lay, ((out, out_scales) if fp8_out else out)
 
@@ -234,16 +264,18 @@ def combine(lay, y, topk_weights=None, bias=None, out=None):
     return out
 
 
-def cast_fp8(x, out=None, out_scales=None):
-    """bf16 [T, H] -> (float8_e4m3fn [T, H], fp32 scales [T, H/128]) (§4.2)."""
+def cast_fp8(x, out=None, out_scales=None, scale_fmt=0):
+    """bf16 [T, H] -> (float8_e4m3fn [T, H], scales [T, groups]) (§4.2); fp32
+    scales per 128-column block unless ``scale_fmt`` (EP_SF_* bits) says otherwise."""
     L = _lib.load()
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
     T, H = x.shape
     if out is None:
         out = torch.empty((T, H), dtype=torch.float8_e4m3fn, device=x.device)
     if out_scales is None:
-        out_scales = torch.empty((T, H // 128), dtype=torch.float32, device=x.device)
-    _check(L.ep_cast_fp8(_ptr(x), T, H, _ptr(out), _ptr(out_scales), _stream(x.device)), "ep_cast_fp8")
+        out_scales = scale_tensor(T, H, scale_fmt, x.device)
+    _check(L.ep_cast_fp8(_ptr(x), T, H, int(scale_fmt), _ptr(out), _ptr(out_scales), _stream(x.device)),
+           "ep_cast_fp8")
     return out, out_scales
 
 

@@ -90,13 +90,14 @@ int empty_layout(ep_layout_t* layout, cudaStream_t s) {
 
 // Argument checks of ep_dispatch against a filled handle; fills the kernel arguments.
 int prepare_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales, int H,
-                     int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales, ep::DispatchArgs* a,
-                     int* elem_bytes) {
+                     int cast_to_fp8, int scale_format, int do_zero_padding, void* recv_x, void* recv_scales,
+                     ep::DispatchArgs* a, int* elem_bytes) {
     int rc = check_handle(layout);
     if (rc != EP_OK) return rc;
     const int T = layout->num_tokens;
     if (H <= 0 || (x_dtype != EP_DTYPE_BF16 && x_dtype != EP_DTYPE_FP8_E4M3)) return EP_ERR_INVALID_ARG;
     if (cast_to_fp8 && x_dtype != EP_DTYPE_BF16) return EP_ERR_INVALID_ARG;
+    if (scale_format != 0 && !cast_to_fp8) return EP_ERR_INVALID_ARG;
     const bool fp8_in = x_dtype == EP_DTYPE_FP8_E4M3;
     const bool fp8_out = fp8_in || cast_to_fp8;
     if (H % 8 != 0 || (fp8_out && H % 128 != 0)) return EP_ERR_INVALID_ARG;
@@ -111,7 +112,7 @@ int prepare_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, cons
     a->x = reinterpret_cast<const uint8_t*>(x);
     a->x_scales = fp8_in ? x_scales : nullptr;
     a->recv = reinterpret_cast<uint8_t*>(recv_x);
-    a->recv_scales = fp8_out ? recv_scales : nullptr;
+    a->recv_scales = fp8_out ? reinterpret_cast<float*>(recv_scales) : nullptr;
     a->pair_slot = layout->pair_slot;
     a->hdr = reinterpret_cast<const ep::WsHeader*>(wsb);
     a->pad_rows = reinterpret_cast<const int32_t*>(wsb + ws.padrows_off);
@@ -122,6 +123,7 @@ int prepare_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, cons
     a->capacity = layout->capacity;
     a->nb = fp8_out ? H / 128 : 0;
     a->zero_pad = do_zero_padding ? 1 : 0;
+    if (!ep::set_scale_format(a, scale_format, layout->capacity)) return EP_ERR_INVALID_ARG;
     *elem_bytes = fp8_in ? 1 : 2;
     return device_sms(&a->sms);
 }
@@ -169,12 +171,21 @@ int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens
     return ep::launch_layout(a, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
+int64_t ep_scale_bytes(int64_t rows, int hidden, int scale_format) {
+    if (rows < 0 || hidden <= 0 || hidden % 128 != 0) return -1;
+    ep::DispatchArgs a;
+    a.nb = hidden / 128;
+    if (!ep::set_scale_format(&a, scale_format, rows)) return -1;
+    return (a.sf_col_major ? a.sf_ld : rows) * a.ng * a.sf_elem;
+}
+
 int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales, int hidden,
-                int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales, void* stream) {
+                int cast_to_fp8, int scale_format, int do_zero_padding, void* recv_x, void* recv_scales,
+                void* stream) {
     ep::DispatchArgs a;
     int elem_bytes = 0;
-    int rc = prepare_dispatch(layout, x, x_dtype, x_scales, hidden, cast_to_fp8, do_zero_padding, recv_x,
-                              recv_scales, &a, &elem_bytes);
+    int rc = prepare_dispatch(layout, x, x_dtype, x_scales, hidden, cast_to_fp8, scale_format, do_zero_padding,
+                              recv_x, recv_scales, &a, &elem_bytes);
     if (rc != EP_OK) return rc;
     if (layout->num_tokens == 0) return EP_OK;   // no tokens, no pairs, no padding rows
     cudaStream_t s = (cudaStream_t)stream;
@@ -185,7 +196,8 @@ int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const flo
 int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
                        int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
                        ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales, int hidden,
-                       int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales, void* stream) {
+                       int cast_to_fp8, int scale_format, int do_zero_padding, void* recv_x, void* recv_scales,
+                       void* stream) {
     if (!layout) return EP_ERR_INVALID_ARG;
     ep_layout_t tmp = *layout;   // the handle changes only once every check has passed
     ep::LayoutArgs la;
@@ -194,8 +206,8 @@ int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int n
     int rc = prepare_layout(topk_idx, topk_weights, num_tokens, num_topk, num_experts, num_ranks,
                             expert_alignment, num_max_tokens_per_rank, &tmp, &la);
     if (rc != EP_OK) return rc;
-    rc = prepare_dispatch(&tmp, x, x_dtype, x_scales, hidden, cast_to_fp8, do_zero_padding, recv_x, recv_scales,
-                          &da, &elem_bytes);
+    rc = prepare_dispatch(&tmp, x, x_dtype, x_scales, hidden, cast_to_fp8, scale_format, do_zero_padding, recv_x,
+                          recv_scales, &da, &elem_bytes);
     if (rc != EP_OK) return rc;
     *layout = tmp;
     cudaStream_t s = (cudaStream_t)stream;
@@ -238,18 +250,20 @@ int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float
     return ep::launch_combine(a, (cudaStream_t)stream) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
-int ep_cast_fp8(const void* x, int num_tokens, int hidden, void* x_fp8, float* scales, void* stream) {
+int ep_cast_fp8(const void* x, int num_tokens, int hidden, int scale_format, void* x_fp8, void* scales,
+                void* stream) {
     const int T = num_tokens, H = hidden;
     if (T < 0 || H <= 0 || H % 128 != 0) return EP_ERR_INVALID_ARG;
     if (H > 16384) return EP_ERR_UNSUPPORTED;
     if (T > 0 && (!x || !x_fp8 || !scales)) return EP_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(x_fp8, 16) || !aligned(scales, 16)) return EP_ERR_INVALID_ARG;
+    if (ep_scale_bytes(T, H, scale_format) < 0) return EP_ERR_INVALID_ARG;
     if (T == 0) return EP_OK;
     ep::DispatchArgs a;
     a.x = reinterpret_cast<const uint8_t*>(x);
     a.x_scales = nullptr;
     a.recv = reinterpret_cast<uint8_t*>(x_fp8);
-    a.recv_scales = scales;
+    a.recv_scales = reinterpret_cast<float*>(scales);
     a.pair_slot = nullptr;   // row t -> row t
     a.hdr = nullptr;
     a.pad_rows = nullptr;
@@ -260,6 +274,7 @@ int ep_cast_fp8(const void* x, int num_tokens, int hidden, void* x_fp8, float* s
     a.capacity = T;
     a.nb = H / 128;
     a.zero_pad = 0;
+    if (!ep::set_scale_format(&a, scale_format, T)) return EP_ERR_INVALID_ARG;
     int rc = device_sms(&a.sms);
     if (rc != EP_OK) return rc;
     return ep::launch_dispatch_cast(a, (cudaStream_t)stream) == cudaSuccess ? EP_OK : EP_ERR_CUDA;

@@ -135,19 +135,44 @@ __global__ void __launch_bounds__(32) dispatch_copy_kernel(DispatchArgs a, uint3
 }
 
 // ---------------------------------------------------------------------------
-// Cast kernel: bf16 rows in, e4m3 rows + fp32 per-128-column scales out.
+// Cast kernel: bf16 rows in, e4m3 rows and their scales out.  The scale
+// variants (EP_SF_* bits): one scale per 128-column block or per row
+// (kPerRow), amax / 448 or that rounded up to a power of two (kPow2), stored
+// as fp32 or as a UE8M0 exponent byte, row-major or TMA-aligned column-major
+// (the last two are runtime fields of DispatchArgs).
 // ---------------------------------------------------------------------------
 
-// Quantise 4 consecutive values of one 128-column block held by this lane;
-// the warp holds the whole block (32 lanes x 4 values).
-__device__ __forceinline__ uint32_t cast_block4(uint2 raw, float* scale_out) {
-    const float f0 = __uint_as_float(raw.x << 16), f1 = __uint_as_float(raw.x & 0xffff0000u);
-    const float f2 = __uint_as_float(raw.y << 16), f3 = __uint_as_float(raw.y & 0xffff0000u);
-    float m = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
+__device__ __forceinline__ float warp_max(float m) {
 #pragma unroll
     for (int d = 16; d >= 1; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
-    const float s = __fdiv_rn(fmaxf(m, 1e-4f), 448.0f);
-    *scale_out = s;
+    return m;
+}
+
+// max |x| of one 128-column block: the warp holds it as 32 lanes x 4 values
+__device__ __forceinline__ float block_amax(uint2 raw) {
+    const float f0 = __uint_as_float(raw.x << 16), f1 = __uint_as_float(raw.x & 0xffff0000u);
+    const float f2 = __uint_as_float(raw.y << 16), f3 = __uint_as_float(raw.y & 0xffff0000u);
+    return warp_max(fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3))));
+}
+
+// The smallest power of two >= s for a positive normal s: clear the mantissa
+// and, unless it was already zero, step the exponent up by one.
+__device__ __forceinline__ float pow2_ceil(float s) {
+    uint32_t u = __float_as_uint(s);
+    if (u & 0x7fffffu) u = (u & 0x7f800000u) + 0x800000u;
+    return __uint_as_float(u);
+}
+
+template <bool kPow2>
+__device__ __forceinline__ float make_scale(float amax) {
+    const float s = __fdiv_rn(fmaxf(amax, 1e-4f), 448.0f);
+    return kPow2 ? pow2_ceil(s) : s;
+}
+
+// e4m3 codes of the lane's 4 values under scale s
+__device__ __forceinline__ uint32_t quant4(uint2 raw, float s) {
+    const float f0 = __uint_as_float(raw.x << 16), f1 = __uint_as_float(raw.x & 0xffff0000u);
+    const float f2 = __uint_as_float(raw.y << 16), f3 = __uint_as_float(raw.y & 0xffff0000u);
     const __nv_fp8x2_storage_t lo =
         __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f0, s), __fdiv_rn(f1, s)), __NV_SATFINITE, __NV_E4M3);
     const __nv_fp8x2_storage_t hi =
@@ -155,9 +180,33 @@ __device__ __forceinline__ uint32_t cast_block4(uint2 raw, float* scale_out) {
     return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
+// Scale g of a row staged in shared memory: fp32, or the UE8M0 byte (the
+// biased exponent of a power-of-two scale).
+__device__ __forceinline__ void put_scale(uint8_t* row_sf, int g, float s, int elem) {
+    if (elem == 4)
+        reinterpret_cast<float*>(row_sf)[g] = s;
+    else
+        row_sf[g] = (uint8_t)((__float_as_uint(s) >> 23) & 0xffu);
+}
+
+// Byte offset of scale (row, g) in the scale array.
+__device__ __forceinline__ int64_t sf_offset(const DispatchArgs& a, int64_t row, int g) {
+    return (a.sf_col_major ? (int64_t)g * a.sf_ld + row : row * a.ng + g) * a.sf_elem;
+}
+
+// One scale element from shared memory (src, element g) to global memory.
+__device__ __forceinline__ void copy_scale(uint8_t* sf, int64_t off, const uint8_t* src, int g, int elem) {
+    if (elem == 4)
+        *reinterpret_cast<float*>(sf + off) = reinterpret_cast<const float*>(src)[g];
+    else
+        sf[off] = src[g];
+}
+
+template <bool kPerRow, bool kPow2>
 __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArgs a, int stages) {
+    constexpr int kWarps = kCastThreads / 32;
     extern __shared__ __align__(128) uint8_t smem[];
-    const int H = a.H, nb = a.nb, K = a.K;
+    const int H = a.H, nb = a.nb, K = a.K, ng = a.ng, elem = a.sf_elem;
     const uint32_t in_stride = round_up_u32(2u * H, 128);
     const uint32_t out_bytes = (uint32_t)H + 4u * nb;       // e4m3 row, then its scales
     const uint32_t out_stride = round_up_u32(out_bytes, 128);
@@ -165,8 +214,11 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
     uint8_t* out = smem + (size_t)stages * in_stride;
     uint64_t* full = reinterpret_cast<uint64_t*>(out + 2 * (size_t)out_stride);
     int32_t* slots = reinterpret_cast<int32_t*>(full + stages);
+    float* bmax = reinterpret_cast<float*>(slots + stages * 32);   // per-row scales: block maxima
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool bulk_scales = ((4u * nb) % 16u) == 0;
+    uint8_t* sf = reinterpret_cast<uint8_t*>(a.recv_scales);
+    const uint32_t sf_row_bytes = (uint32_t)ng * (uint32_t)elem;
+    const bool bulk_scales = !a.sf_col_major && (sf_row_bytes % 16u) == 0;
 
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
@@ -211,13 +263,28 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
         }
         const uint8_t* src = in + (size_t)s * in_stride;
         uint8_t* dst = out + (size_t)o * out_stride;
-        float* dst_scales = reinterpret_cast<float*>(dst + H);
-        for (int b = warp; b < nb; b += kCastThreads / 32) {
-            const uint2 raw = *reinterpret_cast<const uint2*>(src + (size_t)b * 256 + lane * 8);
-            float sc;
-            const uint32_t q = cast_block4(raw, &sc);
-            *reinterpret_cast<uint32_t*>(dst + (size_t)b * 128 + lane * 4) = q;
-            if (lane == 0) dst_scales[b] = sc;
+        uint8_t* dst_sf = dst + H;   // this row's ng scales, elem bytes each
+        if (kPerRow) {
+            for (int b = warp; b < nb; b += kWarps) {
+                const float m = block_amax(*reinterpret_cast<const uint2*>(src + (size_t)b * 256 + lane * 8));
+                if (lane == 0) bmax[b] = m;
+            }
+            __syncthreads();
+            float m = 0.0f;
+            for (int b = lane; b < nb; b += 32) m = fmaxf(m, bmax[b]);
+            const float sc = make_scale<kPow2>(warp_max(m));
+            for (int b = warp; b < nb; b += kWarps) {
+                const uint2 raw = *reinterpret_cast<const uint2*>(src + (size_t)b * 256 + lane * 8);
+                *reinterpret_cast<uint32_t*>(dst + (size_t)b * 128 + lane * 4) = quant4(raw, sc);
+            }
+            if (tid == 0) put_scale(dst_sf, 0, sc, elem);
+        } else {
+            for (int b = warp; b < nb; b += kWarps) {
+                const uint2 raw = *reinterpret_cast<const uint2*>(src + (size_t)b * 256 + lane * 8);
+                const float sc = make_scale<kPow2>(block_amax(raw));
+                *reinterpret_cast<uint32_t*>(dst + (size_t)b * 128 + lane * 4) = quant4(raw, sc);
+                if (lane == 0) put_scale(dst_sf, b, sc, elem);
+            }
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -226,14 +293,14 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
                 const int32_t slot = slots[s * 32 + lane];
                 if (slot >= 0 && (int64_t)slot < a.capacity) {
                     bulk_store(a.recv + (int64_t)slot * H, dst, (uint32_t)H);
-                    if (bulk_scales) bulk_store(a.recv_scales + (int64_t)slot * nb, dst_scales, 4u * nb);
+                    if (bulk_scales) bulk_store(sf + (int64_t)slot * sf_row_bytes, dst_sf, sf_row_bytes);
                 }
             }
             if (!bulk_scales) {
                 for (int k = 0; k < K; ++k) {
                     const int32_t slot = slots[s * 32 + k];
                     if (slot < 0 || (int64_t)slot >= a.capacity) continue;
-                    for (int b = lane; b < nb; b += 32) a.recv_scales[(int64_t)slot * nb + b] = dst_scales[b];
+                    for (int g = lane; g < ng; g += 32) copy_scale(sf, sf_offset(a, slot, g), dst_sf, g, elem);
                 }
             }
             bulk_commit();
@@ -258,13 +325,31 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
             if (row < 0 || (int64_t)row >= a.capacity) continue;
             bulk_store(a.recv + (int64_t)row * H, zero, (uint32_t)H);
             if (bulk_scales)
-                bulk_store(a.recv_scales + (int64_t)row * nb, zero + H, 4u * nb);
+                bulk_store(sf + (int64_t)row * sf_row_bytes, zero + H, sf_row_bytes);
             else
-                for (int b = 0; b < nb; ++b) a.recv_scales[(int64_t)row * nb + b] = 0.0f;
+                for (int g = 0; g < ng; ++g) copy_scale(sf, sf_offset(a, row, g), zero + H, g, elem);
         }
         bulk_commit();
         bulk_wait_all<0>();
     }
+}
+
+template <bool kPerRow, bool kPow2>
+cudaError_t launch_cast_variant(const DispatchArgs& a, cudaStream_t s) {
+    auto kernel = dispatch_cast_kernel<kPerRow, kPow2>;
+    const uint32_t in_stride = round_up_u32(2u * a.H, 128);
+    const uint32_t out_stride = round_up_u32((uint32_t)a.H + 4u * a.nb, 128);
+    const int stages = 3;   // H <= 16384: at most 130 KB of stages
+    const size_t smem = (size_t)stages * in_stride + 2 * (size_t)out_stride + (size_t)stages * 8 +
+                        (size_t)stages * 32 * 4 + (size_t)a.nb * 4;
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    int ctas_per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, kernel, kCastThreads, smem);
+    if (err != cudaSuccess) return err;
+    if (ctas_per_sm > 4) ctas_per_sm = 4;
+    if (ctas_per_sm < 1) ctas_per_sm = 1;
+    return launch_pdl(kernel, dim3(a.sms * ctas_per_sm), dim3(kCastThreads), smem, s, false, a, stages);
 }
 
 }  // namespace
@@ -291,20 +376,21 @@ cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStre
 }
 
 cudaError_t launch_dispatch_cast(const DispatchArgs& a, cudaStream_t s) {
-    const uint32_t in_stride = round_up_u32(2u * a.H, 128);
-    const uint32_t out_stride = round_up_u32((uint32_t)a.H + 4u * a.nb, 128);
-    const int stages = 3;   // H <= 16384: at most 130 KB of stages
-    const size_t smem = (size_t)stages * in_stride + 2 * (size_t)out_stride + (size_t)stages * 8 +
-                        (size_t)stages * 32 * 4;
-    cudaError_t err =
-        cudaFuncSetAttribute(dispatch_cast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    int ctas_per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, dispatch_cast_kernel, kCastThreads, smem);
-    if (err != cudaSuccess) return err;
-    if (ctas_per_sm > 4) ctas_per_sm = 4;
-    if (ctas_per_sm < 1) ctas_per_sm = 1;
-    return launch_pdl(dispatch_cast_kernel, dim3(a.sms * ctas_per_sm), dim3(kCastThreads), smem, s, false, a, stages);
+    const bool per_row = (a.sf_format & EP_SF_PER_ROW) != 0, pow2 = (a.sf_format & EP_SF_POW2) != 0;
+    if (per_row) return pow2 ? launch_cast_variant<true, true>(a, s) : launch_cast_variant<true, false>(a, s);
+    return pow2 ? launch_cast_variant<false, true>(a, s) : launch_cast_variant<false, false>(a, s);
+}
+
+bool set_scale_format(DispatchArgs* a, int scale_format, int64_t rows) {
+    if (scale_format & ~(EP_SF_PER_ROW | EP_SF_POW2 | EP_SF_UE8M0 | EP_SF_COL_MAJOR)) return false;
+    if ((scale_format & EP_SF_UE8M0) && !(scale_format & EP_SF_POW2)) return false;
+    a->sf_format = scale_format;
+    a->ng = (scale_format & EP_SF_PER_ROW) ? 1 : a->nb;
+    a->sf_elem = (scale_format & EP_SF_UE8M0) ? 1 : 4;
+    a->sf_col_major = (scale_format & EP_SF_COL_MAJOR) ? 1 : 0;
+    const int64_t per16 = 16 / a->sf_elem;
+    a->sf_ld = (rows + per16 - 1) / per16 * per16;
+    return true;
 }
 
 }  // namespace ep

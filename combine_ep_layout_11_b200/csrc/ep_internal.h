@@ -35,17 +35,29 @@ struct DispatchArgs {
     const uint8_t* x;          // token rows, row_bytes each (bf16 or e4m3)
     const float* x_scales;     // [T][nb] for e4m3 input
     uint8_t* recv;             // receive rows of the output type
-    float* recv_scales;        // [capacity][nb] for e4m3 output
+    float* recv_scales;        // e4m3 output: [capacity][nb] fp32 (copy); cast: see sf_* below
     const int32_t* pair_slot;  // [T*K]; nullptr: row t goes to row t (plain cast)
     const WsHeader* hdr;       // num_pad
     const int32_t* pad_rows;
     WsHeader* status_hdr;      // status word
     int T, K, H;
     int64_t capacity;
-    int nb;                    // scales per row (H/128) when FP8 is involved
+    int nb;                    // 128-column blocks per row (H/128) when FP8 is involved
     int zero_pad;
     int sms;
+    // scale output of the cast (EP_SF_* bits): ng scales per row (nb, or 1 per
+    // row), sf_elem bytes each (4: fp32, 1: UE8M0); scale (row, g) at byte
+    // (row * ng + g) * sf_elem, or (g * sf_ld + row) * sf_elem column-major
+    int sf_format;
+    int ng;
+    int sf_elem;
+    int sf_col_major;
+    int64_t sf_ld;
 };
+
+// Fill the sf_* fields for `rows` output rows; returns false for an invalid
+// format (unknown bits, UE8M0 without power-of-two rounding).
+bool set_scale_format(DispatchArgs* a, int scale_format, int64_t rows);
 
 // bf16 -> bf16 or e4m3 -> e4m3 row scatter through TMA bulk copies.
 cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStream_t s);

@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define EP_B200_VERSION 2
+#define EP_B200_VERSION 3
 
 /* Host return codes. */
 #define EP_OK 0
@@ -77,6 +77,27 @@ extern "C" {
 /* Element types of token rows. */
 #define EP_DTYPE_BF16 0
 #define EP_DTYPE_FP8_E4M3 1
+
+/*
+ * Scale formats of the FP8 cast (bits of `scale_format`; 0 = one fp32 scale
+ * per 128-column block, row-major [rows, H/128], the default).
+ *   EP_SF_PER_ROW    one scale per row, [rows] (§4.2 per_token_cast_to_fp8:
+ *                    amax over the whole row)
+ *   EP_SF_POW2       each scale rounded up to the smallest power of two not
+ *                    below amax / 448 (§3.3 round_scale), so no value saturates
+ *   EP_SF_UE8M0      scales stored as one UE8M0 byte each, value 2^(b - 127)
+ *                    (§3.3 use_ue8m0); needs EP_SF_POW2
+ *   EP_SF_COL_MAJOR  TMA-aligned column-major scales (§2.1
+ *                    use_tma_aligned_col_major_sf): scale (row, g) at element
+ *                    g * ld + row, ld = rows rounded up to a multiple of 16
+ *                    bytes of elements (4 fp32 or 16 UE8M0 entries); entries
+ *                    [rows, ld) of each column are not written
+ * ep_scale_bytes gives the size of the scale array for a row count.
+ */
+#define EP_SF_PER_ROW 0x1
+#define EP_SF_POW2 0x2
+#define EP_SF_UE8M0 0x4
+#define EP_SF_COL_MAJOR 0x8
 
 /* Supported ranges (EP_ERR_UNSUPPORTED beyond them). */
 #define EP_MAX_TOPK 32
@@ -144,6 +165,13 @@ size_t ep_workspace_bytes(int num_tokens, int num_topk, int num_experts, int exp
  * never overflow (a pure host function). */
 int64_t ep_capacity_rows(int num_tokens, int num_topk, int num_experts, int expert_alignment);
 
+/* Bytes of the scale array of `rows` FP8 rows of `hidden` columns in
+ * `scale_format` (EP_SF_* bits); -1 if the arguments are invalid (rows < 0,
+ * hidden not a positive multiple of 128, unknown bits, UE8M0 without
+ * EP_SF_POW2).  A pure host function.  For ep_dispatch, rows = the handle's
+ * capacity; for ep_cast_fp8, rows = num_tokens. */
+int64_t ep_scale_bytes(int64_t rows, int hidden, int scale_format);
+
 /*
  * Routing layout (§2.1: V2 derives the layout from topk_idx; §3.1: the
  * per-expert receive counts).
@@ -172,17 +200,22 @@ int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens
  *                e4m3 bytes [T, H] if x_dtype == EP_DTYPE_FP8_E4M3
  *   x_scales     device fp32 [T, H/128] for FP8 input, else ignored
  *   hidden H     > 0; H % 8 == 0 for bf16, H % 128 == 0 whenever FP8 is involved
- *   cast_to_fp8  1: bf16 input is cast on the way (§4.2, per 128-column block,
- *                the same bytes ep_cast_fp8 writes) and the receive rows are FP8
+ *   cast_to_fp8  1: bf16 input is cast on the way (§4.2, the same bytes
+ *                ep_cast_fp8 writes for that scale_format) and the receive rows
+ *                are FP8
+ *   scale_format EP_SF_* bits of the cast's scales (0: fp32 per 128-column
+ *                block, row-major); must be 0 unless cast_to_fp8
  *   do_zero_padding  1: the alignment padding rows (and their scales) are zeroed;
  *                0: they are left untouched
  *   recv_x       device, 16-byte aligned: [capacity, H] of the output type
- *   recv_scales  device fp32 [capacity, H/128] when the output is FP8, else ignored
+ *   recv_scales  device, 16-byte aligned, when the output is FP8: fp32
+ *                [capacity, H/128] for FP8 input, else ep_scale_bytes(capacity,
+ *                H, scale_format) bytes in that format; ignored for bf16 output
  * Rows that no pair selects and that are not padding are left untouched.
  */
 int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales,
-                int hidden, int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales,
-                void* stream);
+                int hidden, int cast_to_fp8, int scale_format, int do_zero_padding, void* recv_x,
+                void* recv_scales, void* stream);
 
 /*
  * Layout and dispatch in one call, as V2's dispatch() derives its layout from
@@ -195,7 +228,8 @@ int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const flo
 int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
                        int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
                        ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales, int hidden,
-                       int cast_to_fp8, int do_zero_padding, void* recv_x, float* recv_scales, void* stream);
+                       int cast_to_fp8, int scale_format, int do_zero_padding, void* recv_x,
+                       void* recv_scales, void* stream);
 
 /*
  * Combine (§2.2 weighted, with 0, 1 or 2 output biases; §3.2 unweighted when
@@ -219,16 +253,19 @@ int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float
                const void* bias0, const void* bias1, void* out, void* stream);
 
 /*
- * FP8 cast (§4.2 per_token_cast_to_fp8 with 128-column blocks): for token t
- * and block b, amax = max |x| over the block (clamped below at 1e-4),
- * s = amax / 448 (fp32 division), q = e4m3(x / s) with an fp32 division,
- * round-to-nearest-even and saturation to +-448; scales[t, b] = s.
- * Dequantisation is float(q) * s.
- *   x       device bf16 [T, H], 16-byte aligned, H % 128 == 0
- *   x_fp8   device e4m3 [T, H], 16-byte aligned
- *   scales  device fp32 [T, H/128]
+ * FP8 cast (§4.2 per_token_cast_to_fp8; by default with 128-column blocks):
+ * for token t and group g (a 128-column block, or the whole row with
+ * EP_SF_PER_ROW), amax = max |x| over the group (clamped below at 1e-4),
+ * s = amax / 448 (fp32 division), with EP_SF_POW2 rounded up to a power of two,
+ * q = e4m3(x / s) with an fp32 division, round-to-nearest-even and saturation
+ * to +-448; scale (t, g) = s, stored as fp32 or as a UE8M0 byte, row-major or
+ * column-major as scale_format says.  Dequantisation is float(q) * s.
+ *   x             device bf16 [T, H], 16-byte aligned, H % 128 == 0, H <= 16384
+ *   scale_format  EP_SF_* bits
+ *   x_fp8         device e4m3 [T, H], 16-byte aligned
+ *   scales        device, 16-byte aligned, ep_scale_bytes(T, H, scale_format) bytes
  */
-int ep_cast_fp8(const void* x, int num_tokens, int hidden, void* x_fp8, float* scales,
+int ep_cast_fp8(const void* x, int num_tokens, int hidden, int scale_format, void* x_fp8, void* scales,
                 void* stream);
 
 /* Size of the library-owned workspace behind ep_layout_no_alloc. */

@@ -46,7 +46,7 @@ def test_struct_size_matches_header(lib):
 
 
 def test_pure_host_functions(lib):
-    assert lib.ep_version() == 2
+    assert lib.ep_version() == 3
     assert lib.ep_capacity_rows(4096, 8, 256, 128) == 4096 * 8 + 256 * 127
     assert lib.ep_capacity_rows(128, 4, 16, 1) == 512
     ws = lib.ep_workspace_bytes(4096, 8, 256, 128)
@@ -54,6 +54,19 @@ def test_pure_host_functions(lib):
     assert lib.ep_workspace_bytes(-1, 8, 256, 1) == 0
     assert lib.ep_status_string(0) == b"ok"
     assert lib.ep_status_string(4) == b"bounded wait ran out"
+
+
+def test_scale_bytes(lib):
+    # row-major fp32 per block, per row; UE8M0 bytes; column-major padded to 16 bytes per column
+    assert lib.ep_scale_bytes(100, 7168, 0) == 100 * 56 * 4
+    assert lib.ep_scale_bytes(100, 7168, 1) == 100 * 4
+    assert lib.ep_scale_bytes(100, 7168, 2 | 4) == 100 * 56
+    assert lib.ep_scale_bytes(101, 7168, 8) == 56 * 104 * 4
+    assert lib.ep_scale_bytes(101, 7168, 2 | 4 | 8) == 56 * 112
+    assert lib.ep_scale_bytes(101, 7168, 1 | 2 | 4 | 8) == 112
+    assert lib.ep_scale_bytes(0, 128, 8) == 0
+    for rows, H, fmt in [(-1, 128, 0), (8, 100, 0), (8, 128, 4), (8, 128, 16)]:
+        assert lib.ep_scale_bytes(rows, H, fmt) == -1
 
 
 def _handle(ws_bytes=1 << 20, magic=0):
@@ -106,35 +119,42 @@ def test_layout_dispatch_host_checks(lib):
     p = ctypes.c_void_p(0x10000)
     s = _handle()
     # layout-side errors
-    assert lib.ep_layout_dispatch(p, None, 8, 2, 8, 3, 1, 0, ctypes.byref(s), p, 0, None, 256, 0, 0, p, None,
+    assert lib.ep_layout_dispatch(p, None, 8, 2, 8, 3, 1, 0, ctypes.byref(s), p, 0, None, 256, 0, 0, 0, p, None,
                                   None) == 1
     # dispatch-side errors leave the handle untouched
-    assert lib.ep_layout_dispatch(p, None, 8, 2, 8, 2, 1, 0, ctypes.byref(s), p, 0, None, 100, 0, 0, p, None,
+    assert lib.ep_layout_dispatch(p, None, 8, 2, 8, 2, 1, 0, ctypes.byref(s), p, 0, None, 100, 0, 0, 0, p, None,
                                   None) == 1
     assert s.magic == 0 and s.num_tokens == 0
-    assert lib.ep_layout_dispatch(p, None, 8, 2, 8, 2, 1, 0, None, p, 0, None, 256, 0, 0, p, None, None) == 1
+    assert lib.ep_layout_dispatch(p, None, 8, 2, 8, 2, 1, 0, None, p, 0, None, 256, 0, 0, 0, p, None,
+                                  None) == 1
 
 
 def test_dispatch_combine_host_checks(lib):
     s = _handle()                        # not filled by ep_layout: rejected
     p = ctypes.c_void_p(0x10000)
-    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 256, 0, 0, p, None, None) == 1
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 256, 0, 0, 0, p, None, None) == 1
     assert lib.ep_combine(ctypes.byref(s), p, 256, None, None, None, p, None) == 1
     s = _handle(magic=0x45504C31)        # a handle as ep_layout leaves it
     s.num_tokens, s.num_topk, s.num_experts, s.num_ranks, s.expert_alignment = 8, 2, 8, 2, 1
-    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 100, 0, 0, p, None, None) == 1      # H % 8
-    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 136, 1, 0, p, p, None) == 1         # FP8: H % 128
-    assert lib.ep_dispatch(ctypes.byref(s), p, 1, None, 256, 0, 0, p, p, None) == 1         # fp8 in, no scales
-    assert lib.ep_dispatch(ctypes.byref(s), p, 1, p, 256, 1, 0, p, p, None) == 1            # cast of fp8 input
-    assert lib.ep_dispatch(ctypes.byref(s), ctypes.c_void_p(0x10008), 0, None, 256, 0, 0, p, None, None) == 1
-    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 32768, 1, 0, p, p, None) == 6       # cast row too large
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 100, 0, 0, 0, p, None, None) == 1      # H % 8
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 136, 1, 0, 0, p, p, None) == 1         # FP8: H % 128
+    assert lib.ep_dispatch(ctypes.byref(s), p, 1, None, 256, 0, 0, 0, p, p, None) == 1         # fp8 in, no scales
+    assert lib.ep_dispatch(ctypes.byref(s), p, 1, p, 256, 1, 0, 0, p, p, None) == 1            # cast of fp8 input
+    assert lib.ep_dispatch(ctypes.byref(s), ctypes.c_void_p(0x10008), 0, None, 256, 0, 0, 0, p, None, None) == 1
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 32768, 1, 0, 0, p, p, None) == 6       # cast row too large
     assert lib.ep_combine(ctypes.byref(s), p, 100, None, None, None, p, None) == 1          # H % 8
     assert lib.ep_combine(ctypes.byref(s), p, 256, None, None, None, ctypes.c_void_p(0x10004), None) == 1
     assert lib.ep_combine(ctypes.byref(s), p, 256, None, None, p, p, None) == 1             # bias1 alone
     assert lib.ep_combine(ctypes.byref(s), p, 256, None, ctypes.c_void_p(0x10008), None, p, None) == 1
     assert lib.ep_combine(ctypes.byref(s), p, 256, None, p, ctypes.c_void_p(0x10002), p, None) == 1
-    assert lib.ep_cast_fp8(p, 8, 100, p, p, None) == 1
-    assert lib.ep_cast_fp8(p, 8, 32768, p, p, None) == 6
+    assert lib.ep_cast_fp8(p, 8, 100, 0, p, p, None) == 1
+    assert lib.ep_cast_fp8(p, 8, 32768, 0, p, p, None) == 6
+    # scale formats: only with the cast; UE8M0 needs power-of-two rounding; no unknown bits
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 256, 0, 2, 0, p, p, None) == 1
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 256, 1, 4, 0, p, p, None) == 1
+    assert lib.ep_dispatch(ctypes.byref(s), p, 0, None, 256, 1, 16, 0, p, p, None) == 1
+    assert lib.ep_cast_fp8(p, 8, 256, 4, p, p, None) == 1
+    assert lib.ep_cast_fp8(p, 0, 256, 32, p, p, None) == 1
     flags = ctypes.c_uint32(0)
     assert lib.ep_get_status(ctypes.byref(s), None, None) == 1
     assert lib.ep_selftest_bounded_wait(ctypes.byref(s), 2_000_000_000, None) == 1

@@ -70,7 +70,7 @@ def test_no_alloc_layout_matches_ep_layout_twice(ep):
         assert rc == 0, lib.ep_status_string(rc)
         assert s.workspace and s.workspace_bytes == 4 << 20
         recv = torch.empty_like(ref_recv)
-        rc = lib.ep_dispatch(ctypes.byref(s), ctypes.c_void_p(x.data_ptr()), 0, None, cfg["H"], 0,
+        rc = lib.ep_dispatch(ctypes.byref(s), ctypes.c_void_p(x.data_ptr()), 0, None, cfg["H"], 0, 0,
                              int(cfg["zero_pad"]), ctypes.c_void_p(recv.data_ptr()), None, stream)
         assert rc == 0
         flags = ctypes.c_uint32(0)
