@@ -50,6 +50,9 @@ def parse():
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--fused", action="store_true",
                    help="the single ep_layout_dispatch call instead of ep_layout + ep_dispatch")
+    p.add_argument("--layout", default="expand", choices=["expand", "rank"],
+                   help="expand: one receive row per (token, k) pair (ep_layout); rank: one per (token, rank) "
+                        "reached (ep_rank_layout) with V1's unweighted combine")
     return p.parse_args()
 
 
@@ -170,6 +173,18 @@ def algorithmic_bytes(cfg, cnt, A):
     return dict(layout=layout_b, dispatch=dispatch_b, combine=combine_b, N=N, Np=Np, pad_rows=Np - N)
 
 
+def algorithmic_bytes_rank(cfg, rows, N):
+    """The per-token-per-rank form: `rows` receive rows, one per (token, rank) reached."""
+    T, H, K, E, R = cfg["T"], cfg["H"], cfg["K"], cfg["E"], cfg["R"]
+    nb = H // 128
+    out_row = (H + 4 * nb) if cfg["fp8"] else 2 * H
+    # idx and weights read, is_token_in_rank + token_slot, recv_src + recv_topk_idx/weights, counts
+    layout_b = T * K * 12 + T * R * 5 + rows * (4 + K * 12) + E * 8 + R * 8
+    dispatch_b = T * 2 * H + rows * out_row + T * R * 4
+    combine_b = rows * 2 * H + T * 2 * H + T * R * 4
+    return dict(layout=layout_b, dispatch=dispatch_b, combine=combine_b, N=N, Np=rows, pad_rows=0)
+
+
 # --------------------------------------------------------------------------
 # our implementation
 # --------------------------------------------------------------------------
@@ -193,7 +208,14 @@ def run_ours(args, rank, world, local_rank):
     idx = torch.from_numpy(inp["topk_idx"]).to(dev)
     w = torch.from_numpy(inp["topk_weights"]).to(dev)
     x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
-    lay = ep.Layout(T, K, E, R, A, dev, num_max_tokens_per_rank=cfg["max_tokens_per_rank"])
+    per_rank = args.layout == "rank"
+    if per_rank and args.fused:
+        raise SystemExit("--fused applies to the expand layout only")
+    if per_rank:
+        lay = ep.RankLayout(T, K, E, R, A, dev)
+    else:
+        lay = ep.Layout(T, K, E, R, A, dev, num_max_tokens_per_rank=cfg["max_tokens_per_rank"])
+    cw = None if per_rank else w            # V1's combine is a plain sum over the ranks
     cap = lay.capacity
     fp8 = cfg["fp8"]
     recv = torch.empty((cap, H), dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16, device=dev)
@@ -208,22 +230,30 @@ def run_ours(args, rank, world, local_rank):
         else:
             ep.dispatch(lay, x, do_zero_padding=cfg["zero_pad"], out=recv)
 
+    def do_layout(d_idx, d_w):
+        if per_rank:
+            ep.rank_layout(d_idx, d_w, E, R, A, out=lay)
+        else:
+            ep.layout(d_idx, d_w, E, R, A, cfg["max_tokens_per_rank"], out=lay)
+
     # expert outputs for combine: identity experts (bf16), or seeded outputs for FP8
-    ep.layout(idx, w, E, R, A, cfg["max_tokens_per_rank"], out=lay)
+    do_layout(idx, w)
     dispatch()
     torch.cuda.synchronize(dev)
     if fp8:
         y = torch.from_numpy(workload.expert_outputs(cfg, cap).view(np.int16)).to(dev).view(torch.bfloat16)
     else:
         y = recv.clone()
-    cnt = lay.num_recv_tokens_per_expert.cpu().numpy()
-    nbytes = algorithmic_bytes(cfg, cnt, A)
+    if per_rank:
+        nbytes = algorithmic_bytes_rank(cfg, lay.num_recv_rows(), int((idx >= 0).sum()))
+    else:
+        nbytes = algorithmic_bytes(cfg, lay.num_recv_tokens_per_expert.cpu().numpy(), A)
 
     def step(evs=None):
         if evs:
             evs[0].record(stream)
         if not args.fused:
-            ep.layout(idx, w, E, R, A, cfg["max_tokens_per_rank"], out=lay)
+            do_layout(idx, w)
             if evs:
                 evs[1].record(stream)
             dispatch()
@@ -234,7 +264,7 @@ def run_ours(args, rank, world, local_rank):
                 evs[1].record(stream)
         if evs:
             evs[2].record(stream)
-        ep.combine(lay, y, w, out=out)
+        ep.combine(lay, y, cw, out=out)
         if evs:
             evs[3].record(stream)
 
@@ -244,7 +274,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     code, flags = ep.get_status(lay)
     assert code == 0, "device status %d (flags %d)" % (code, flags)
-    if not fp8 and cfg["drop"] == 0:   # identity experts with weights summing to 1 reproduce x
+    if not fp8 and cfg["drop"] == 0 and not per_rank:   # identity experts, weights summing to 1: x again
         has = (idx >= 0).any(dim=1)
         assert torch.equal(out[has].float(), x[has].float()), "combine(dispatch(x)) != x"
 
@@ -280,7 +310,7 @@ def run_ours(args, rank, world, local_rank):
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush)
+        e2e = run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush, do_layout, per_rank)
         e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dist, dev)
 
     if rank != 0:
@@ -317,8 +347,9 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "fp8-e4m3/bf16" if fp8 else "bf16",
         "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
-        "config": {"workload": "%s: T=%d H=%d E=%d top-%d R=%d align=%d zero_pad=%s%s" % (
-            cfg["name"], T, H, E, K, R, A, cfg["zero_pad"], " fp8-cast" if fp8 else ""),
+        "config": {"workload": "%s: T=%d H=%d E=%d top-%d R=%d align=%d zero_pad=%s%s%s" % (
+            cfg["name"], T, H, E, K, R, A, cfg["zero_pad"], " fp8-cast" if fp8 else "",
+            " layout=per-rank (one row per token and rank reached, unweighted combine)" if per_rank else ""),
             "global_batch": T * world, "parallelism": "replicas x%d (R=%d virtual ranks per GPU)" % (world, R),
             "l2": "flushed by a 256 MiB write before every step, outside the timed events",
             "pairs": nbytes["N"], "recv_rows": nbytes["Np"], "pad_rows": nbytes["pad_rows"],
@@ -333,9 +364,9 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "kernel": top_kernel,
                      "achieved": round(disp_gbs, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(disp_gbs / peak, 4),
-                     "traffic": ncu_traffic(top_kernel, cfg["name"]),
+                     "traffic": ncu_traffic(top_kernel, cfg["name"] + ("/per-rank" if per_rank else "")),
                      "algorithmic_bytes_per_launch": top_bytes},
-        "gpu_launches": args.steps * (2 if (args.fused and not fp8) else 3),
+        "gpu_launches": args.steps * (5 if per_rank else (2 if (args.fused and not fp8) else 3)),
         "wall_s_timed_region": round(wall, 4),
     }
     if clock_info:
@@ -345,14 +376,14 @@ def run_ours(args, rank, world, local_rank):
                        "ms_per_step": round(e2e["ms_per_step"], 4),
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, inp)
+        line["cpu_baseline"] = cpu_baseline(cfg, inp, per_rank)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
     return line
 
 
-def run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush):
+def run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush, do_layout, per_rank):
     """Same step through the public API with host buffers: pinned H2D of the
     step's inputs, the three calls, D2H of the combined output, all timed."""
     T, H = cfg["T"], cfg["H"]
@@ -379,9 +410,9 @@ def run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush):
                                cast_to_fp8=fp8, do_zero_padding=cfg["zero_pad"], out_layout=lay, out=recv,
                                out_scales=recv_s)
         else:
-            ep.layout(d_idx, d_w, cfg["E"], cfg["R"], cfg["A"], cfg["max_tokens_per_rank"], out=lay)
+            do_layout(d_idx, d_w)
             ep.dispatch(lay, xb, cast_to_fp8=fp8, do_zero_padding=cfg["zero_pad"], out=recv, out_scales=recv_s)
-        ep.combine(lay, y, d_w, out=d_out)
+        ep.combine(lay, y, None if per_rank else d_w, out=d_out)
         h_out.copy_(d_out.view(torch.int16), non_blocking=True)
         if e1:
             e1.record(stream)
@@ -403,29 +434,32 @@ def run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush):
 # --------------------------------------------------------------------------
 # CPU oracle: the baseline leg and the reference arm
 # --------------------------------------------------------------------------
-def oracle_step_inputs(cfg, inp):
+def oracle_step_inputs(cfg, inp, per_rank=False):
     import oracle
-    lay = oracle.layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"],
-                        cfg["max_tokens_per_rank"])
+    if per_rank:
+        lay = oracle.rank_layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"])
+    else:
+        lay = oracle.layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"],
+                            cfg["max_tokens_per_rank"])
     y = oracle.dispatch_rows(inp["x"], lay, cfg["zero_pad"]) if not cfg["fp8"] else \
         workload.expert_outputs(cfg, int(lay["off"][-1]))
     return dict(inp, y=y)
 
 
-def time_oracle(cfg, inp, budget_s=10.0, min_steps=1, max_steps=None):
+def time_oracle(cfg, inp, budget_s=10.0, min_steps=1, max_steps=None, per_rank=False):
     import oracle
-    full = oracle_step_inputs(cfg, inp)
+    full = oracle_step_inputs(cfg, inp, per_rank)
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle.step(full, cfg)
+        oracle.step(full, cfg, per_rank)
         n += 1
         el = time.perf_counter() - t0
         if (n >= min_steps and el >= budget_s) or (max_steps and n >= max_steps):
             return n, el
 
 
-def cpu_baseline(cfg, inp):
-    n, el = time_oracle(cfg, inp, budget_s=10.0)
+def cpu_baseline(cfg, inp, per_rank=False):
+    n, el = time_oracle(cfg, inp, budget_s=10.0, per_rank=per_rank)
     return {"value": round(cfg["T"] * n / el, 1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": "%d full step(s) of the %s workload (layout, dispatch%s, combine), single-threaded C, "
                       "%d host cores present" % (n, cfg["name"], " with cast" if cfg["fp8"] else "",
@@ -437,14 +471,15 @@ def run_reference(args, rank, world):
         return None
     cfg = workload.config(args.workload)
     inp = workload.inputs(cfg)
-    full = oracle_step_inputs(cfg, inp)
+    per_rank = args.layout == "rank"
+    full = oracle_step_inputs(cfg, inp, per_rank)
     import oracle
     for _ in range(args.warmup):
-        oracle.step(full, cfg)
+        oracle.step(full, cfg, per_rank)
     ts = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.step(full, cfg)
+        oracle.step(full, cfg, per_rank)
         ts.append(time.perf_counter() - t0)
     ms = float(np.mean(ts)) * 1e3
     v = round(cfg["T"] / (ms * 1e-3), 1)
@@ -452,7 +487,7 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp8-e4m3/bf16" if cfg["fp8"] else "bf16",
             "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
-            "config": {"workload": cfg["name"], "global_batch": cfg["T"]},
+            "config": {"workload": cfg["name"] + (" layout=per-rank" if per_rank else ""), "global_batch": cfg["T"]},
             "impl": "reference",
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": "the full %s workload per step (single-threaded C oracle)" % cfg["name"]},

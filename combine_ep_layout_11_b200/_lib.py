@@ -29,7 +29,7 @@ class EpLayout(ctypes.Structure):
         ("expert_alignment", ctypes.c_int32),
         ("num_max_tokens_per_rank", ctypes.c_int32),
         ("magic", ctypes.c_uint32),
-        ("reserved", ctypes.c_uint32),
+        ("kind", ctypes.c_uint32),
         ("cumulative_local_expert_recv_stats", ctypes.c_void_p),
     ]
 
@@ -43,6 +43,8 @@ SIGNATURES = {
     "ep_layout": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp]),
     "ep_layout_no_alloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp]),
     "ep_scale_bytes": (_i64, [_i64, _i, _i]),
+    "ep_rank_workspace_bytes": (_sz, [_i, _i, _i]),
+    "ep_rank_layout": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _LP, _vp]),
     "ep_dispatch": (_i, [_LP, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "ep_layout_dispatch": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp,
                                 _vp]),

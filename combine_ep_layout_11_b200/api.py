@@ -172,6 +172,85 @@ def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment=1,
     return lay
 
 
+class RankLayout:
+    """The handle of the per-token-per-rank layout (§2.1 without do_expand; §3.1's
+    V1 layout quantities) plus its extra outputs.
+
+    Tensors (device): ``num_tokens_per_rank`` [R], ``rank_offset`` [R+1],
+    ``token_slot`` [T, R] (receive row of (t, r), -1 if t does not reach r),
+    ``is_token_in_rank`` bool [T, R], ``num_tokens_per_expert`` and
+    ``num_recv_tokens_per_expert`` (aligned) [E], ``recv_src_token`` [capacity],
+    ``recv_topk_idx`` int64 / ``recv_topk_weights`` fp32 [capacity, K].
+    ``dispatch`` and ``combine`` (without weights: V1's plain sum) take it as
+    their handle.
+    """
+
+    def __init__(self, num_tokens, num_topk, num_experts, num_ranks, expert_alignment, device, capacity=None):
+        T, K, E, R = num_tokens, num_topk, num_experts, num_ranks
+        if capacity is None:
+            capacity = T * R
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.num_tokens, self.num_topk, self.num_experts, self.num_ranks = T, K, E, R
+        self.expert_alignment = expert_alignment
+        self.capacity = int(capacity)
+        self.device = dev
+        n = max(self.capacity, 1)
+        self.num_tokens_per_rank = torch.empty(R, **i32)
+        self.rank_offset = torch.empty(R + 1, **i32)
+        self._token_slot_buf = torch.empty(max(T * R, 1), **i32)
+        self.token_slot = self._token_slot_buf[:T * R].view(T, R)
+        self._in_rank_buf = torch.empty(max(T * R, 1), dtype=torch.uint8, device=dev)
+        self.is_token_in_rank = self._in_rank_buf[:T * R].view(T, R).view(torch.bool)
+        self.num_tokens_per_expert = torch.empty(E, **i32)
+        self.num_recv_tokens_per_expert = torch.empty(E, **i32)
+        self.recv_src_token = torch.empty(n, **i32)
+        self.recv_topk_idx = torch.empty((n, K), dtype=torch.int64, device=dev)
+        self.recv_topk_weights = torch.empty((n, K), dtype=torch.float32, device=dev)
+        nbytes = int(_lib.load().ep_rank_workspace_bytes(T, R, E))
+        if nbytes == 0:
+            raise EpError(EP_ERR_INVALID_ARG, "workspace size")
+        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)   # zeroed before first use
+        st = _lib.EpLayout()
+        st.num_recv_tokens_per_expert = self.num_tokens_per_rank.data_ptr()
+        st.expert_offset = self.rank_offset.data_ptr()
+        st.pair_slot = self._token_slot_buf.data_ptr()
+        st.recv_src_token = self.recv_src_token.data_ptr()
+        st.workspace = self.workspace.data_ptr()
+        st.workspace_bytes = nbytes
+        st.capacity = self.capacity
+        self.struct = st
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+    def num_recv_rows(self):
+        """Rows in use, rank_offset[R] (reads the device: synchronises)."""
+        return int(self.rank_offset[-1].item())
+
+
+def rank_layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment=1, capacity=None, out=None):
+    """Per-token-per-rank layout of ``topk_idx`` [T, K] int64 (§2.1 default
+    receive form; §3.1 num_tokens_per_rank / is_token_in_rank /
+    num_tokens_per_expert).  ``out`` may be a ``RankLayout`` of the same sizes."""
+    L = _lib.load()
+    assert topk_idx.dtype == torch.int64 and topk_idx.dim() == 2 and topk_idx.is_contiguous()
+    T, K = topk_idx.shape
+    if topk_weights is not None:
+        assert topk_weights.dtype == torch.float32 and topk_weights.shape == (T, K)
+        assert topk_weights.is_contiguous()
+    if out is not None:
+        assert (out.num_tokens, out.num_topk, out.num_experts, out.num_ranks) == (T, K, num_experts, num_ranks)
+    lay = out if out is not None else RankLayout(T, K, num_experts, num_ranks, expert_alignment,
+                                                 topk_idx.device, capacity)
+    lay.expert_alignment = expert_alignment
+    _check(L.ep_rank_layout(_ptr(topk_idx), _ptr(topk_weights), T, K, num_experts, num_ranks, expert_alignment,
+                            _ptr(lay._in_rank_buf), _ptr(lay.num_tokens_per_expert),
+                            _ptr(lay.num_recv_tokens_per_expert), _ptr(lay.recv_topk_idx),
+                            _ptr(lay.recv_topk_weights), lay.ref(), _stream(topk_idx.device)), "ep_rank_layout")
+    return lay
+
+
 def dispatch(lay, x, x_scales=None, cast_to_fp8=False, do_zero_padding=False, out=None, out_scales=None,
              scale_fmt=0):
     """Scatter token rows into the receive buffer (§2.1 dispatch()).

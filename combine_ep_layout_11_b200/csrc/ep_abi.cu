@@ -57,6 +57,7 @@ int prepare_layout(const int64_t* topk_idx, const float* topk_weights, int T, in
     layout->expert_alignment = A;
     layout->num_max_tokens_per_rank = num_max_tokens_per_rank;
     layout->magic = kLayoutMagic;
+    layout->kind = EP_LAYOUT_EXPAND;
 
     uint8_t* wsb = reinterpret_cast<uint8_t*>(layout->workspace);
     a->topk_idx = topk_idx;
@@ -171,6 +172,103 @@ int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens
     return ep::launch_layout(a, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
+size_t ep_rank_workspace_bytes(int num_tokens, int num_ranks, int num_experts) {
+    if (num_tokens < 0 || num_ranks < 1 || num_experts < 1) return 0;
+    return ep::rank_ws_layout(num_tokens, num_ranks, num_experts).total;
+}
+
+int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
+                   int num_experts, int num_ranks, int expert_alignment, uint8_t* is_token_in_rank,
+                   int32_t* num_tokens_per_expert, int32_t* num_recv_tokens_per_expert, int64_t* recv_topk_idx,
+                   float* recv_topk_weights, ep_layout_t* layout, void* stream) {
+    const int T = num_tokens, K = num_topk, E = num_experts, R = num_ranks, A = expert_alignment;
+    if (!layout) return EP_ERR_INVALID_ARG;
+    if (T < 0 || K < 1 || E < 1 || R < 1 || A < 1) return EP_ERR_INVALID_ARG;
+    if (K > EP_MAX_TOPK || E > EP_MAX_EXPERTS || R > EP_MAX_TOPK) return EP_ERR_UNSUPPORTED;
+    if (E % R != 0 || T % R != 0) return EP_ERR_INVALID_ARG;
+    if ((int64_t)T * R > INT_MAX) return EP_ERR_UNSUPPORTED;
+    if (layout->capacity < 0) return EP_ERR_INVALID_ARG;
+    if (layout->capacity > INT_MAX) return EP_ERR_UNSUPPORTED;
+    if ((T > 0 && !topk_idx) || !layout->num_recv_tokens_per_expert || !layout->expert_offset ||
+        !layout->pair_slot || !layout->recv_src_token || !layout->workspace)
+        return EP_ERR_INVALID_ARG;
+    if (!aligned(topk_idx, 8) || !aligned(topk_weights, 4) || !aligned(num_tokens_per_expert, 4) ||
+        !aligned(num_recv_tokens_per_expert, 4) || !aligned(recv_topk_idx, 8) || !aligned(recv_topk_weights, 4) ||
+        !aligned(layout->num_recv_tokens_per_expert, 4) || !aligned(layout->expert_offset, 4) ||
+        !aligned(layout->pair_slot, 4) || !aligned(layout->recv_src_token, 4) || !aligned(layout->workspace, 256))
+        return EP_ERR_INVALID_ARG;
+    const ep::RankWsLayout ws = ep::rank_ws_layout(T, R, E);
+    if (layout->workspace_bytes < ws.total) return EP_ERR_INVALID_ARG;
+
+    layout->num_tokens = T;
+    layout->num_topk = R;
+    layout->num_experts = R;
+    layout->num_ranks = R;
+    layout->expert_alignment = 1;
+    layout->num_max_tokens_per_rank = 0;
+    layout->magic = kLayoutMagic;
+    layout->kind = EP_LAYOUT_PER_RANK;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t* wsb = reinterpret_cast<uint8_t*>(layout->workspace);
+    if (T == 0) {
+        if (cudaMemsetAsync(layout->workspace, 0, sizeof(ep::WsHeader), s) != cudaSuccess ||
+            cudaMemsetAsync(layout->num_recv_tokens_per_expert, 0, (size_t)R * 4, s) != cudaSuccess ||
+            cudaMemsetAsync(layout->expert_offset, 0, (size_t)(R + 1) * 4, s) != cudaSuccess ||
+            (num_tokens_per_expert && cudaMemsetAsync(num_tokens_per_expert, 0, (size_t)E * 4, s) != cudaSuccess) ||
+            (num_recv_tokens_per_expert &&
+             cudaMemsetAsync(num_recv_tokens_per_expert, 0, (size_t)E * 4, s) != cudaSuccess))
+            return EP_ERR_CUDA;
+        return EP_OK;
+    }
+    int64_t* rank_idx = reinterpret_cast<int64_t*>(wsb + ws.rank_idx_off);
+    int32_t* counts = reinterpret_cast<int32_t*>(wsb + ws.counts_off);
+
+    ep::RankPrepArgs p;
+    p.topk_idx = topk_idx;
+    p.T = T; p.K = K; p.E = E; p.R = R;
+    p.rank_idx = rank_idx;
+    p.in_rank = is_token_in_rank;
+    p.counts = counts;
+    p.hdr = header(layout);
+
+    ep::LayoutArgs la;
+    la.topk_idx = rank_idx;
+    la.topk_weights = nullptr;
+    la.T = T; la.K = R; la.E = R; la.R = R; la.A = 1;
+    la.C = 0;
+    la.CT = 0;
+    la.capacity = layout->capacity;
+    la.cnt = layout->num_recv_tokens_per_expert;
+    la.off = layout->expert_offset;
+    la.pair_slot = layout->pair_slot;
+    la.recv_src = layout->recv_src_token;
+    la.recv_w = reinterpret_cast<float*>(wsb + ws.scratch_w_off);
+    la.recv_lexp = reinterpret_cast<int32_t*>(wsb + ws.scratch_lexp_off);
+    la.hdr = header(layout);
+    la.table = reinterpret_cast<int32_t*>(wsb + ws.expand.table_off);
+    la.padpre = reinterpret_cast<int32_t*>(wsb + ws.expand.padpre_off);
+    la.pad_rows = reinterpret_cast<int32_t*>(wsb + ws.expand.padrows_off);
+    la.stats = nullptr;
+
+    ep::RankPostArgs post;
+    post.topk_idx = topk_idx;
+    post.topk_weights = topk_weights;
+    post.rank_off = layout->expert_offset;
+    post.recv_src = layout->recv_src_token;
+    post.counts = counts;
+    post.T = T; post.K = K; post.E = E; post.R = R; post.A = A;
+    post.capacity = layout->capacity;
+    post.recv_topk_idx = recv_topk_idx;
+    post.recv_topk_w = recv_topk_weights;
+    post.num_tokens_per_expert = num_tokens_per_expert;
+    post.num_recv_per_expert = num_recv_tokens_per_expert;
+
+    int sms = 0;
+    int rc = device_sms(&sms);
+    if (rc != EP_OK) return rc;
+    return ep::launch_rank_layout(p, la, post, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
 int64_t ep_scale_bytes(int64_t rows, int hidden, int scale_format) {
     if (rows < 0 || hidden <= 0 || hidden % 128 != 0) return -1;
     ep::DispatchArgs a;
@@ -230,6 +328,7 @@ int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float
     if (H <= 0 || H % 8 != 0) return EP_ERR_INVALID_ARG;
     if (T > 0 && (!y || !out)) return EP_ERR_INVALID_ARG;
     if (bias1 && !bias0) return EP_ERR_INVALID_ARG;
+    if (layout->kind == EP_LAYOUT_PER_RANK && topk_weights) return EP_ERR_INVALID_ARG;
     if (!aligned(y, 16) || !aligned(out, 16) || !aligned(topk_weights, 4) || !aligned(bias0, 16) ||
         !aligned(bias1, 16))
         return EP_ERR_INVALID_ARG;

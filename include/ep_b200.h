@@ -16,7 +16,11 @@
  *                §4.1 refs.py ordered_accumulate: one fixed order, so results
  *                are bitwise reproducible.
  *   ep_cast_fp8  §4.2 math.py per_token_cast_to_fp8, with one fp32 scale per
- *                128-column block of a token row.
+ *                128-column block of a token row (or the §3.3 / §2.1 scale
+ *                variants: per row, power of two, UE8M0, column-major).
+ *   ep_rank_layout  §2.1 dispatch() without do_expand (one receive row per
+ *                token and destination rank) with §3.1's V1 layout quantities;
+ *                its handle serves ep_dispatch and §3.2's unweighted combine.
  * The placement also matches the last stages of the Ascend full-mesh dispatch
  * on the "URMA" tag page (count reconciliation, prefix-sum placement, reorder).
  *
@@ -58,7 +62,7 @@
 extern "C" {
 #endif
 
-#define EP_B200_VERSION 3
+#define EP_B200_VERSION 4
 
 /* Host return codes. */
 #define EP_OK 0
@@ -154,9 +158,13 @@ typedef struct ep_layout_t {
     int32_t expert_alignment;
     int32_t num_max_tokens_per_rank;
     uint32_t magic;
-    uint32_t reserved;
+    uint32_t kind;                                 /* EP_LAYOUT_*, set by the layout call */
     int32_t* cumulative_local_expert_recv_stats;   /* optional, see above */
 } ep_layout_t;
+
+/* Receive forms of a handle (its `kind` field). */
+#define EP_LAYOUT_EXPAND 0     /* ep_layout: one row per selected (token, k) pair */
+#define EP_LAYOUT_PER_RANK 1   /* ep_rank_layout: one row per (token, rank) reached */
 
 /* Bytes of workspace ep_layout needs for these sizes (a pure host function). */
 size_t ep_workspace_bytes(int num_tokens, int num_topk, int num_experts, int expert_alignment);
@@ -192,6 +200,47 @@ int64_t ep_scale_bytes(int64_t rows, int hidden, int scale_format);
 int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
               int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
               ep_layout_t* layout, void* stream);
+
+/*
+ * Per-token-per-rank layout: the receive form of §2.1 dispatch() without
+ * do_expand, with the V1 layout quantities of §3.1 (num_tokens_per_rank,
+ * is_token_in_rank, num_tokens_per_expert) and V1's receive outputs
+ * (recv_topk_idx, recv_topk_weights, num_recv_tokens_per_expert_list).
+ * Token t reaches rank r when some topk_idx[t, k] is one of r's experts
+ * [r*E/R, (r+1)*E/R); it then gets one receive row in r's region.  Rows of
+ * rank r are [off[r], off[r+1]) in ascending token order (source rank, then
+ * token).  No padding rows.
+ *   topk_idx, topk_weights, T, K, E, R as for ep_layout; 1 <= R <= 32
+ *   expert_alignment A >= 1: only for num_recv_tokens_per_expert
+ *   is_token_in_rank            device uint8 [T, R] or NULL: 1 / 0
+ *   num_tokens_per_expert       device int32 [E] or NULL: pairs per expert
+ *   num_recv_tokens_per_expert  device int32 [E] or NULL: align(that, A)
+ *   recv_topk_idx               device int64 [capacity, K] or NULL: for row
+ *                               (t, r), topk_idx[t, k] - r*E/R where that
+ *                               expert is on r, else -1
+ *   recv_topk_weights           device fp32 [capacity, K] or NULL: the topk
+ *                               weight (1 without weights) on those entries, else 0
+ *   layout  in: the handle's pointers, capacity (T*R rows never overflow),
+ *           workspace of ep_rank_workspace_bytes(T, R, E) bytes (zero-filled
+ *           before first use, like ep_layout's);
+ *           the fields then mean: num_recv_tokens_per_expert = num_tokens_per_rank
+ *           [R], expert_offset = rank offsets [R+1] (off[R] = rows used),
+ *           pair_slot = token_slot [T, R] (row of (t, r) or -1),
+ *           recv_src_token [capacity]; recv_weight and recv_local_expert are
+ *           not used and may be NULL.
+ *           out: kind = EP_LAYOUT_PER_RANK, num_tokens = T, and num_topk =
+ *           num_experts = num_ranks = R (each token has R possible
+ *           destinations), expert_alignment = 1.
+ * The handle works with ep_dispatch (rows per (token, rank)) and ep_combine
+ * (§3.2 V1: topk_weights must be NULL; out[t] = the plain sum over the ranks
+ * the token reached, in ascending rank order, plus the biases).  Device-side
+ * errors as for ep_layout.  Four launches: a memset, three kernels.
+ */
+size_t ep_rank_workspace_bytes(int num_tokens, int num_ranks, int num_experts);
+int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
+                   int num_experts, int num_ranks, int expert_alignment, uint8_t* is_token_in_rank,
+                   int32_t* num_tokens_per_expert, int32_t* num_recv_tokens_per_expert, int64_t* recv_topk_idx,
+                   float* recv_topk_weights, ep_layout_t* layout, void* stream);
 
 /*
  * Dispatch (§2.1): for every selected pair (t, k), receive row
@@ -243,7 +292,8 @@ int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int n
  *   y            device bf16 [capacity, H], 16-byte aligned: expert outputs in
  *                receive order; padding rows are never read
  *   hidden H     > 0, H % 8 == 0
- *   topk_weights device fp32 [T, K] or NULL (unit weights)
+ *   topk_weights device fp32 [T, K] or NULL (unit weights); must be NULL for
+ *                a per-rank handle (EP_LAYOUT_PER_RANK: K = R, a plain sum)
  *   bias0, bias1 device bf16 [T, H], 16-byte aligned, or NULL; bias1 without
  *                bias0 is EP_ERR_INVALID_ARG
  *   out          device bf16 [T, H], 16-byte aligned; may not alias y, and may

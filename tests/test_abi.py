@@ -46,7 +46,7 @@ def test_struct_size_matches_header(lib):
 
 
 def test_pure_host_functions(lib):
-    assert lib.ep_version() == 3
+    assert lib.ep_version() == 4
     assert lib.ep_capacity_rows(4096, 8, 256, 128) == 4096 * 8 + 256 * 127
     assert lib.ep_capacity_rows(128, 4, 16, 1) == 512
     ws = lib.ep_workspace_bytes(4096, 8, 256, 128)
@@ -96,6 +96,40 @@ def test_layout_host_checks(lib, T, K, E, R, A, limit, expect):
     s = _handle()
     rc = lib.ep_layout(ctypes.c_void_p(0x10000), None, T, K, E, R, A, limit, ctypes.byref(s), None)
     assert rc == expect
+
+
+@pytest.mark.parametrize("T,K,E,R,A,expect", [
+    (8, 2, 8, 3, 1, 1),          # E % R
+    (9, 2, 8, 2, 1, 1),          # T % R
+    (8, 0, 8, 2, 1, 1),          # K < 1
+    (64, 2, 64, 64, 1, 6),       # R above 32
+    (8, 2, 8, 2, 0, 1),          # A < 1
+])
+def test_rank_layout_host_checks(lib, T, K, E, R, A, expect):
+    s = _handle()
+    p = ctypes.c_void_p(0x10000)
+    assert lib.ep_rank_layout(p, None, T, K, E, R, A, None, None, None, None, None, ctypes.byref(s), None) == expect
+
+
+def test_rank_layout_workspace_and_pointers(lib):
+    p = ctypes.c_void_p(0x10000)
+    ws = lib.ep_rank_workspace_bytes(4096, 8, 256)
+    assert ws % 256 == 0 and ws >= lib.ep_workspace_bytes(4096, 8, 8, 1) + 4096 * 8 * 16 + 256 * 4
+    assert lib.ep_rank_workspace_bytes(-1, 8, 256) == 0
+    s = _handle(ws_bytes=ws - 256)
+    assert lib.ep_rank_layout(p, None, 4096, 8, 256, 8, 1, None, None, None, None, None, ctypes.byref(s), None) == 1
+    s = _handle()
+    s.recv_src_token = 0
+    assert lib.ep_rank_layout(p, None, 8, 2, 8, 2, 1, None, None, None, None, None, ctypes.byref(s), None) == 1
+    s = _handle()
+    s.recv_weight = 0                                   # not used by the per-rank form: accepted up to launch
+    s.recv_local_expert = 0
+    assert lib.ep_rank_layout(p, None, 8, 2, 8, 2, 1, None, None, None, ctypes.c_void_p(0x10004), None,
+                              ctypes.byref(s), None) == 1          # misaligned recv_topk_idx
+    # a per-rank handle takes no combine weights (V1: a plain sum)
+    s = _handle(magic=0x45504C31)
+    s.num_tokens, s.num_topk, s.num_experts, s.num_ranks, s.expert_alignment, s.kind = 8, 2, 2, 2, 1, 1
+    assert lib.ep_combine(ctypes.byref(s), p, 256, p, None, None, p, None) == 1
 
 
 def test_layout_rejects_misaligned_recv_stats(lib):
