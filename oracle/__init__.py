@@ -63,7 +63,7 @@ def _load(path):
     L = ctypes.CDLL(path)
     vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
     L.orc_layout.restype = i32
-    L.orc_layout.argtypes = [vp, vp, i64, i64, i64, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp]
+    L.orc_layout.argtypes = [vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp]
     L.orc_dispatch_rows.restype = None
     L.orc_dispatch_rows.argtypes = [vp, i64, i64, i64, vp, vp, vp, i64, i32, vp]
     L.orc_cast_fp8.restype = None
@@ -114,7 +114,7 @@ def capacity_rows(T, K, E, A):
 
 
 def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment,
-           num_max_tokens_per_rank=0, capacity=None):
+           num_max_tokens_per_rank=0, capacity=None, slab=0):
     """Expand layout of the selected (token, k) pairs ([API] §2.1, [URMA] prefix placement).
 
     Returns a dict with ``cnt`` [E], ``off`` [E+1], ``pair_slot`` [T, K],
@@ -137,7 +137,7 @@ def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment,
     recv_w = np.zeros(max(capacity, 1), np.float32)
     recv_lexp = np.full(max(capacity, 1), -1, np.int32)
     rc = lib().orc_layout(_p(topk_idx), _p(topk_weights), T, K, E, int(num_ranks),
-                          int(expert_alignment), int(num_max_tokens_per_rank), int(capacity),
+                          int(expert_alignment), int(num_max_tokens_per_rank), int(capacity), int(slab),
                           _p(cnt), _p(off), _p(pair_slot), _p(recv_src), _p(recv_w), _p(recv_lexp))
     if rc != OK:
         raise OracleError(rc, "layout")
@@ -145,6 +145,15 @@ def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment,
                 recv_w=recv_w[:capacity], recv_lexp=recv_lexp[:capacity],
                 num_experts=E, num_ranks=int(num_ranks), expert_alignment=int(expert_alignment),
                 capacity=int(capacity))
+
+
+def ll_layout(topk_idx, topk_weights, num_experts, num_ranks, num_max_dispatch_tokens_per_rank):
+    """Low-latency fixed-slab layout ([API] §3.3): expert e owns rows
+    [e * S, (e + 1) * S) with S = R * num_max_dispatch_tokens_per_rank, its pairs
+    first (token-major, k-minor), the rest padding; capacity E * S."""
+    R, M = int(num_ranks), int(num_max_dispatch_tokens_per_rank)
+    S = R * M
+    return layout(topk_idx, topk_weights, num_experts, R, 1, M, capacity=int(num_experts) * S, slab=S)
 
 
 def rank_layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment=1, capacity=None):
@@ -359,16 +368,22 @@ def bf16_to_f32(b):
     return (b.astype(np.uint32) << 16).view(np.float32)
 
 
-def step(inp, cfg):
+def step(inp, cfg, per_rank=False):
     """One pass of the whole path on host arrays: layout, dispatch (with the
     fused cast in FP8 mode) and combine of the given expert outputs.  Used by the
-    benchmark's CPU baseline.  Returns (layout, recv rows, combined out)."""
-    lay = layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"],
-                 cfg.get("max_tokens_per_rank", 0))
+    benchmark's CPU baseline.  ``per_rank``: the per-token-per-rank layout and
+    V1's unweighted combine instead of the expand layout.  Returns (layout,
+    recv rows, combined out)."""
+    if per_rank:
+        lay = rank_layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"])
+    else:
+        lay = layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"],
+                     cfg.get("max_tokens_per_rank", 0))
     if cfg.get("fp8"):
         q, s = cast_fp8(inp["x"])
         recv = (dispatch_rows(q, lay, cfg["zero_pad"]), dispatch_rows(s, lay, cfg["zero_pad"]))
     else:
         recv = dispatch_rows(inp["x"], lay, cfg["zero_pad"])
-    out = combine(inp["y"], lay["pair_slot"], inp["topk_weights"], inp.get("bias0"), inp.get("bias1"))
+    w = None if per_rank else inp["topk_weights"]
+    out = combine(inp["y"], lay["pair_slot"], w, inp.get("bias0"), inp.get("bias1"))
     return lay, recv, out

@@ -173,14 +173,19 @@ static int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
  * Rows of expert e are [off[e], off[e] + cnt[e]) in token-major, k-minor
  * order of the pairs, followed by align(cnt[e], A) - cnt[e] padding rows.
  * Because each rank owns a contiguous run of experts, this is the order
- * (destination rank, local expert, source token). */
+ * (destination rank, local expert, source token).
+ * slab > 0 gives the low-latency form ([API] §3.3 low_latency_dispatch:
+ * num_max_dispatch_tokens_per_rank, a receive buffer of
+ * [E/R, R * max_tokens, H] per rank): every expert owns a fixed slab of
+ * `slab` = R * max_tokens rows, off[e] = e * slab, the rows after its pairs
+ * are padding, and more pairs than the slab holds is ORC_ERR_CAPACITY. */
 int orc_layout(const int64_t* topk_idx, const float* topk_weights,
                int64_t T, int64_t K, int64_t E, int64_t R, int64_t A,
-               int64_t max_tokens_per_rank, int64_t capacity,
+               int64_t max_tokens_per_rank, int64_t capacity, int64_t slab,
                int32_t* cnt, int32_t* off, int32_t* pair_slot,
                int32_t* recv_src, float* recv_w, int32_t* recv_lexp)
 {
-    if (T < 0 || K < 1 || E < 1 || R < 1 || A < 1 || E % R != 0 || T % R != 0)
+    if (T < 0 || K < 1 || E < 1 || R < 1 || A < 1 || E % R != 0 || T % R != 0 || slab < 0)
         return ORC_ERR_INVALID_ARG;
     if (max_tokens_per_rank > 0 && T / R > max_tokens_per_rank)
         return ORC_ERR_CAPACITY;
@@ -197,10 +202,18 @@ int orc_layout(const int64_t* topk_idx, const float* topk_weights,
         if (topk_idx[i] >= 0)
             cnt[topk_idx[i]] += 1;
 
-    /* 3. exclusive prefix sum of the aligned counts */
+    /* 3. exclusive prefix sum of the aligned counts; with a fixed slab of
+     *    `slab` rows per expert (the low-latency layout) off[e] = e * slab */
     off[0] = 0;
-    for (int64_t e = 0; e < E; e++)
-        off[e + 1] = (int32_t)(off[e] + align_up(cnt[e], A));
+    for (int64_t e = 0; e < E; e++) {
+        if (slab > 0) {
+            if (cnt[e] > slab)
+                return ORC_ERR_CAPACITY;
+            off[e + 1] = (int32_t)((e + 1) * slab);
+        } else {
+            off[e + 1] = (int32_t)(off[e] + align_up(cnt[e], A));
+        }
+    }
     if (off[E] > capacity)
         return ORC_ERR_CAPACITY;
 

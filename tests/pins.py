@@ -682,6 +682,50 @@ def pin_rank_combine_identity():
     assert np.array_equal(out[has], expect[has]) and np.all(out[~has] == 0)
 
 
+def pin_ll_layout_golden():
+    g = _golden("ll_layout_example.json")
+    lay = oracle.ll_layout(np.array(g["topk_idx"], np.int64), None, g["E"], g["R"], g["max_tokens"])
+    assert lay["cnt"].tolist() == g["cnt"] and lay["off"].tolist() == g["off"]
+    assert lay["pair_slot"].tolist() == g["pair_slot"] and lay["recv_src"].tolist() == g["recv_src"]
+    # more pairs for one expert than its slab holds: a capacity error
+    try:
+        oracle.ll_layout(np.zeros((2, 2), np.int64), None, 2, 1, 2)     # 4 pairs, slab of 2
+    except oracle.OracleError as err:
+        assert err.code == 2
+    else:
+        raise AssertionError("slab overflow not reported")
+
+
+def pin_ll_layout_vs_expand(n=80, seed=43):
+    """The fixed-slab form is the A = 1 expand layout with every expert moved to
+    e * S: same counts, same order within an expert, padding to the slab end."""
+    rng = np.random.default_rng(seed)
+    for i in range(n):
+        R = int(rng.choice([1, 2, 4]))
+        E = R * int(rng.integers(1, 5))
+        T = R * int(rng.integers(0, 6))
+        K = int(rng.integers(1, 4))
+        M = max(T // R, 1) + int(rng.integers(0, 3))
+        idx = rng.integers(-1, E, (T, K)).astype(np.int64)
+        w = rng.random((T, K)).astype(np.float32)
+        S = R * M
+        ex = oracle.layout(idx, w, E, R, 1)
+        try:
+            ll = oracle.ll_layout(idx, w, E, R, M)
+        except oracle.OracleError as err:
+            assert err.code == 2 and (ex["cnt"] > S).any()        # an expert overflows its slab
+            continue
+        assert np.array_equal(ll["cnt"], ex["cnt"])
+        assert np.array_equal(ll["off"], np.arange(E + 1) * S)
+        e_of = np.where(idx >= 0, idx, 0)
+        sel = idx >= 0
+        assert np.array_equal((ll["pair_slot"] - ll["off"][e_of])[sel], (ex["pair_slot"] - ex["off"][e_of])[sel])
+        assert np.all(ll["pair_slot"][~sel] == -1)
+        for e in range(E):
+            pad = ll["recv_src"][e * S + ll["cnt"][e]:(e + 1) * S]
+            assert np.all(pad == -1)
+
+
 ALL_PINS = [
     pin_layout_exhaustive, pin_layout_random, pin_layout_invariants_workloads, pin_layout_errors,
     pin_routing_table_golden, pin_dispatch_rows, pin_e4m3_decode_table, pin_e4m3_encode_vs_torch,
@@ -691,4 +735,5 @@ ALL_PINS = [
     pin_cast_variants_vs_torch, pin_round_scale_properties, pin_fp8_variants_golden, pin_ue8m0,
     pin_cast_variants_roundtrip, pin_scales_col_major,
     pin_rank_layout_vs_numpy, pin_rank_layout_golden, pin_rank_layout_matches_expand, pin_rank_combine_identity,
+    pin_ll_layout_golden, pin_ll_layout_vs_expand,
 ]

@@ -29,3 +29,12 @@ def test_routing_table_worked_examples():
 
 def test_dispatch_rows_vs_fancy_indexing():
     pins.pin_dispatch_rows()
+
+
+def test_ll_layout_hand_derived():
+    """§3.3 low-latency fixed-slab layout: a hand-derived example."""
+    pins.pin_ll_layout_golden()
+
+
+def test_ll_layout_is_the_expand_layout_moved_to_slabs():
+    pins.pin_ll_layout_vs_expand()

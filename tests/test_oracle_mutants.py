@@ -48,6 +48,7 @@ MUTANTS = {
                        "if (e >= 0 && e % R == r)\n                    in = 1;"),
     "rank_list_unaligned": ("num_recv_per_expert[e] = (int32_t)align_up(num_tokens_per_expert[e], A);",
                             "num_recv_per_expert[e] = num_tokens_per_expert[e];"),
+    "ll_slab_off_by_one": ("off[e + 1] = (int32_t)((e + 1) * slab);", "off[e + 1] = (int32_t)(e * slab);"),
     "bf16_truncates": ("if (dropped > 0x8000u || (dropped == 0x8000u && (upper & 1u)))", "if (0)"),
     "bf16_ties_away": ("if (dropped > 0x8000u || (dropped == 0x8000u && (upper & 1u)))",
                        "if (dropped >= 0x8000u)"),
