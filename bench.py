@@ -50,9 +50,10 @@ def parse():
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--fused", action="store_true",
                    help="the single ep_layout_dispatch call instead of ep_layout + ep_dispatch")
-    p.add_argument("--layout", default="expand", choices=["expand", "rank"],
+    p.add_argument("--layout", default="expand", choices=["expand", "rank", "ll"],
                    help="expand: one receive row per (token, k) pair (ep_layout); rank: one per (token, rank) "
-                        "reached (ep_rank_layout) with V1's unweighted combine")
+                        "reached (ep_rank_layout) with V1's unweighted combine; ll: the low-latency fixed "
+                        "slab of R * max_tokens rows per expert (ep_ll_layout)")
     return p.parse_args()
 
 
@@ -160,10 +161,10 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # algorithmic bytes (the minimum each step must move)
 # --------------------------------------------------------------------------
-def algorithmic_bytes(cfg, cnt, A):
+def algorithmic_bytes(cfg, cnt, A, slab=0):
     T, H, K, E = cfg["T"], cfg["H"], cfg["K"], cfg["E"]
     N = int(cnt.sum())
-    Np = int(((cnt + A - 1) // A * A).sum())
+    Np = E * slab if slab else int(((cnt + A - 1) // A * A).sum())
     pad = (Np - N) if cfg["zero_pad"] else 0
     nb = H // 128
     out_row = (H + 4 * nb) if cfg["fp8"] else 2 * H
@@ -209,10 +210,14 @@ def run_ours(args, rank, world, local_rank):
     w = torch.from_numpy(inp["topk_weights"]).to(dev)
     x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
     per_rank = args.layout == "rank"
-    if per_rank and args.fused:
+    slab = args.layout == "ll"
+    M = cfg["max_tokens_per_rank"] or T // R
+    if args.layout != "expand" and args.fused:
         raise SystemExit("--fused applies to the expand layout only")
     if per_rank:
         lay = ep.RankLayout(T, K, E, R, A, dev)
+    elif slab:
+        lay = ep.ll_layout(idx, w, E, R, M)
     else:
         lay = ep.Layout(T, K, E, R, A, dev, num_max_tokens_per_rank=cfg["max_tokens_per_rank"])
     cw = None if per_rank else w            # V1's combine is a plain sum over the ranks
@@ -233,6 +238,8 @@ def run_ours(args, rank, world, local_rank):
     def do_layout(d_idx, d_w):
         if per_rank:
             ep.rank_layout(d_idx, d_w, E, R, A, out=lay)
+        elif slab:
+            ep.ll_layout(d_idx, d_w, E, R, M, out=lay)
         else:
             ep.layout(d_idx, d_w, E, R, A, cfg["max_tokens_per_rank"], out=lay)
 
@@ -246,6 +253,8 @@ def run_ours(args, rank, world, local_rank):
         y = recv.clone()
     if per_rank:
         nbytes = algorithmic_bytes_rank(cfg, lay.num_recv_rows(), int((idx >= 0).sum()))
+    elif slab:
+        nbytes = algorithmic_bytes(cfg, lay.num_recv_tokens_per_expert.cpu().numpy(), 1, slab=R * M)
     else:
         nbytes = algorithmic_bytes(cfg, lay.num_recv_tokens_per_expert.cpu().numpy(), A)
 
@@ -349,7 +358,8 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
         "config": {"workload": "%s: T=%d H=%d E=%d top-%d R=%d align=%d zero_pad=%s%s%s" % (
             cfg["name"], T, H, E, K, R, A, cfg["zero_pad"], " fp8-cast" if fp8 else "",
-            " layout=per-rank (one row per token and rank reached, unweighted combine)" if per_rank else ""),
+            " layout=per-rank (one row per token and rank reached, unweighted combine)" if per_rank else
+            (" layout=ll (fixed slab of R*%d rows per expert)" % M) if slab else ""),
             "global_batch": T * world, "parallelism": "replicas x%d (R=%d virtual ranks per GPU)" % (world, R),
             "l2": "flushed by a 256 MiB write before every step, outside the timed events",
             "pairs": nbytes["N"], "recv_rows": nbytes["Np"], "pad_rows": nbytes["pad_rows"],
@@ -364,9 +374,10 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "kernel": top_kernel,
                      "achieved": round(disp_gbs, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(disp_gbs / peak, 4),
-                     "traffic": ncu_traffic(top_kernel, cfg["name"] + ("/per-rank" if per_rank else "")),
+                     "traffic": ncu_traffic(top_kernel, cfg["name"] + ("" if args.layout == "expand"
+                                                                       else "/" + args.layout)),
                      "algorithmic_bytes_per_launch": top_bytes},
-        "gpu_launches": args.steps * (5 if per_rank else (2 if (args.fused and not fp8) else 3)),
+        "gpu_launches": args.steps * (4 if per_rank else (2 if (args.fused and not fp8) else 3)),
         "wall_s_timed_region": round(wall, 4),
     }
     if clock_info:
@@ -376,7 +387,7 @@ def run_ours(args, rank, world, local_rank):
                        "ms_per_step": round(e2e["ms_per_step"], 4),
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, inp, per_rank)
+        line["cpu_baseline"] = cpu_baseline(cfg, inp, args.layout)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -434,32 +445,28 @@ def run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush, do
 # --------------------------------------------------------------------------
 # CPU oracle: the baseline leg and the reference arm
 # --------------------------------------------------------------------------
-def oracle_step_inputs(cfg, inp, per_rank=False):
+def oracle_step_inputs(cfg, inp, form="expand"):
     import oracle
-    if per_rank:
-        lay = oracle.rank_layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"])
-    else:
-        lay = oracle.layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"],
-                            cfg["max_tokens_per_rank"])
+    lay = oracle.step_layout(inp, cfg, form)
     y = oracle.dispatch_rows(inp["x"], lay, cfg["zero_pad"]) if not cfg["fp8"] else \
         workload.expert_outputs(cfg, int(lay["off"][-1]))
     return dict(inp, y=y)
 
 
-def time_oracle(cfg, inp, budget_s=10.0, min_steps=1, max_steps=None, per_rank=False):
+def time_oracle(cfg, inp, budget_s=10.0, min_steps=1, max_steps=None, form="expand"):
     import oracle
-    full = oracle_step_inputs(cfg, inp, per_rank)
+    full = oracle_step_inputs(cfg, inp, form)
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle.step(full, cfg, per_rank)
+        oracle.step(full, cfg, form)
         n += 1
         el = time.perf_counter() - t0
         if (n >= min_steps and el >= budget_s) or (max_steps and n >= max_steps):
             return n, el
 
 
-def cpu_baseline(cfg, inp, per_rank=False):
-    n, el = time_oracle(cfg, inp, budget_s=10.0, per_rank=per_rank)
+def cpu_baseline(cfg, inp, form="expand"):
+    n, el = time_oracle(cfg, inp, budget_s=10.0, form=form)
     return {"value": round(cfg["T"] * n / el, 1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": "%d full step(s) of the %s workload (layout, dispatch%s, combine), single-threaded C, "
                       "%d host cores present" % (n, cfg["name"], " with cast" if cfg["fp8"] else "",
@@ -471,15 +478,15 @@ def run_reference(args, rank, world):
         return None
     cfg = workload.config(args.workload)
     inp = workload.inputs(cfg)
-    per_rank = args.layout == "rank"
-    full = oracle_step_inputs(cfg, inp, per_rank)
+    form = args.layout
+    full = oracle_step_inputs(cfg, inp, form)
     import oracle
     for _ in range(args.warmup):
-        oracle.step(full, cfg, per_rank)
+        oracle.step(full, cfg, form)
     ts = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.step(full, cfg, per_rank)
+        oracle.step(full, cfg, form)
         ts.append(time.perf_counter() - t0)
     ms = float(np.mean(ts)) * 1e3
     v = round(cfg["T"] / (ms * 1e-3), 1)
@@ -487,7 +494,8 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp8-e4m3/bf16" if cfg["fp8"] else "bf16",
             "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
-            "config": {"workload": cfg["name"] + (" layout=per-rank" if per_rank else ""), "global_batch": cfg["T"]},
+            "config": {"workload": cfg["name"] + ("" if form == "expand" else " layout=" + form),
+                       "global_batch": cfg["T"]},
             "impl": "reference",
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": "the full %s workload per step (single-threaded C oracle)" % cfg["name"]},

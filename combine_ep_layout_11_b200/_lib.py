@@ -44,6 +44,8 @@ SIGNATURES = {
     "ep_layout_no_alloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp]),
     "ep_scale_bytes": (_i64, [_i64, _i, _i]),
     "ep_rank_workspace_bytes": (_sz, [_i, _i, _i]),
+    "ep_ll_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "ep_ll_layout": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _LP, _vp]),
     "ep_rank_layout": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _LP, _vp]),
     "ep_dispatch": (_i, [_LP, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "ep_layout_dispatch": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _LP, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp,

@@ -88,7 +88,7 @@ class Layout:
     """
 
     def __init__(self, num_tokens, num_topk, num_experts, num_ranks, expert_alignment, device,
-                 capacity=None, num_max_tokens_per_rank=0):
+                 capacity=None, num_max_tokens_per_rank=0, workspace_nbytes=None):
         T, K, E, A = num_tokens, num_topk, num_experts, expert_alignment
         if capacity is None:
             capacity = capacity_rows(T, K, E, A)
@@ -108,7 +108,7 @@ class Layout:
         self.recv_src_token = torch.empty(n, **i32)
         self.recv_weight = torch.empty(n, dtype=torch.float32, device=dev)
         self.recv_local_expert = torch.empty(n, **i32)
-        nbytes = workspace_bytes(T, K, E, A)
+        nbytes = workspace_bytes(T, K, E, A) if workspace_nbytes is None else int(workspace_nbytes)
         if nbytes == 0:
             raise EpError(EP_ERR_INVALID_ARG, "workspace size")
         self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)   # zeroed before first use
@@ -170,6 +170,33 @@ def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment=1,
                        expert_alignment, num_max_tokens_per_rank, lay.ref(), _stream(topk_idx.device)),
            "ep_layout")
     return lay
+
+
+def ll_layout(topk_idx, topk_weights, num_experts, num_ranks, num_max_dispatch_tokens_per_rank, out=None,
+              cumulative_local_expert_recv_stats=None):
+    """Low-latency fixed-slab layout (§3.3): expert e owns receive rows
+    [e*S, (e+1)*S) with S = num_ranks * num_max_dispatch_tokens_per_rank, its
+    pairs first (token-major, k-minor), the rest padding.  Returns a ``Layout``
+    (capacity E*S) usable by ``dispatch`` and ``combine``."""
+    L = _lib.load()
+    assert topk_idx.dtype == torch.int64 and topk_idx.dim() == 2 and topk_idx.is_contiguous()
+    T, K = topk_idx.shape
+    E, R, M = num_experts, num_ranks, num_max_dispatch_tokens_per_rank
+    if topk_weights is not None:
+        assert topk_weights.dtype == torch.float32 and topk_weights.shape == (T, K)
+        assert topk_weights.is_contiguous()
+    if out is None:
+        nbytes = int(L.ep_ll_workspace_bytes(T, K, E, R, M))
+        if nbytes == 0:
+            raise EpError(EP_ERR_INVALID_ARG, "workspace size")
+        out = Layout(T, K, E, R, 1, topk_idx.device, capacity=E * R * M, num_max_tokens_per_rank=M,
+                     workspace_nbytes=nbytes)
+    else:
+        assert (out.num_tokens, out.num_topk, out.num_experts) == (T, K, E), "layout size mismatch"
+    _set_recv_stats(out, cumulative_local_expert_recv_stats)
+    _check(L.ep_ll_layout(_ptr(topk_idx), _ptr(topk_weights), T, K, E, R, M, out.ref(), _stream(topk_idx.device)),
+           "ep_ll_layout")
+    return out
 
 
 class RankLayout:

@@ -77,6 +77,11 @@ int prepare_layout(const int64_t* topk_idx, const float* topk_weights, int T, in
     a->padpre = reinterpret_cast<int32_t*>(wsb + ws.padpre_off);
     a->pad_rows = reinterpret_cast<int32_t*>(wsb + ws.padrows_off);
     a->stats = layout->cumulative_local_expert_recv_stats;
+    a->slab = 0;
+    a->src_idx = nullptr;
+    a->src_K = 0;
+    a->src_E = 0;
+    a->in_rank = nullptr;
     return EP_OK;
 }
 
@@ -220,19 +225,8 @@ int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_t
             return EP_ERR_CUDA;
         return EP_OK;
     }
-    int64_t* rank_idx = reinterpret_cast<int64_t*>(wsb + ws.rank_idx_off);
-    int32_t* counts = reinterpret_cast<int32_t*>(wsb + ws.counts_off);
-
-    ep::RankPrepArgs p;
-    p.topk_idx = topk_idx;
-    p.T = T; p.K = K; p.E = E; p.R = R;
-    p.rank_idx = rank_idx;
-    p.in_rank = is_token_in_rank;
-    p.counts = counts;
-    p.hdr = header(layout);
-
     ep::LayoutArgs la;
-    la.topk_idx = rank_idx;
+    la.topk_idx = nullptr;   // keys come from src_idx
     la.topk_weights = nullptr;
     la.T = T; la.K = R; la.E = R; la.R = R; la.A = 1;
     la.C = 0;
@@ -249,15 +243,20 @@ int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_t
     la.padpre = reinterpret_cast<int32_t*>(wsb + ws.expand.padpre_off);
     la.pad_rows = reinterpret_cast<int32_t*>(wsb + ws.expand.padrows_off);
     la.stats = nullptr;
+    la.slab = 0;
+    la.src_idx = topk_idx;
+    la.src_K = K;
+    la.src_E = E;
+    la.in_rank = is_token_in_rank;
 
     ep::RankPostArgs post;
     post.topk_idx = topk_idx;
     post.topk_weights = topk_weights;
-    post.rank_off = layout->expert_offset;
-    post.recv_src = layout->recv_src_token;
-    post.counts = counts;
+    post.token_slot = layout->pair_slot;
     post.T = T; post.K = K; post.E = E; post.R = R; post.A = A;
     post.capacity = layout->capacity;
+    post.counts = reinterpret_cast<int32_t*>(wsb + ws.counts_off);
+    post.done = reinterpret_cast<uint32_t*>(wsb + ws.done_off);
     post.recv_topk_idx = recv_topk_idx;
     post.recv_topk_w = recv_topk_weights;
     post.num_tokens_per_expert = num_tokens_per_expert;
@@ -266,7 +265,41 @@ int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_t
     int sms = 0;
     int rc = device_sms(&sms);
     if (rc != EP_OK) return rc;
-    return ep::launch_rank_layout(p, la, post, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    return ep::launch_rank_layout(la, post, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+size_t ep_ll_workspace_bytes(int num_tokens, int num_topk, int num_experts, int num_ranks,
+                             int num_max_dispatch_tokens_per_rank) {
+    if (num_tokens < 0 || num_topk < 1 || num_experts < 1 || num_ranks < 1 || num_max_dispatch_tokens_per_rank < 1)
+        return 0;
+    const int64_t slab = (int64_t)num_ranks * num_max_dispatch_tokens_per_rank;
+    if (slab > INT_MAX - 1) return 0;
+    // the padding-row list holds up to E * slab rows: the expand sizing with A = slab + 1
+    return ep::ws_layout(num_tokens, num_topk, num_experts, (int)(slab + 1)).total;
+}
+
+int ep_ll_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
+                 int num_experts, int num_ranks, int num_max_dispatch_tokens_per_rank, ep_layout_t* layout,
+                 void* stream) {
+    const int M = num_max_dispatch_tokens_per_rank;
+    if (!layout || M < 1 || num_ranks < 1 || num_experts < 1) return EP_ERR_INVALID_ARG;
+    const int64_t slab = (int64_t)num_ranks * M;
+    if (slab * num_experts > INT_MAX) return EP_ERR_UNSUPPORTED;
+    if (layout->workspace_bytes <
+        ep_ll_workspace_bytes(num_tokens, num_topk, num_experts, num_ranks, M))
+        return EP_ERR_INVALID_ARG;
+    ep_layout_t tmp = *layout;   // the handle changes only once every check has passed
+    ep::LayoutArgs a;
+    int rc = prepare_layout(topk_idx, topk_weights, num_tokens, num_topk, num_experts, num_ranks, 1, M, &tmp, &a);
+    if (rc != EP_OK) return rc;
+    a.slab = (int)slab;
+    tmp.kind = EP_LAYOUT_LL_SLAB;
+    *layout = tmp;
+    cudaStream_t s = (cudaStream_t)stream;
+    // with no tokens the kernel still runs (one CTA): every slab row is padding
+    int sms = 0;
+    if ((rc = device_sms(&sms)) != EP_OK) return rc;
+    return ep::launch_layout(a, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
 int64_t ep_scale_bytes(int64_t rows, int hidden, int scale_format) {
@@ -285,7 +318,8 @@ int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const flo
     int rc = prepare_dispatch(layout, x, x_dtype, x_scales, hidden, cast_to_fp8, scale_format, do_zero_padding,
                               recv_x, recv_scales, &a, &elem_bytes);
     if (rc != EP_OK) return rc;
-    if (layout->num_tokens == 0) return EP_OK;   // no tokens, no pairs, no padding rows
+    // no tokens: no pairs, and no padding rows except in the fixed-slab form
+    if (layout->num_tokens == 0 && layout->kind != EP_LAYOUT_LL_SLAB) return EP_OK;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t err = cast_to_fp8 ? ep::launch_dispatch_cast(a, s) : ep::launch_dispatch_copy(a, elem_bytes, s);
     return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;

@@ -75,7 +75,8 @@ inline WsLayout ws_layout(int T, int K, int E, int A) {
     (void)K;
     WsLayout w;
     w.table_off = 256;
-    w.padpre_off = round_up(w.table_off + (T > 0 ? (size_t)kMaxChunks * round4(E) * 4 : 0), 256);
+    (void)T;
+    w.padpre_off = round_up(w.table_off + (size_t)kMaxChunks * round4(E) * 4, 256);
     w.padrows_off = round_up(w.padpre_off + ((size_t)E + 1) * 4, 256);
     w.total = round_up(w.padrows_off + (size_t)E * (size_t)(A > 1 ? A - 1 : 0) * 4 + 4, 256);
     return w;

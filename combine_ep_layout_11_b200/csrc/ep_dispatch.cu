@@ -202,6 +202,19 @@ __device__ __forceinline__ void copy_scale(uint8_t* sf, int64_t off, const uint8
         sf[off] = src[g];
 }
 
+// A row-major scale row that is not a multiple of 16 bytes (so not a TMA
+// store) goes out in the widest word dividing its length: 8, 4, 2 or 1 bytes.
+__device__ __forceinline__ void copy_word(uint8_t* dst, const uint8_t* src, int w) {
+    if (w == 8)
+        *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+    else if (w == 4)
+        *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(src);
+    else if (w == 2)
+        *reinterpret_cast<uint16_t*>(dst) = *reinterpret_cast<const uint16_t*>(src);
+    else
+        *dst = *src;
+}
+
 template <bool kPerRow, bool kPow2>
 __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArgs a, int stages) {
     constexpr int kWarps = kCastThreads / 32;
@@ -219,6 +232,8 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
     uint8_t* sf = reinterpret_cast<uint8_t*>(a.recv_scales);
     const uint32_t sf_row_bytes = (uint32_t)ng * (uint32_t)elem;
     const bool bulk_scales = !a.sf_col_major && (sf_row_bytes % 16u) == 0;
+    const int sf_word = sf_row_bytes % 8u == 0 ? 8 : sf_row_bytes % 4u == 0 ? 4 : sf_row_bytes % 2u == 0 ? 2 : 1;
+    const int sf_words = (int)sf_row_bytes / sf_word;
 
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
@@ -296,11 +311,18 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
                     if (bulk_scales) bulk_store(sf + (int64_t)slot * sf_row_bytes, dst_sf, sf_row_bytes);
                 }
             }
-            if (!bulk_scales) {
+            if (a.sf_col_major) {
                 for (int k = 0; k < K; ++k) {
                     const int32_t slot = slots[s * 32 + k];
                     if (slot < 0 || (int64_t)slot >= a.capacity) continue;
                     for (int g = lane; g < ng; g += 32) copy_scale(sf, sf_offset(a, slot, g), dst_sf, g, elem);
+                }
+            } else if (!bulk_scales) {
+                for (int q = lane; q < K * sf_words; q += 32) {
+                    const int k = q / sf_words, wd = q - k * sf_words;
+                    const int32_t slot = slots[s * 32 + k];
+                    if (slot < 0 || (int64_t)slot >= a.capacity) continue;
+                    copy_word(sf + (int64_t)slot * sf_row_bytes + wd * sf_word, dst_sf + wd * sf_word, sf_word);
                 }
             }
             bulk_commit();
@@ -326,8 +348,11 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
             bulk_store(a.recv + (int64_t)row * H, zero, (uint32_t)H);
             if (bulk_scales)
                 bulk_store(sf + (int64_t)row * sf_row_bytes, zero + H, sf_row_bytes);
-            else
+            else if (a.sf_col_major)
                 for (int g = 0; g < ng; ++g) copy_scale(sf, sf_offset(a, row, g), zero + H, g, elem);
+            else
+                for (int wd = 0; wd < sf_words; ++wd)
+                    copy_word(sf + (int64_t)row * sf_row_bytes + wd * sf_word, zero + H + wd * sf_word, sf_word);
         }
         bulk_commit();
         bulk_wait_all<0>();

@@ -25,6 +25,16 @@ struct LayoutArgs {
     int32_t* padpre;
     int32_t* pad_rows;
     int32_t* stats;             // [E] running receive counts, nullable
+    // Low-latency form: > 0 gives every expert a fixed slab of `slab` rows
+    // (off[e] = e * slab, the rest of the slab is padding); 0: aligned counts.
+    int slab;
+    // Per-rank keys (ep_rank_layout): nullptr for the expand layout.  Otherwise
+    // pair i = (t, r) of a [T, R] table (K = E = R here), whose key is r when
+    // token t has an expert on rank r, read from src_idx [T, src_K] with src_E
+    // experts; in_rank [T*R] (nullable) gets 1 / 0 per pair.
+    const int64_t* src_idx;
+    int src_K, src_E;
+    uint8_t* in_rank;
 };
 
 // One cooperative kernel: per-chunk counts, a grid barrier, the scans and the
@@ -86,45 +96,35 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_selftest_wait(WsHeader* hdr, uint64_t timeout_ns, cudaStream_t s);
 
 // Per-token-per-rank layout (ep_rank_layout.cu).  Workspace: the expand-layout
-// workspace of the derived [T, R] table (E' = K' = R, A = 1), then the table
-// itself (int64 [T*R]), scratch targets for the layout kernel's per-row
-// weight and local-expert writes (meaningless here), and the per-expert
-// pair counts (int32 [E]).
+// workspace of the [T, R] (token, rank) table (E' = K' = R, A = 1), scratch
+// targets for the layout kernel's per-row weight and local-expert writes
+// (meaningless here), the per-expert pair counts (int32 [E]) and a counter of
+// finished CTAs; both are zero between calls.
 struct RankWsLayout {
     WsLayout expand;
-    size_t rank_idx_off;
     size_t scratch_w_off;
     size_t scratch_lexp_off;
     size_t counts_off;
+    size_t done_off;
     size_t total;
 };
 RankWsLayout rank_ws_layout(int T, int R, int E);
 
-struct RankPrepArgs {
-    const int64_t* topk_idx;   // [T*K]
-    int T, K, E, R;
-    int64_t* rank_idx;         // [T*R] derived table (workspace)
-    uint8_t* in_rank;          // [T*R] is_token_in_rank, nullable
-    int32_t* counts;           // [E] pair counts (workspace)
-    WsHeader* hdr;
-};
-
 struct RankPostArgs {
     const int64_t* topk_idx;   // [T*K]
     const float* topk_weights; // [T*K] or nullptr
-    const int32_t* rank_off;   // [R+1]
-    const int32_t* recv_src;   // [capacity]
-    const int32_t* counts;     // [E]
+    const int32_t* token_slot; // [T*R]
     int T, K, E, R, A;
     int64_t capacity;
+    int32_t* counts;           // [E] workspace, zero on entry and on exit
+    uint32_t* done;            // workspace counter, zero on entry and on exit
     int64_t* recv_topk_idx;    // [capacity][K], nullable
     float* recv_topk_w;        // [capacity][K], nullable
     int32_t* num_tokens_per_expert;   // [E], nullable
     int32_t* num_recv_per_expert;     // [E] aligned, nullable
 };
 
-// memset of the counts, prep kernel, layout kernel on the derived table, post kernel.
-cudaError_t launch_rank_layout(const RankPrepArgs& p, LayoutArgs la, const RankPostArgs& post, int sms,
-                               cudaStream_t s);
+// The layout kernel with per-rank keys, then the post kernel.
+cudaError_t launch_rank_layout(LayoutArgs la, const RankPostArgs& post, int sms, cudaStream_t s);
 
 }  // namespace ep

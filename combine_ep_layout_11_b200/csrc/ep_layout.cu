@@ -32,36 +32,43 @@ namespace {
 // most 64 table rows (one batch of 16-byte loads per thread).
 constexpr int kLayoutChunks = 64;
 
-template <int NT>
+template <int NT, bool kRankKeys>
 __global__ void __launch_bounds__(NT) layout_kernel(LayoutArgs a) {
     extern __shared__ __align__(16) int32_t sm[];
     pdl_wait();
     pdl_launch_dependents();
-    layout_dev::layout_body<NT>(a, sm);
+    layout_dev::layout_body<NT, kRankKeys>(a, sm);
 }
 
-template <int NT>
+template <int NT, bool kRankKeys>
 cudaError_t launch_layout_nt(LayoutArgs a, int sms, cudaStream_t s) {
+    auto kernel = layout_kernel<NT, kRankKeys>;
     const size_t smem = layout_dev::layout_smem_ints(a.E) * sizeof(int32_t);
-    cudaError_t err = cudaFuncSetAttribute(layout_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_kernel<NT>, NT, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, NT, smem);
     if (err != cudaSuccess) return err;
     int max_chunks = sms * (per_sm > 0 ? per_sm : 1);
     if (max_chunks > kLayoutChunks) max_chunks = kLayoutChunks;
-    const Chunking ch = chunking(a.T, a.K, max_chunks, NT);
+    Chunking ch = chunking(a.T, a.K, max_chunks, NT);
+    if (ch.num_chunks == 0) {   // no tokens (the fixed-slab form still has its padding rows to list)
+        ch.num_chunks = 1;
+        ch.chunk_tokens = 0;
+    }
     a.C = ch.num_chunks;
     a.CT = ch.chunk_tokens;
-    return launch_pdl(layout_kernel<NT>, dim3(a.C), dim3(NT), smem, s, true, a);
+    return launch_pdl(kernel, dim3(a.C), dim3(NT), smem, s, true, a);
 }
 
 }  // namespace
 
 cudaError_t launch_layout(LayoutArgs a, int sms, cudaStream_t s) {
-    return layout_dev::layout_threads(a.E) == layout_dev::kWideThreads
-               ? launch_layout_nt<layout_dev::kWideThreads>(a, sms, s)
-               : launch_layout_nt<layout_dev::kNarrowThreads>(a, sms, s);
+    const bool wide = layout_dev::layout_threads(a.E) == layout_dev::kWideThreads;
+    if (a.src_idx != nullptr)   // per-rank keys: E = R <= 32, always the wide CTA
+        return launch_layout_nt<layout_dev::kWideThreads, true>(a, sms, s);
+    return wide ? launch_layout_nt<layout_dev::kWideThreads, false>(a, sms, s)
+                : launch_layout_nt<layout_dev::kNarrowThreads, false>(a, sms, s);
 }
 
 }  // namespace ep

@@ -45,6 +45,42 @@ __device__ __forceinline__ int align_up_i(int x, int a) { return (x + a - 1) / a
 
 __device__ __forceinline__ int valid_expert(int64_t e, int E) { return (e >= 0 && e < E) ? (int)e : -1; }
 
+// Key of pair i: its expert id (-1 if unselected), or with per-rank keys
+// (kRankKeys; pairs are (t, r) of a [T, R] table with R = a.K) the rank r when
+// token t has one of its experts there, else -1.  `bad` collects ids outside
+// [-1, E).  The token's ids are loaded eight at a time, all eight before any
+// is used, so a key costs one memory round trip per eight experts.
+template <bool kRankKeys>
+__device__ __forceinline__ int pair_key(const LayoutArgs& a, int64_t i, bool& bad) {
+    if (!kRankKeys) {
+        const int64_t e = a.topk_idx[i];
+        const int key = valid_expert(e, a.E);
+        bad |= (key < 0 && e != -1);
+        return key;
+    }
+    const int R = a.K;
+    const int64_t t = i / R;
+    const int r = (int)(i - t * R);
+    const int El = a.src_E / R;
+    const int64_t* row = a.src_idx + t * a.src_K;
+    int key = -1;
+    for (int k0 = 0; k0 < a.src_K; k0 += 8) {
+        int64_t ev[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ev[j] = k0 + j < a.src_K ? row[k0 + j] : -1;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int64_t e = ev[j];
+            if (e >= 0 && e < a.src_E) {
+                if (e / El == r) key = r;
+            } else if (e != -1) {
+                bad = true;
+            }
+        }
+    }
+    return key;
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -145,7 +181,7 @@ __device__ __forceinline__ bool grid_barrier(WsHeader* hdr, uint32_t n, uint32_t
 //           running offset, plus the chunk base: the stable token-major,
 //           k-minor order, equal to the sequential definition bit for bit;
 //   pads    receive-row metadata of the padding rows of experts c, c + C, ...
-template <int NT>
+template <int NT, bool kRankKeys = false>
 __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     constexpr int kW = NT / 32;
     __shared__ long long s_scratch[kW];
@@ -155,9 +191,11 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     LayoutSmem L(sm, E);
     int32_t* my = L.wh + (size_t)w * Ep;
 
+    __shared__ int s_over;
     if (tid == 0) {
         s_gen0 = ld_relaxed_u32(&a.hdr->bar_gen);   // read before arriving at the barrier
         if (c == 0) a.hdr->status = 0;
+        s_over = 0;
     }
     for (int e = lane; e < Ep; e += 32) my[e] = 0;
     __syncwarp();
@@ -168,13 +206,7 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     const int64_t per = ((p1 - p0 + kW - 1) / kW + 31) / 32 * 32;
     const int64_t q0 = min(p0 + w * per, p1), q1 = min(q0 + per, p1);
     bool bad = false;
-    auto load_key = [&](int64_t i) -> int {
-        if (i >= q1) return -1;
-        const int64_t e = a.topk_idx[i];
-        const int key = valid_expert(e, E);
-        bad |= (key < 0 && e != -1);
-        return key;
-    };
+    auto load_key = [&](int64_t i) -> int { return i < q1 ? pair_key<kRankKeys>(a, i, bad) : -1; };
     auto count_round = [&](int key) {
         const uint32_t peers = __match_any_sync(0xffffffffu, key);
         if (key >= 0 && lane == __ffs(peers) - 1) my[key] += __popc(peers);
@@ -258,18 +290,21 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     const int ipt = (E + NT - 1) / NT;
     const int e0 = min(tid * ipt, E), e1 = min(e0 + ipt, E);
     long long loc = 0;
+    // rows of expert e: its count aligned up to A, or the fixed slab; padding
+    // rows: the rest (none when an expert overflows its slab)
+    auto rows_of = [&](int e) { return a.slab > 0 ? a.slab : align_up_i(L.cnt[e], a.A); };
     for (int e = e0; e < e1; ++e) {
-        const int al = align_up_i(L.cnt[e], a.A);
-        loc += ((long long)al << 32) + (al - L.cnt[e]);
+        const int al = rows_of(e);
+        loc += ((long long)al << 32) + max(al - L.cnt[e], 0);
     }
     long long total = 0;
     long long prefix = block_exclusive_scan64<NT>(loc, s_scratch, &total);
     for (int e = e0; e < e1; ++e) {
-        const int al = align_up_i(L.cnt[e], a.A);
+        const int al = rows_of(e);
         L.off[e] = (int)(prefix >> 32);
         L.padpre[e] = (int)(prefix & 0xffffffffll);
         L.base[e] += (int)(prefix >> 32);
-        prefix += ((long long)al << 32) + (al - L.cnt[e]);
+        prefix += ((long long)al << 32) + max(al - L.cnt[e], 0);
     }
     const int total_rows = (int)(total >> 32), total_pad = (int)(total & 0xffffffffll);
     if (tid == 0) {
@@ -279,6 +314,7 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     if (c == 0) {
         for (int e = tid; e < E; e += NT) {
             a.cnt[e] = L.cnt[e];
+            if (a.slab > 0 && L.cnt[e] > a.slab) s_over = 1;   // more pairs than the slab holds
             if (a.stats) a.stats[e] += L.cnt[e];
             a.off[e] = L.off[e];
             a.padpre[e] = L.padpre[e];
@@ -303,7 +339,9 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
             __syncwarp();
             if (key >= 0 && lane == __ffs(peers) - 1) my[key] += __popc(peers);
             __syncwarp();
+            if (a.slab > 0 && slot >= 0 && slot - L.off[key] >= a.slab) slot = -1;   // past its slab: dropped
             if (i < q1) {
+                if (kRankKeys && a.in_rank) a.in_rank[i] = key >= 0 ? 1 : 0;
                 a.pair_slot[i] = slot;
                 if (slot >= 0 && (int64_t)slot < a.capacity) {
                     a.recv_src[slot] = (int32_t)(i / K);
@@ -315,9 +353,10 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
 #pragma unroll
         for (int r = 0; r < kKeyRounds; ++r)
             if (q0 + 32 * r < q1) assign_round(q0 + 32 * r, keys[r]);
+        bool unused = false;
         for (int64_t qb = q0 + 32 * kKeyRounds; qb < q1; qb += 32) {
             const int64_t i = qb + lane;
-            assign_round(qb, (i < q1) ? valid_expert(a.topk_idx[i], E) : -1);
+            assign_round(qb, (i < q1) ? pair_key<kRankKeys>(a, i, unused) : -1);
         }
     }
 
@@ -336,7 +375,7 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     }
     if (c == 0 && tid == 0) {   // fold the flags of this call into the status word
         uint32_t flags = atomicExch(&a.hdr->pending, 0u);
-        if ((int64_t)total_rows > a.capacity) flags |= kDevCapacity;
+        if ((int64_t)total_rows > a.capacity || s_over) flags |= kDevCapacity;
         if (flags) atomicOr(&a.hdr->status, flags);
     }
     __syncthreads();

@@ -7,19 +7,22 @@
 //
 // A token reaches rank r when one of its experts lives there (e / (E/R) == r).
 // The receive rows are the (rank, token) pairs in rank-major, token-ascending
-// order.  That is exactly the expand layout of a derived routing table with
-// one "expert" per rank - entry (t, r) = r if the token reaches r, else -1 -
-// with E' = K' = R and alignment 1, so the rows come from the same layout
-// kernel (per-chunk counts, one grid barrier, scan, stable slots):
-//   1. rank_prep_kernel reads topk_idx once and writes the derived table
-//      [T, R] to the workspace, is_token_in_rank [T, R], and the per-expert
-//      pair counts (a shared-memory histogram per CTA, then one global add
-//      per expert and CTA; integer sums, so the result does not depend on
-//      the order of the adds);
-//   2. layout_kernel on the derived table gives num_tokens_per_rank, the rank
-//      offsets, token_slot [T, R] and recv_src_token;
-//   3. rank_post_kernel writes recv_topk_idx / recv_topk_weights row by row
-//      and the expert counts, plain and aligned.
+// order.  That is exactly the expand layout of a (token, rank) table with one
+// "expert" per rank - entry (t, r) = r if the token reaches r, else -1 - with
+// E' = K' = R and alignment 1, so the rows come from the same layout kernel
+// (per-chunk counts, one grid barrier, scan, stable slots), whose keys are
+// computed from topk_idx on the fly (LayoutArgs::src_idx):
+//   1. layout_kernel with per-rank keys: num_tokens_per_rank, the rank
+//      offsets, token_slot [T, R], recv_src_token and is_token_in_rank;
+//   2. rank_post_kernel, over the (token, rank) pairs: recv_topk_idx /
+//      recv_topk_weights of every row, and the per-expert pair counts - each
+//      selected (t, k) is local to exactly one reached rank, so counting the
+//      local entries of every row counts every pair once.  A shared-memory
+//      histogram per CTA goes to a zeroed workspace array with one atomic add
+//      per expert; the last CTA to finish (a counter, after a fence) writes
+//      the plain and aligned counts and zeroes the array and the counter for
+//      the next call.  Integer sums, so the result does not depend on the
+//      order of the adds.
 #include "ep_internal.h"
 
 namespace ep {
@@ -28,76 +31,60 @@ namespace {
 
 constexpr int kRankThreads = 256;
 
-__global__ void __launch_bounds__(kRankThreads) rank_prep_kernel(const int64_t* topk_idx, int T, int K, int E,
-                                                                 int R, int64_t* rank_idx, uint8_t* in_rank,
-                                                                 int32_t* counts, WsHeader* hdr) {
-    extern __shared__ int32_t hist[];   // [E]
-    for (int e = threadIdx.x; e < E; e += kRankThreads) hist[e] = 0;
-    __syncthreads();
-    pdl_wait();
-    pdl_launch_dependents();
-    const int El = E / R;
-    const int64_t stride = (int64_t)gridDim.x * kRankThreads;
-    bool bad = false;
-    for (int64_t t = (int64_t)blockIdx.x * kRankThreads + threadIdx.x; t < T; t += stride) {
-        uint32_t mask = 0;
-        for (int k = 0; k < K; ++k) {
-            const int64_t e = topk_idx[t * K + k];
-            if (e >= 0 && e < E) {
-                mask |= 1u << (int)(e / El);
-                atomicAdd(&hist[e], 1);
-            } else if (e != -1) {
-                bad = true;   // outside [-1, E): reported, treated as -1
-            }
-        }
-        for (int r = 0; r < R; ++r) {
-            const bool in = (mask >> r) & 1u;
-            rank_idx[t * R + r] = in ? r : -1;
-            if (in_rank) in_rank[t * R + r] = in ? 1 : 0;
-        }
-    }
-    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(&hdr->pending, kDevBadExpert);
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += kRankThreads)
-        if (hist[e]) atomicAdd(&counts[e], hist[e]);
-}
-
-// Rank of receive row `row`: the r with rank_off[r] <= row < rank_off[r + 1].
-__device__ __forceinline__ int row_rank(const int32_t* rank_off, int R, int row) {
-    int lo = 0, hi = R - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (rank_off[mid] <= row) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
-
 __global__ void __launch_bounds__(kRankThreads) rank_post_kernel(RankPostArgs a) {
+    extern __shared__ int32_t hist[];   // [E]
+    __shared__ int s_last;
+    for (int e = threadIdx.x; e < a.E; e += kRankThreads) hist[e] = 0;
+    __syncthreads();
     pdl_wait();
     pdl_launch_dependents();
     const int El = a.E / a.R, K = a.K;
     const int64_t stride = (int64_t)gridDim.x * kRankThreads;
-    const int64_t gid = (int64_t)blockIdx.x * kRankThreads + threadIdx.x;
-    int64_t rows = a.rank_off[a.R];
-    if (rows > a.capacity) rows = a.capacity;
-    if (a.recv_topk_idx || a.recv_topk_w) {
-        for (int64_t row = gid; row < rows; row += stride) {
-            const int r = row_rank(a.rank_off, a.R, (int)row);
-            const int64_t t = a.recv_src[row];
-            for (int k = 0; k < K; ++k) {
-                const int64_t e = a.topk_idx[t * K + k];
+    const int64_t n = (int64_t)a.T * a.R;
+    for (int64_t i = (int64_t)blockIdx.x * kRankThreads + threadIdx.x; i < n; i += stride) {
+        const int32_t slot = a.token_slot[i];
+        if (slot < 0) continue;
+        const int64_t t = i / a.R;
+        const int r = (int)(i - t * a.R);
+        const bool write = (int64_t)slot < a.capacity;
+        // the token's ids and weights eight at a time, all loads before any use
+        for (int k0 = 0; k0 < K; k0 += 8) {
+            int64_t ev[8];
+            float wv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const bool in = k0 + j < K;
+                ev[j] = in ? a.topk_idx[t * K + k0 + j] : -1;
+                wv[j] = (in && a.topk_weights) ? a.topk_weights[t * K + k0 + j] : 1.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int k = k0 + j;
+                if (k >= K) break;
+                const int64_t e = ev[j];
                 const bool local = e >= 0 && e < a.E && e / El == r;
-                if (a.recv_topk_idx) a.recv_topk_idx[row * K + k] = local ? e - (int64_t)r * El : -1;
-                if (a.recv_topk_w)
-                    a.recv_topk_w[row * K + k] = local ? (a.topk_weights ? a.topk_weights[t * K + k] : 1.0f) : 0.0f;
+                if (local) atomicAdd(&hist[e], 1);
+                if (write && a.recv_topk_idx) a.recv_topk_idx[(int64_t)slot * K + k] = local ? e - (int64_t)r * El : -1;
+                if (write && a.recv_topk_w) a.recv_topk_w[(int64_t)slot * K + k] = local ? wv[j] : 0.0f;
             }
         }
     }
-    for (int64_t e = gid; e < a.E; e += stride) {
-        const int32_t c = a.counts[e];
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.E; e += kRankThreads)
+        if (hist[e]) atomicAdd(&a.counts[e], hist[e]);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(a.done, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();   // every other CTA's adds are visible before the counter said so
+    for (int e = threadIdx.x; e < a.E; e += kRankThreads) {
+        const int32_t c = __ldcg(&a.counts[e]);
         if (a.num_tokens_per_expert) a.num_tokens_per_expert[e] = c;
         if (a.num_recv_per_expert) a.num_recv_per_expert[e] = (c + a.A - 1) / a.A * a.A;
+        a.counts[e] = 0;
     }
+    if (threadIdx.x == 0) *a.done = 0;
 }
 
 }  // namespace
@@ -106,32 +93,23 @@ RankWsLayout rank_ws_layout(int T, int R, int E) {
     RankWsLayout w;
     w.expand = ws_layout(T, R, R, 1);
     const size_t n = (size_t)(T > 0 ? T : 0) * (size_t)R;
-    w.rank_idx_off = w.expand.total;
-    w.scratch_w_off = round_up(w.rank_idx_off + n * 8, 256);
+    w.scratch_w_off = w.expand.total;
     w.scratch_lexp_off = round_up(w.scratch_w_off + n * 4, 256);
     w.counts_off = round_up(w.scratch_lexp_off + n * 4, 256);
-    w.total = round_up(w.counts_off + (size_t)E * 4, 256);
+    w.done_off = round_up(w.counts_off + (size_t)E * 4, 256);
+    w.total = round_up(w.done_off + 4, 256);
     return w;
 }
 
-cudaError_t launch_rank_layout(const RankPrepArgs& p, LayoutArgs la, const RankPostArgs& post, int sms,
-                               cudaStream_t s) {
-    cudaError_t err = cudaMemsetAsync(p.counts, 0, (size_t)p.E * 4, s);
+cudaError_t launch_rank_layout(LayoutArgs la, const RankPostArgs& post, int sms, cudaStream_t s) {
+    cudaError_t err = launch_layout(la, sms, s);
     if (err != cudaSuccess) return err;
-    const size_t smem = (size_t)p.E * 4;
-    int grid = (p.T + kRankThreads - 1) / kRankThreads;
+    const int64_t n = (int64_t)post.T * post.R;
+    int64_t grid = (n + kRankThreads - 1) / kRankThreads;
     if (grid > 2 * sms) grid = 2 * sms;
     if (grid < 1) grid = 1;
-    err = launch_pdl(rank_prep_kernel, dim3(grid), dim3(kRankThreads), smem, s, false, p.topk_idx, p.T, p.K, p.E,
-                     p.R, p.rank_idx, p.in_rank, p.counts, p.hdr);
-    if (err != cudaSuccess) return err;
-    err = launch_layout(la, sms, s);
-    if (err != cudaSuccess) return err;
-    const int64_t rows = (int64_t)p.T * p.R;
-    int64_t pg = (rows + kRankThreads - 1) / kRankThreads;
-    if (pg > 2 * sms) pg = 2 * sms;
-    if (pg < 1) pg = 1;
-    return launch_pdl(rank_post_kernel, dim3((unsigned)pg), dim3(kRankThreads), 0, s, false, post);
+    return launch_pdl(rank_post_kernel, dim3((unsigned)grid), dim3(kRankThreads), (size_t)post.E * 4, s, false,
+                      post);
 }
 
 }  // namespace ep

@@ -21,6 +21,8 @@
  *   ep_rank_layout  §2.1 dispatch() without do_expand (one receive row per
  *                token and destination rank) with §3.1's V1 layout quantities;
  *                its handle serves ep_dispatch and §3.2's unweighted combine.
+ *   ep_ll_layout §3.3 low_latency_dispatch: a fixed slab of R * max_tokens
+ *                receive rows per expert.
  * The placement also matches the last stages of the Ascend full-mesh dispatch
  * on the "URMA" tag page (count reconciliation, prefix-sum placement, reorder).
  *
@@ -62,7 +64,7 @@
 extern "C" {
 #endif
 
-#define EP_B200_VERSION 4
+#define EP_B200_VERSION 5
 
 /* Host return codes. */
 #define EP_OK 0
@@ -165,6 +167,7 @@ typedef struct ep_layout_t {
 /* Receive forms of a handle (its `kind` field). */
 #define EP_LAYOUT_EXPAND 0     /* ep_layout: one row per selected (token, k) pair */
 #define EP_LAYOUT_PER_RANK 1   /* ep_rank_layout: one row per (token, rank) reached */
+#define EP_LAYOUT_LL_SLAB 2    /* ep_ll_layout: a fixed slab of rows per expert */
 
 /* Bytes of workspace ep_layout needs for these sizes (a pure host function). */
 size_t ep_workspace_bytes(int num_tokens, int num_topk, int num_experts, int expert_alignment);
@@ -234,13 +237,35 @@ int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens
  * The handle works with ep_dispatch (rows per (token, rank)) and ep_combine
  * (§3.2 V1: topk_weights must be NULL; out[t] = the plain sum over the ranks
  * the token reached, in ascending rank order, plus the biases).  Device-side
- * errors as for ep_layout.  Four launches: a memset, three kernels.
+ * errors as for ep_layout.  Two kernels.
  */
 size_t ep_rank_workspace_bytes(int num_tokens, int num_ranks, int num_experts);
 int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
                    int num_experts, int num_ranks, int expert_alignment, uint8_t* is_token_in_rank,
                    int32_t* num_tokens_per_expert, int32_t* num_recv_tokens_per_expert, int64_t* recv_topk_idx,
                    float* recv_topk_weights, ep_layout_t* layout, void* stream);
+
+/*
+ * Low-latency fixed-slab layout (§3.3 low_latency_dispatch: every rank has
+ * the same num_max_dispatch_tokens_per_rank M; a rank receives
+ * [E/R, R*M, H]).  With S = R*M, expert e owns receive rows [e*S, (e+1)*S):
+ * its pairs first, in token-major, k-minor order (as ep_layout), then padding
+ * rows up to the end of the slab.  Arguments and results as for ep_layout with
+ * expert_alignment 1 and num_max_tokens_per_rank M (T/R > M is
+ * EP_ERR_CAPACITY), except that expert_offset[e] = e*S, the receive buffers
+ * need capacity >= E*S rows, and the workspace is
+ * ep_ll_workspace_bytes(T, K, E, R, M) bytes.  An expert with more than S
+ * pairs (only possible when a token repeats an expert) sets EP_DEV_CAPACITY;
+ * its pairs past the slab get pair_slot -1 and are not written.  Sets kind =
+ * EP_LAYOUT_LL_SLAB; the handle serves ep_dispatch (do_zero_padding zeroes
+ * the unused slab rows) and ep_combine (weighted, as §3.4's low-latency
+ * combine).  T = 0 is allowed: every slab row is then padding.
+ */
+size_t ep_ll_workspace_bytes(int num_tokens, int num_topk, int num_experts, int num_ranks,
+                             int num_max_dispatch_tokens_per_rank);
+int ep_ll_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
+                 int num_experts, int num_ranks, int num_max_dispatch_tokens_per_rank, ep_layout_t* layout,
+                 void* stream);
 
 /*
  * Dispatch (§2.1): for every selected pair (t, k), receive row

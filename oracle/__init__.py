@@ -368,14 +368,27 @@ def bf16_to_f32(b):
     return (b.astype(np.uint32) << 16).view(np.float32)
 
 
-def step(inp, cfg, per_rank=False):
+def step_layout(inp, cfg, form="expand"):
+    """The layout of one step: ``form`` "expand" (the default), "rank" (the
+    per-token-per-rank layout) or "ll" (the fixed-slab layout with
+    max_tokens_per_rank, or T / R, tokens per rank)."""
+    if form == "rank":
+        return rank_layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"])
+    if form == "ll":
+        return ll_layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"],
+                         cfg.get("max_tokens_per_rank", 0) or cfg["T"] // cfg["R"])
+    return layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"],
+                  cfg.get("max_tokens_per_rank", 0))
+
+
+def step(inp, cfg, form="expand"):
     """One pass of the whole path on host arrays: layout, dispatch (with the
     fused cast in FP8 mode) and combine of the given expert outputs.  Used by the
-    benchmark's CPU baseline.  ``per_rank``: the per-token-per-rank layout and
-    V1's unweighted combine instead of the expand layout.  Returns (layout,
-    recv rows, combined out)."""
-    if per_rank:
-        lay = rank_layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"])
+    benchmark's CPU baseline.  ``form`` as for ``step_layout``; the per-rank
+    form combines without weights (V1).  Returns (layout, recv rows, combined out)."""
+    per_rank = form == "rank"
+    if form != "expand":
+        lay = step_layout(inp, cfg, form)
     else:
         lay = layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"],
                      cfg.get("max_tokens_per_rank", 0))

@@ -46,7 +46,7 @@ def test_struct_size_matches_header(lib):
 
 
 def test_pure_host_functions(lib):
-    assert lib.ep_version() == 4
+    assert lib.ep_version() == 5
     assert lib.ep_capacity_rows(4096, 8, 256, 128) == 4096 * 8 + 256 * 127
     assert lib.ep_capacity_rows(128, 4, 16, 1) == 512
     ws = lib.ep_workspace_bytes(4096, 8, 256, 128)
@@ -114,7 +114,7 @@ def test_rank_layout_host_checks(lib, T, K, E, R, A, expect):
 def test_rank_layout_workspace_and_pointers(lib):
     p = ctypes.c_void_p(0x10000)
     ws = lib.ep_rank_workspace_bytes(4096, 8, 256)
-    assert ws % 256 == 0 and ws >= lib.ep_workspace_bytes(4096, 8, 8, 1) + 4096 * 8 * 16 + 256 * 4
+    assert ws % 256 == 0 and ws >= lib.ep_workspace_bytes(4096, 8, 8, 1) + 4096 * 8 * 8 + 256 * 4
     assert lib.ep_rank_workspace_bytes(-1, 8, 256) == 0
     s = _handle(ws_bytes=ws - 256)
     assert lib.ep_rank_layout(p, None, 4096, 8, 256, 8, 1, None, None, None, None, None, ctypes.byref(s), None) == 1
@@ -130,6 +130,19 @@ def test_rank_layout_workspace_and_pointers(lib):
     s = _handle(magic=0x45504C31)
     s.num_tokens, s.num_topk, s.num_experts, s.num_ranks, s.expert_alignment, s.kind = 8, 2, 2, 2, 1, 1
     assert lib.ep_combine(ctypes.byref(s), p, 256, p, None, None, p, None) == 1
+
+
+def test_ll_layout_host_checks(lib):
+    p = ctypes.c_void_p(0x10000)
+    ws = lib.ep_ll_workspace_bytes(128, 8, 256, 8, 128)
+    assert ws >= 256 * 8 * 128 * 4                              # room to list every slab row as padding
+    assert lib.ep_ll_workspace_bytes(128, 8, 256, 8, 0) == 0
+    s = _handle(ws_bytes=ws)
+    assert lib.ep_ll_layout(p, None, 128, 8, 256, 8, 0, ctypes.byref(s), None) == 1        # M < 1
+    assert lib.ep_ll_layout(p, None, 128, 8, 256, 8, 8, ctypes.byref(s), None) == 2        # T/R = 16 > M = 8
+    s = _handle(ws_bytes=ws - 256)
+    assert lib.ep_ll_layout(p, None, 128, 8, 256, 8, 128, ctypes.byref(s), None) == 1      # workspace too small
+    assert s.magic == 0
 
 
 def test_layout_rejects_misaligned_recv_stats(lib):
