@@ -41,8 +41,8 @@ FLUSH_BYTES = 256 << 20
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=30)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="prefill_bf16", choices=sorted(workload.WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
@@ -308,7 +308,9 @@ def run_ours(args, rank, world, local_rank):
     if dist:
         dist.barrier()
     clock_info = clocks.stop() if clocks else None
-    ms_per_step = max_over_ranks(np.mean([e[0].elapsed_time(e[1]) for e in evs]), dist, dev)
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    ms_per_step = max_over_ranks(np.mean(step_ms), dist, dev)
+    ms_median = max_over_ranks(float(np.median(step_ms)), dist, dev)
     # per-kernel breakdown: the same K steps again with events between the kernels
     evk = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     for i in range(args.steps):
@@ -329,6 +331,7 @@ def run_ours(args, rank, world, local_rank):
         return None
 
     peak, peak_kind = measured_peaks()
+    payload_rows = nbytes["Np"] - nbytes["pad_rows"]
     k_ms = per.mean(axis=0)   # layout, dispatch, combine (fused: layout+dispatch, -, combine)
     total_bytes = nbytes["layout"] + nbytes["dispatch"] + nbytes["combine"]
     if not args.fused:
@@ -364,6 +367,11 @@ def run_ours(args, rank, world, local_rank):
             "l2": "flushed by a 256 MiB write before every step, outside the timed events",
             "pairs": nbytes["N"], "recv_rows": nbytes["Np"], "pad_rows": nbytes["pad_rows"],
             "load": workload.load_stats(inp["topk_idx"], E)},
+        "ms_per_step_median": round(ms_median, 5),
+        # the count_bytes convention: one row copy in dispatch and one row read in
+        # combine per receive row that holds data
+        "payload_gbs": round(payload_rows * ((H + 4 * (H // 128) if fp8 else 2 * H) + 2 * H)
+                             / (ms_per_step * 1e-3) / 1e9, 1),
         "hbm_gbs": round(total_bytes / (ms_per_step * 1e-3) / 1e9, 1),
         "hbm_frac_of_measured": round(total_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4),
         "hbm_frac_of_nominal_8tbs": round(total_bytes / (ms_per_step * 1e-3) / 1e9 / 8000.0, 4),

@@ -13,7 +13,9 @@
 // A work item is (token, 32*V 16-byte columns); a warp issues the loads of KB
 // rows of its item together before summing them, so each lane keeps KB*V
 // loads in flight, and every row is read in contiguous 32*V*16-byte pieces.
-// Padding rows are never read.
+// The item's selected entries are first packed to the front of the warp (in
+// ascending k), so -1 entries take no place in a batch.  Padding rows are
+// never read.
 #include <cuda_bf16.h>
 
 #include "ep_internal.h"
@@ -84,13 +86,29 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
     int next_slot;
     float next_w;
     fetch(gw, next_slot, next_w);
+    // per warp: the item's selected entries moved to the front, in ascending k
+    __shared__ int2 packed[kCombineThreads / 32][32];
+    int2* my_packed = packed[threadIdx.x >> 5];
     for (int64_t it = gw; it < items; it += nw) {
         const int64_t t = it / nch;
         const int ch = (int)(it % nch);
         int my_slot = next_slot;
-        const float my_w = next_w;
+        float my_w = next_w;
         fetch(it + nw, next_slot, next_w);
         if ((int64_t)my_slot >= a.capacity) my_slot = -1;
+        // compaction: lane k with a selected entry writes it to position
+        // popc(selected below k); the loop below then runs over nsel entries
+        // with no holes, in the same ascending-k order
+        const uint32_t sel = __ballot_sync(0xffffffffu, lane < K && my_slot >= 0);
+        const int nsel = __popc(sel);
+        if ((sel >> lane) & 1u) my_packed[__popc(sel & lanemask_lt())] = make_int2(my_slot, __float_as_int(my_w));
+        __syncwarp();
+        if (lane < nsel) {
+            const int2 p = my_packed[lane];
+            my_slot = p.x;
+            my_w = __int_as_float(p.y);
+        }
+        __syncwarp();
         float acc[V][8];
 #pragma unroll
         for (int v = 0; v < V; ++v)
@@ -112,13 +130,13 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
             }
         }
 
-        for (int k0 = 0; k0 < K; k0 += KB) {
+        for (int k0 = 0; k0 < max(nsel, 1); k0 += KB) {
             uint4 rows[KB][V];
 #pragma unroll
             for (int kk = 0; kk < KB; ++kk) {
                 const int k = k0 + kk;
                 const int slot = __shfl_sync(0xffffffffu, my_slot, k & 31);
-                const bool use = (k < K) && slot >= 0;
+                const bool use = k < nsel;
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
                     const int col = ch * per_item + v * 32 + lane;
@@ -133,9 +151,8 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
 #pragma unroll
             for (int kk = 0; kk < KB; ++kk) {
                 const int k = k0 + kk;
-                const int slot = __shfl_sync(0xffffffffu, my_slot, k & 31);
                 const float w = __shfl_sync(0xffffffffu, my_w, k & 31);
-                if (k < K && slot >= 0) {
+                if (k < nsel) {
 #pragma unroll
                     for (int v = 0; v < V; ++v) accumulate8(acc[v], rows[kk][v], w);
                 }
@@ -170,11 +187,12 @@ __global__ void selftest_wait_kernel(WsHeader* hdr, uint64_t timeout_ns) {
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
-    // items of 2 KB per row, rows loaded 4 at a time: contiguous 2 KB reads per
-    // row keep DRAM pages open (measured faster than 1 KB items with 8 rows in
-    // flight, and than staging the rows through shared memory with TMA); with
-    // a bias, 2 rows at a time keep the bias registers from spilling
-    auto kernel = a.bias0 ? combine_kernel<4, 2, 2, true> : combine_kernel<4, 2, 4, false>;
+    // 1 KB of each row per item, two rows in flight per lane without a bias,
+    // eight with one: the fastest of the (columns per lane, rows per batch)
+    // pairs measured on the prefill and decode workloads, expand and per-rank
+    // handles, once the selected entries are packed (2-8 rows per batch,
+    // 512 B - 4 KB per row and item)
+    auto kernel = a.bias0 ? combine_kernel<2, 2, 8, true> : combine_kernel<2, 2, 2, false>;
     int blocks_per_sm = 0;
     cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kernel, kCombineThreads, 0);
     if (err != cudaSuccess) return err;
