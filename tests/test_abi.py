@@ -222,3 +222,32 @@ def test_product_path_has_no_cpu_fallback():
             L.load()
     finally:
         L._LIB_PATH, L._lib = saved
+
+
+def _cc(args, tmp_path):
+    import subprocess
+    res = subprocess.run(args, capture_output=True, text=True, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-3000:]
+    return res
+
+
+def test_header_is_plain_c_and_cpp(tmp_path):
+    """The ABI header compiles on its own as C11 and as C++17 (no torch, no CUDA types)."""
+    src = tmp_path / "hdr.c"
+    src.write_text('#include "ep_b200.h"\nint main(void) { return ep_version() == EP_B200_VERSION ? 0 : 1; }\n')
+    _cc(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only", "-I", "include", str(src)],
+        tmp_path)
+    cpp = tmp_path / "hdr.cpp"
+    cpp.write_text(src.read_text())
+    _cc(["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-I", "include", str(cpp)], tmp_path)
+
+
+def test_c_client_builds_and_links(lib, tmp_path):
+    """tests/c_abi_client.c, a torch-free C program over the ABI, compiles and
+    links against libep_b200.so (it runs on a GPU in test_gpu_c_abi.py)."""
+    from combine_ep_layout_11_b200 import build
+    exe = tmp_path / "c_abi_client"
+    _cc(["gcc", "-std=c11", "-O2", "-Wall", "-Wextra", "-Werror", "-I", "include", "-I", "/usr/local/cuda/include",
+         "tests/c_abi_client.c", "-o", str(exe), "-L", os.path.dirname(build.LIB), "-lep_b200",
+         "-L", "/usr/local/cuda/lib64", "-lcudart"], tmp_path)
+    assert exe.exists()
