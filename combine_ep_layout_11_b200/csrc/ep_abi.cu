@@ -82,6 +82,13 @@ int prepare_layout(const int64_t* topk_idx, const float* topk_weights, int T, in
     a->src_K = 0;
     a->src_E = 0;
     a->in_rank = nullptr;
+    a->src_w = nullptr;
+    a->src_A = 1;
+    a->src_counts = nullptr;
+    a->n_exp_out = nullptr;
+    a->n_recv_out = nullptr;
+    a->rank_topk_idx = nullptr;
+    a->rank_topk_w = nullptr;
     return EP_OK;
 }
 
@@ -248,24 +255,18 @@ int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_t
     la.src_K = K;
     la.src_E = E;
     la.in_rank = is_token_in_rank;
-
-    ep::RankPostArgs post;
-    post.topk_idx = topk_idx;
-    post.topk_weights = topk_weights;
-    post.token_slot = layout->pair_slot;
-    post.T = T; post.K = K; post.E = E; post.R = R; post.A = A;
-    post.capacity = layout->capacity;
-    post.counts = reinterpret_cast<int32_t*>(wsb + ws.counts_off);
-    post.done = reinterpret_cast<uint32_t*>(wsb + ws.done_off);
-    post.recv_topk_idx = recv_topk_idx;
-    post.recv_topk_w = recv_topk_weights;
-    post.num_tokens_per_expert = num_tokens_per_expert;
-    post.num_recv_per_expert = num_recv_tokens_per_expert;
+    la.src_w = topk_weights;
+    la.src_A = A;
+    la.src_counts = reinterpret_cast<int32_t*>(wsb + ws.counts_off);
+    la.n_exp_out = num_tokens_per_expert;
+    la.n_recv_out = num_recv_tokens_per_expert;
+    la.rank_topk_idx = recv_topk_idx;
+    la.rank_topk_w = recv_topk_weights;
 
     int sms = 0;
     int rc = device_sms(&sms);
     if (rc != EP_OK) return rc;
-    return ep::launch_rank_layout(la, post, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    return ep::launch_layout(la, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
 size_t ep_ll_workspace_bytes(int num_tokens, int num_topk, int num_experts, int num_ranks,

@@ -35,6 +35,16 @@ struct LayoutArgs {
     const int64_t* src_idx;
     int src_K, src_E;
     uint8_t* in_rank;
+    // Per-rank keys only, all nullable: the per-expert pair counts (plain and
+    // aligned to src_A), counted through src_counts ([src_E] workspace, zero
+    // between calls), and each reached row's rank-local expert ids and weights.
+    const float* src_w;
+    int src_A;
+    int32_t* src_counts;
+    int32_t* n_exp_out;
+    int32_t* n_recv_out;
+    int64_t* rank_topk_idx;
+    float* rank_topk_w;
 };
 
 // One cooperative kernel: per-chunk counts, a grid barrier, the scans and the
@@ -98,33 +108,15 @@ cudaError_t launch_selftest_wait(WsHeader* hdr, uint64_t timeout_ns, cudaStream_
 // Per-token-per-rank layout (ep_rank_layout.cu).  Workspace: the expand-layout
 // workspace of the [T, R] (token, rank) table (E' = K' = R, A = 1), scratch
 // targets for the layout kernel's per-row weight and local-expert writes
-// (meaningless here), the per-expert pair counts (int32 [E]) and a counter of
-// finished CTAs; both are zero between calls.
+// (meaningless here) and the per-expert pair counts (int32 [E], zero between
+// calls).
 struct RankWsLayout {
     WsLayout expand;
     size_t scratch_w_off;
     size_t scratch_lexp_off;
     size_t counts_off;
-    size_t done_off;
     size_t total;
 };
 RankWsLayout rank_ws_layout(int T, int R, int E);
-
-struct RankPostArgs {
-    const int64_t* topk_idx;   // [T*K]
-    const float* topk_weights; // [T*K] or nullptr
-    const int32_t* token_slot; // [T*R]
-    int T, K, E, R, A;
-    int64_t capacity;
-    int32_t* counts;           // [E] workspace, zero on entry and on exit
-    uint32_t* done;            // workspace counter, zero on entry and on exit
-    int64_t* recv_topk_idx;    // [capacity][K], nullable
-    float* recv_topk_w;        // [capacity][K], nullable
-    int32_t* num_tokens_per_expert;   // [E], nullable
-    int32_t* num_recv_per_expert;     // [E] aligned, nullable
-};
-
-// The layout kernel with per-rank keys, then the post kernel.
-cudaError_t launch_rank_layout(LayoutArgs la, const RankPostArgs& post, int sms, cudaStream_t s);
 
 }  // namespace ep

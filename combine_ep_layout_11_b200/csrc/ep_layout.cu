@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(NT) layout_kernel(LayoutArgs a) {
 template <int NT, bool kRankKeys>
 cudaError_t launch_layout_nt(LayoutArgs a, int sms, cudaStream_t s) {
     auto kernel = layout_kernel<NT, kRankKeys>;
-    const size_t smem = layout_dev::layout_smem_ints(a.E) * sizeof(int32_t);
+    const size_t smem = layout_dev::layout_smem_ints(a.E, kRankKeys ? a.src_E : 0) * sizeof(int32_t);
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     int per_sm = 0;

@@ -16,10 +16,11 @@ constexpr int kKeyRounds = 4;   // rounds of 32 pairs per warp whose expert ids 
 __host__ __device__ inline int layout_threads(int E) { return E <= kWideMaxExperts ? kWideThreads : kNarrowThreads; }
 
 // Shared memory of layout_body, in ints: per-warp counts [warps][Ep], counts,
-// bases, offsets and padding prefix [Ep (+4)], scan partials [8 * threads].
-__host__ __device__ inline size_t layout_smem_ints(int E) {
+// bases, offsets and padding prefix [Ep (+4)], scan partials [8 * threads];
+// with per-rank keys also a histogram of the src_E experts.
+__host__ __device__ inline size_t layout_smem_ints(int E, int src_E = 0) {
     const int Ep = round4(E), nt = layout_threads(E);
-    return (size_t)(nt / 32) * Ep + 4 * (size_t)Ep + 8 + 8 * (size_t)nt;
+    return (size_t)(nt / 32) * Ep + 4 * (size_t)Ep + 8 + 8 * (size_t)nt + (size_t)round4(src_E);
 }
 
 // Where layout_body leaves its per-chunk results in shared memory.
@@ -30,6 +31,7 @@ struct LayoutSmem {
     int32_t* off;      // [Ep + 4] aligned offsets, off[E] = rows used
     int32_t* padpre;   // [Ep + 4] padding prefix, padpre[E] = padding rows
     int32_t* part;     // [8 * threads] scan partials
+    int32_t* ehist;    // [src_E] per-rank keys: pairs per expert in this chunk
     __host__ __device__ LayoutSmem(int32_t* sm, int E) {
         const int Ep = round4(E), nw = layout_threads(E) / 32;
         wh = sm;
@@ -38,6 +40,7 @@ struct LayoutSmem {
         off = base + Ep;
         padpre = off + Ep + 4;
         part = padpre + Ep + 4;
+        ehist = part + 8 * layout_threads(E);
     }
 };
 
@@ -51,7 +54,7 @@ __device__ __forceinline__ int valid_expert(int64_t e, int E) { return (e >= 0 &
 // [-1, E).  The token's ids are loaded eight at a time, all eight before any
 // is used, so a key costs one memory round trip per eight experts.
 template <bool kRankKeys>
-__device__ __forceinline__ int pair_key(const LayoutArgs& a, int64_t i, bool& bad) {
+__device__ __forceinline__ int pair_key(const LayoutArgs& a, int64_t i, bool& bad, int32_t* hist = nullptr) {
     if (!kRankKeys) {
         const int64_t e = a.topk_idx[i];
         const int key = valid_expert(e, a.E);
@@ -72,7 +75,11 @@ __device__ __forceinline__ int pair_key(const LayoutArgs& a, int64_t i, bool& ba
         for (int j = 0; j < 8; ++j) {
             const int64_t e = ev[j];
             if (e >= 0 && e < a.src_E) {
-                if (e / El == r) key = r;
+                if (e / El == r) {
+                    key = r;
+                    // each selected (t, k) is local to exactly one rank: counted once
+                    if (hist) atomicAdd(&hist[e], 1);
+                }
             } else if (e != -1) {
                 bad = true;
             }
@@ -102,6 +109,61 @@ __device__ __forceinline__ uint32_t atom_add_release_u32(uint32_t* p, uint32_t v
 
 // Exclusive scan of one 64-bit value per thread across a CTA of NT threads;
 // *total gets the sum.  `scratch` holds NT / 32 values.
+// Per-rank keys: the rank-local expert ids and weights of receive row `slot`,
+// which holds pair i = (t, r).  Entries whose expert is on another rank get -1
+// and weight 0.  With K a multiple of 4 and 16-byte aligned arrays a row goes
+// out in 16-byte stores (two per four ids, one per four weights).
+__device__ __forceinline__ void write_rank_row(const LayoutArgs& a, int64_t i, int slot) {
+    if (!a.rank_topk_idx && !a.rank_topk_w) return;
+    const int R = a.K, K = a.src_K;
+    const int64_t t = i / R;
+    const int r = (int)(i - t * R);
+    const int El = a.src_E / R;
+    const int64_t* row = a.src_idx + t * K;
+    int64_t* oi = a.rank_topk_idx ? a.rank_topk_idx + (int64_t)slot * K : nullptr;
+    float* ow = a.rank_topk_w ? a.rank_topk_w + (int64_t)slot * K : nullptr;
+    const bool vec = (K % 4) == 0 && ((reinterpret_cast<uintptr_t>(a.rank_topk_idx) |
+                                       reinterpret_cast<uintptr_t>(a.rank_topk_w)) & 15u) == 0;
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        int64_t ev[8];
+        float wv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const bool in = k0 + j < K;
+            ev[j] = in ? row[k0 + j] : -1;
+            wv[j] = (in && a.src_w) ? a.src_w[t * K + k0 + j] : 1.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j += 4) {
+            const int k = k0 + j;
+            if (k >= K) break;
+            long long o[4];
+            float w4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int64_t e = ev[j + q];
+                const bool local = k + q < K && e >= 0 && e < a.src_E && e / El == r;
+                o[q] = local ? e - (int64_t)r * El : -1;
+                w4[q] = local ? wv[j + q] : 0.0f;
+            }
+            if (vec) {
+                if (oi) {
+                    reinterpret_cast<longlong2*>(oi + k)[0] = make_longlong2(o[0], o[1]);
+                    reinterpret_cast<longlong2*>(oi + k)[1] = make_longlong2(o[2], o[3]);
+                }
+                if (ow) *reinterpret_cast<float4*>(ow + k) = make_float4(w4[0], w4[1], w4[2], w4[3]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (k + q >= K) break;
+                    if (oi) oi[k + q] = o[q];
+                    if (ow) ow[k + q] = w4[q];
+                }
+            }
+        }
+    }
+}
+
 template <int NT>
 __device__ __forceinline__ long long block_exclusive_scan64(long long v, long long* scratch, long long* total) {
     constexpr int kW = NT / 32;
@@ -198,6 +260,10 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
         s_over = 0;
     }
     for (int e = lane; e < Ep; e += 32) my[e] = 0;
+    if (kRankKeys) {
+        for (int e = tid; e < a.src_E; e += NT) L.ehist[e] = 0;
+        __syncthreads();
+    }
     __syncwarp();
 
     // ---- count ----
@@ -206,7 +272,9 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     const int64_t per = ((p1 - p0 + kW - 1) / kW + 31) / 32 * 32;
     const int64_t q0 = min(p0 + w * per, p1), q1 = min(q0 + per, p1);
     bool bad = false;
-    auto load_key = [&](int64_t i) -> int { return i < q1 ? pair_key<kRankKeys>(a, i, bad) : -1; };
+    auto load_key = [&](int64_t i) -> int {
+        return i < q1 ? pair_key<kRankKeys>(a, i, bad, kRankKeys ? L.ehist : nullptr) : -1;
+    };
     auto count_round = [&](int key) {
         const uint32_t peers = __match_any_sync(0xffffffffu, key);
         if (key >= 0 && lane == __ffs(peers) - 1) my[key] += __popc(peers);
@@ -222,6 +290,10 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     for (int64_t qb = q0 + 32 * kKeyRounds; qb < q1; qb += 32) count_round(load_key(qb + lane));
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&a.hdr->pending, kDevBadExpert);
     __syncthreads();
+    if (kRankKeys && a.src_counts) {   // this chunk's expert counts, added before the barrier
+        for (int e = tid; e < a.src_E; e += NT)
+            if (L.ehist[e]) atomicAdd(&a.src_counts[e], L.ehist[e]);
+    }
     // chunk histogram; the per-warp counts become per-warp starting offsets
     for (int e = tid; e < Ep; e += NT) {
         int run = 0;
@@ -324,6 +396,14 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
             a.padpre[E] = total_pad;
             a.hdr->num_pad = total_pad;
         }
+        if (kRankKeys && a.src_counts) {   // every chunk's adds landed before the barrier
+            for (int e = tid; e < a.src_E; e += NT) {
+                const int32_t n = __ldcg(&a.src_counts[e]);
+                if (a.n_exp_out) a.n_exp_out[e] = n;
+                if (a.n_recv_out) a.n_recv_out[e] = align_up_i(n, a.src_A);
+                a.src_counts[e] = 0;   // ready for the next call; no other CTA reads it after the barrier
+            }
+        }
     }
     __syncthreads();
 
@@ -347,6 +427,7 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
                     a.recv_src[slot] = (int32_t)(i / K);
                     a.recv_w[slot] = a.topk_weights ? a.topk_weights[i] : 1.0f;
                     a.recv_lexp[slot] = key % El;
+                    if (kRankKeys) write_rank_row(a, i, slot);
                 }
             }
         };

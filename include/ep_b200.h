@@ -237,7 +237,9 @@ int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens
  * The handle works with ep_dispatch (rows per (token, rank)) and ep_combine
  * (§3.2 V1: topk_weights must be NULL; out[t] = the plain sum over the ranks
  * the token reached, in ascending rank order, plus the biases).  Device-side
- * errors as for ep_layout.  Two kernels.
+ * errors as for ep_layout.  One kernel; its workspace holds per-expert
+ * counters that the call leaves at zero (zero the workspace again after a
+ * EP_ERR_TIMEOUT).
  */
 size_t ep_rank_workspace_bytes(int num_tokens, int num_ranks, int num_experts);
 int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
