@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--fused", action="store_true",
                    help="the single ep_layout_dispatch call instead of ep_layout + ep_dispatch")
+    p.add_argument("--no-flush", dest="flush", action="store_false",
+                   help="no L2 flush between steps (each step's inputs, x and the expert outputs, exceed L2)")
     p.add_argument("--no-graph", dest="graph", action="store_false",
                    help="launch the calls of every step instead of replaying one captured CUDA graph")
     p.add_argument("--layout", default="expand", choices=["expand", "rank", "ll"],
@@ -315,7 +317,8 @@ def run_ours(args, rank, world, local_rank):
         time.sleep(0.3)
     wall0 = time.perf_counter()
     for i in range(args.steps):
-        flush.zero_()
+        if args.flush:
+            flush.zero_()
         evs[i][0].record(stream)
         run_step()
         evs[i][1].record(stream)
@@ -330,7 +333,8 @@ def run_ours(args, rank, world, local_rank):
     # per-kernel breakdown: the same K steps again with events between the kernels
     evk = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     for i in range(args.steps):
-        flush.zero_()
+        if args.flush:
+            flush.zero_()
         step(evk[i])
     torch.cuda.synchronize(dev)
     per = np.array([[evk[i][j].elapsed_time(evk[i][j + 1]) for j in range(3)] for i in range(args.steps)])
@@ -380,7 +384,9 @@ def run_ours(args, rank, world, local_rank):
             " layout=per-rank (one row per token and rank reached, unweighted combine)" if per_rank else
             (" layout=ll (fixed slab of R*%d rows per expert)" % M) if slab else ""),
             "global_batch": T * world, "parallelism": "replicas x%d (R=%d virtual ranks per GPU)" % (world, R),
-            "l2": "flushed by a 256 MiB write before every step, outside the timed events",
+            "l2": ("flushed by a 256 MiB write before every step, outside the timed events" if args.flush else
+                   "not flushed: the inputs each step reads (x and the expert-output rows, %.0f MB) exceed "
+                   "the 126 MB L2" % ((T + nbytes["Np"] - nbytes["pad_rows"]) * H * 2 / 1e6)),
             "launch": "one CUDA graph per step" if args.graph else "stream launches with programmatic dependent launch",
             "pairs": nbytes["N"], "recv_rows": nbytes["Np"], "pad_rows": nbytes["pad_rows"],
             "load": workload.load_stats(inp["topk_idx"], E)},
