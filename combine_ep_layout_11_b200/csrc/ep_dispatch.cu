@@ -227,7 +227,8 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
     uint8_t* out = smem + (size_t)stages * in_stride;
     uint64_t* full = reinterpret_cast<uint64_t*>(out + 2 * (size_t)out_stride);
     int32_t* slots = reinterpret_cast<int32_t*>(full + stages);
-    float* bmax = reinterpret_cast<float*>(slots + stages * 32);   // per-row scales: block maxima
+    int32_t* oslots = slots + stages * 32;                         // [2][32] slots of each output stage
+    float* bmax = reinterpret_cast<float*>(oslots + 2 * 32);        // per-row scales: block maxima
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t* sf = reinterpret_cast<uint8_t*>(a.recv_scales);
     const uint32_t sf_row_bytes = (uint32_t)ng * (uint32_t)elem;
@@ -301,8 +302,19 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
                 if (lane == 0) put_scale(dst_sf, b, sc, elem);
             }
         }
+        // column-major scales are stored by every warp below; they read the
+        // item's slots from oslots[o], a copy that the refill of input stage s
+        // cannot overwrite (it lives as long as output stage o)
+        if (a.sf_col_major && warp == 0 && lane < K) oslots[o * 32 + lane] = slots[s * 32 + lane];
         fence_proxy_async_smem();
         __syncthreads();
+        if (a.sf_col_major) {
+            for (int q = tid; q < K * ng; q += kCastThreads) {
+                const int k = q / ng, g = q - k * ng;
+                const int32_t slot = oslots[o * 32 + k];
+                if (slot >= 0 && (int64_t)slot < a.capacity) copy_scale(sf, sf_offset(a, slot, g), dst_sf, g, elem);
+            }
+        }
         if (warp == 0) {
             if (lane < K) {
                 const int32_t slot = slots[s * 32 + lane];
@@ -312,11 +324,7 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
                 }
             }
             if (a.sf_col_major) {
-                for (int k = 0; k < K; ++k) {
-                    const int32_t slot = slots[s * 32 + k];
-                    if (slot < 0 || (int64_t)slot >= a.capacity) continue;
-                    for (int g = lane; g < ng; g += 32) copy_scale(sf, sf_offset(a, slot, g), dst_sf, g, elem);
-                }
+                // stored by all warps above
             } else if (!bulk_scales) {
                 for (int q = lane; q < K * sf_words; q += 32) {
                     const int k = q / sf_words, wd = q - k * sf_words;
@@ -366,7 +374,7 @@ cudaError_t launch_cast_variant(const DispatchArgs& a, cudaStream_t s) {
     const uint32_t out_stride = round_up_u32((uint32_t)a.H + 4u * a.nb, 128);
     const int stages = 3;   // H <= 16384: at most 130 KB of stages
     const size_t smem = (size_t)stages * in_stride + 2 * (size_t)out_stride + (size_t)stages * 8 +
-                        (size_t)stages * 32 * 4 + (size_t)a.nb * 4;
+                        (size_t)stages * 32 * 4 + 2 * 32 * 4 + (size_t)a.nb * 4;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     int ctas_per_sm = 0;
