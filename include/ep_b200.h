@@ -23,13 +23,17 @@
  *                its handle serves ep_dispatch and §3.2's unweighted combine.
  *   ep_ll_layout §3.3 low_latency_dispatch: a fixed slab of R * max_tokens
  *                receive rows per expert.
+ *   ep_layout_dispatch  ep_layout and ep_dispatch in one call (§2.1: V2's
+ *                dispatch() derives its layout from topk_idx).
  * The placement also matches the last stages of the Ascend full-mesh dispatch
  * on the "URMA" tag page (count reconciliation, prefix-sum placement, reorder).
  *
  * Conventions for every entry point
  *   - Memory: every array is allocated by the caller; the library never
- *     allocates or frees memory and keeps no state between calls.  "device"
- *     means a pointer to memory of the current CUDA device.
+ *     allocates or frees memory and keeps no state between calls outside the
+ *     caller's workspace (the one exception, ep_layout_no_alloc, uses a fixed
+ *     array of the library's own).  "device" means a pointer to memory of the
+ *     current CUDA device.
  *   - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  *     Every call only enqueues work on that stream and returns; results are
  *     ready when the stream reaches them.  Nothing synchronises the host except
