@@ -44,6 +44,8 @@ def parse():
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="prefill_bf16", choices=sorted(workload.WORKLOADS))
+    p.add_argument("--tokens", type=int, default=None,
+                   help="override the workload's token count T (a multiple of its rank count)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -59,6 +61,16 @@ def parse():
                         "reached (ep_rank_layout) with V1's unweighted combine; ll: the low-latency fixed "
                         "slab of R * max_tokens rows per expert (ep_ll_layout)")
     return p.parse_args()
+
+
+def bench_config(args):
+    """The workload's configuration, with T overridden by --tokens."""
+    cfg = workload.config(args.workload)
+    if args.tokens is not None:
+        if args.tokens < 0 or args.tokens % cfg["R"]:
+            raise SystemExit("--tokens must be a non-negative multiple of R = %d" % cfg["R"])
+        cfg = dict(cfg, T=args.tokens)
+    return cfg
 
 
 def measured_peaks():
@@ -207,7 +219,7 @@ def run_ours(args, rank, world, local_rank):
         import datetime
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
 
-    cfg = workload.config(args.workload)
+    cfg = bench_config(args)
     inp = workload.inputs(cfg)
     T, H, K, E, R, A = cfg["T"], cfg["H"], cfg["K"], cfg["E"], cfg["R"], cfg["A"]
     idx = torch.from_numpy(inp["topk_idx"]).to(dev)
@@ -530,7 +542,7 @@ def cpu_baseline(cfg, inp, form="expand"):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    cfg = workload.config(args.workload)
+    cfg = bench_config(args)
     inp = workload.inputs(cfg)
     form = args.layout
     full = oracle_step_inputs(cfg, inp, form)
@@ -548,7 +560,8 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp8-e4m3/bf16" if cfg["fp8"] else "bf16",
             "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
-            "config": {"workload": cfg["name"] + ("" if form == "expand" else " layout=" + form),
+            "config": {"workload": cfg["name"] + ("" if args.tokens is None else " T=%d" % cfg["T"]) +
+                                   ("" if form == "expand" else " layout=" + form),
                        "global_batch": cfg["T"]},
             "impl": "reference",
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
