@@ -242,8 +242,9 @@ int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens
  * (§3.2 V1: topk_weights must be NULL; out[t] = the plain sum over the ranks
  * the token reached, in ascending rank order, plus the biases).  Device-side
  * errors as for ep_layout.  One kernel; its workspace holds per-expert
- * counters that the call leaves at zero (zero the workspace again after a
- * EP_ERR_TIMEOUT).
+ * counters that the call leaves at zero (zero the workspace again after an
+ * EP_ERR_TIMEOUT, and before reusing a workspace that served another layout
+ * call).
  */
 size_t ep_rank_workspace_bytes(int num_tokens, int num_ranks, int num_experts);
 int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
