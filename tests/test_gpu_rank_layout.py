@@ -160,3 +160,28 @@ def test_rank_layout_deterministic(ep):
         for a, b in zip(first, (lay.token_slot, lay.recv_topk_idx, lay.recv_topk_weights, lay.recv_src_token)):
             assert torch.equal(a.view(torch.uint8) if a.dtype == torch.float32 else a,
                                b.view(torch.uint8) if b.dtype == torch.float32 else b)
+
+
+@pytest.mark.parametrize("form", ["rank", "ll"])
+def test_fp8_input_passthrough_other_forms(ep, form):
+    """(e4m3 rows, fp32 scales) input is carried as is (§2.1: the received rows
+    have the input's type) on the per-rank and fixed-slab handles too."""
+    T, K, E, R, H = 96, 4, 32, 4, 512
+    rng = np.random.default_rng(71)
+    idx = rng.integers(-1, E, (T, K)).astype(np.int64)
+    x = workload.to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
+    q, s = oracle.cast_fp8(x)
+    dq = torch.from_numpy(q).to(DEV).view(torch.float8_e4m3fn)
+    ds = to_dev(s)
+    if form == "rank":
+        ref = oracle.rank_layout(idx, None, E, R)
+        lay = ep.rank_layout(to_dev(idx), None, E, R)
+    else:
+        ref = oracle.ll_layout(idx, None, E, R, T // R + 1)
+        lay = ep.ll_layout(to_dev(idx), None, E, R, T // R + 1)
+    rq, rs = ep.dispatch(lay, dq, x_scales=ds, do_zero_padding=True)
+    torch.cuda.synchronize()
+    assert ep.get_status(lay) == (ep.EP_OK, 0)
+    rows = int(ref["off"][-1])
+    assert np.array_equal(fp8_bits(rq[:rows]), oracle.dispatch_rows(q, ref, True)[:rows])
+    assert np.array_equal(f32_bits(rs[:rows]), oracle.dispatch_rows(s, ref, True)[:rows].view(np.uint32))
