@@ -306,3 +306,29 @@ def test_combine_second_bias_alone_rejected(ep):
     with pytest.raises(ep.EpError) as exc:
         ep.combine(lay, torch.zeros((64, 64), dtype=torch.bfloat16, device=DEV), bias=(None, b))
     assert exc.value.code == ep.EP_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("form", ["expand", "rank"])
+def test_layout_many_rounds_per_warp(ep, form):
+    """More than four rounds of 32 pairs per warp (over 2048 pairs per chunk at
+    the 128-chunk limit), so the assign pass reloads keys beyond the ones it
+    keeps in registers: 65536 tokens x top-8 (524 k pairs), skewed experts."""
+    cfg = dict(workload.config("prefill_bf16"), T=65536)
+    idx, w = workload.routing(cfg)
+    E, R, A = cfg["E"], cfg["R"], cfg["A"]
+    if form == "expand":
+        ref = oracle.layout(idx, w, E, R, A)
+        lay = ep.layout(to_dev(idx), to_dev(w), E, R, A)
+        torch.cuda.synchronize()
+        assert ep.get_status(lay) == (ep.EP_OK, 0)
+        check_layout(lay, ref)
+    else:
+        ref = oracle.rank_layout(idx, w, E, R, A)
+        lay = ep.rank_layout(to_dev(idx), to_dev(w), E, R, A)
+        torch.cuda.synchronize()
+        assert ep.get_status(lay) == (ep.EP_OK, 0)
+        rows = int(ref["rank_off"][-1])
+        assert np.array_equal(lay.token_slot.cpu().numpy(), ref["token_slot"])
+        assert np.array_equal(lay.recv_src_token[:rows].cpu().numpy(), ref["recv_src"][:rows])
+        assert np.array_equal(lay.recv_topk_idx[:rows].cpu().numpy(), ref["recv_topk_idx"][:rows])
+        assert np.array_equal(lay.num_tokens_per_expert.cpu().numpy(), ref["num_tokens_per_expert"])
