@@ -332,3 +332,18 @@ def test_layout_many_rounds_per_warp(ep, form):
         assert np.array_equal(lay.recv_src_token[:rows].cpu().numpy(), ref["recv_src"][:rows])
         assert np.array_equal(lay.recv_topk_idx[:rows].cpu().numpy(), ref["recv_topk_idx"][:rows])
         assert np.array_equal(lay.num_tokens_per_expert.cpu().numpy(), ref["num_tokens_per_expert"])
+
+
+def test_fused_layout_dispatch_many_rounds(ep):
+    """ep_layout_dispatch (one CTA per SM) at 65536 tokens x top-8: about 220
+    pairs per warp, so its layout pass reloads keys too; 512-byte rows."""
+    cfg = dict(workload.config("prefill_bf16"), T=65536, H=256)
+    idx, w = workload.routing(cfg)
+    x = workload.tokens(cfg)
+    E, R, A = cfg["E"], cfg["R"], cfg["A"]
+    ref = oracle.layout(idx, w, E, R, A)
+    lay, recv = ep.layout_dispatch(to_dev(idx), to_dev(w), to_dev_bf16(x), E, R, A, do_zero_padding=True)
+    torch.cuda.synchronize()
+    assert ep.get_status(lay) == (ep.EP_OK, 0)
+    Np = check_layout(lay, ref)
+    assert np.array_equal(bf16_bits(recv[:Np]), oracle.dispatch_rows(x, ref, True)[:Np])
