@@ -420,7 +420,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": ncu_traffic(top_kernel, cfg["name"] + ("" if args.layout == "expand"
                                                                        else "/" + args.layout)),
                      "algorithmic_bytes_per_launch": top_bytes},
-        "gpu_launches": args.steps * (4 if per_rank else (2 if (args.fused and not fp8) else 3)),
+        "gpu_launches": args.steps * (2 if (args.fused and not fp8) else 3),
         "wall_s_timed_region": round(wall, 4),
     }
     if clock_info:
