@@ -628,6 +628,26 @@ def pin_rank_layout_vs_numpy(n=120, seed=37):
                               exp["recv_topk_weights"].view(np.uint32))
 
 
+def pin_rank_layout_exhaustive():
+    """Every topk_idx with T*K <= 4 entries in {-1, 0..E-1}, E in {2, 4}, R in {1, 2, 4},
+    against the numpy restatement."""
+    for E in (2, 4):
+        for (T, K) in [(1, 1), (2, 1), (2, 2), (4, 1), (1, 3), (1, 4)]:
+            for R in (1, 2, 4):
+                if E % R or T % R:
+                    continue
+                for vals in itertools.product(range(-1, E), repeat=T * K):
+                    idx = np.array(vals, np.int64).reshape(T, K)
+                    got = oracle.rank_layout(idx, None, E, R, 2)
+                    exp = _rank_layout_numpy(idx, None, E, R, 2)
+                    rows = int(exp["rank_off"][-1])
+                    for key in ("is_token_in_rank", "num_tokens_per_rank", "rank_off", "token_slot",
+                                "num_tokens_per_expert", "num_recv_tokens_per_expert"):
+                        assert np.array_equal(got[key], exp[key]), (key, idx.tolist(), R)
+                    assert np.array_equal(got["recv_src"][:rows], exp["recv_src"])
+                    assert np.array_equal(got["recv_topk_idx"][:rows], exp["recv_topk_idx"])
+
+
 def pin_rank_layout_golden():
     g = _golden("rank_layout_example.json")
     d = oracle.rank_layout(np.array(g["topk_idx"], np.int64), np.array(g["topk_weights"], np.float32),
@@ -734,6 +754,7 @@ ALL_PINS = [
     pin_combine_permutation, pin_recv_stats,
     pin_cast_variants_vs_torch, pin_round_scale_properties, pin_fp8_variants_golden, pin_ue8m0,
     pin_cast_variants_roundtrip, pin_scales_col_major,
-    pin_rank_layout_vs_numpy, pin_rank_layout_golden, pin_rank_layout_matches_expand, pin_rank_combine_identity,
+    pin_rank_layout_vs_numpy, pin_rank_layout_exhaustive, pin_rank_layout_golden, pin_rank_layout_matches_expand,
+    pin_rank_combine_identity,
     pin_ll_layout_golden, pin_ll_layout_vs_expand,
 ]

@@ -8,6 +8,10 @@ def test_rank_layout_vs_numpy_formulation():
     pins.pin_rank_layout_vs_numpy()
 
 
+def test_rank_layout_exhaustive_small():
+    pins.pin_rank_layout_exhaustive()
+
+
 def test_rank_layout_hand_derived():
     pins.pin_rank_layout_golden()
 
