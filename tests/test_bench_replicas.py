@@ -75,3 +75,33 @@ def test_reference_arm_under_torchrun_prints_one_line():
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["n_gpus"] == 2 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_algorithmic_bytes_accounting():
+    """The bytes the roofline divides by, from the definitions: dispatch reads
+    each token row once and writes every receive row (pairs and, with zero
+    padding, the padding rows) plus the pair slots; combine reads one row per
+    pair, writes one row per token and reads the slots and weights."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    import workload
+    cfg = workload.config("prefill_bf16")
+    T, H, K, E, A = cfg["T"], cfg["H"], cfg["K"], cfg["E"], cfg["A"]
+    cnt = np.full(E, 128, np.int64)
+    cnt[:3] = [1, 129, 0]
+    N = int(cnt.sum())
+    Np = int(((cnt + A - 1) // A * A).sum())
+    b = bench.algorithmic_bytes(cfg, cnt, A)
+    assert (b["N"], b["Np"], b["pad_rows"]) == (N, Np, Np - N)
+    assert b["dispatch"] == T * 2 * H + Np * 2 * H + T * K * 4
+    assert b["combine"] == N * 2 * H + T * 2 * H + T * K * 8
+    fp8 = dict(cfg, fp8=True)
+    assert bench.algorithmic_bytes(fp8, cnt, A)["dispatch"] == T * 2 * H + Np * (H + 4 * H // 128) + T * K * 4
+    nopad = dict(cfg, zero_pad=False)
+    assert bench.algorithmic_bytes(nopad, cnt, A)["dispatch"] == T * 2 * H + N * 2 * H + T * K * 4
+    slab = bench.algorithmic_bytes(nopad, cnt, 1, slab=4096)
+    assert slab["Np"] == E * 4096 and slab["dispatch"] == T * 2 * H + N * 2 * H + T * K * 4
+    rank = bench.algorithmic_bytes_rank(cfg, rows=20000, N=N)
+    assert rank["dispatch"] == T * 2 * H + 20000 * 2 * H + T * cfg["R"] * 4
+    assert rank["combine"] == 20000 * 2 * H + T * 2 * H + T * cfg["R"] * 4
