@@ -70,6 +70,61 @@ def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+# The library sees only pointers, so the binding checks what a pointer cannot
+# carry before it crosses: the tensor's device, dtype, shape and density, and
+# that an output is large enough for every row the kernels may write.  A
+# failed check raises the same EpError(EP_ERR_INVALID_ARG) a rejected call
+# does, and nothing is enqueued.
+def _require(ok, what):
+    if not ok:
+        raise EpError(EP_ERR_INVALID_ARG, what)
+
+
+def _handle_device(device):
+    """torch.device with the index filled in ('cuda' -> the current CUDA device)."""
+    dev = torch.device(device)
+    if dev.type == "cuda" and dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    return dev
+
+
+def _check_tensor(t, what, device, dtype=None, shape=None, dense=True):
+    _require(isinstance(t, torch.Tensor), "%s must be a tensor" % what)
+    _require(t.device.type == "cuda" and t.device == device,
+             "%s must be a CUDA tensor on %s, not on %s" % (what, device, t.device))
+    if dtype is not None:
+        _require(t.dtype == dtype, "%s must be %s, not %s" % (what, dtype, t.dtype))
+    if shape is not None:
+        _require(tuple(t.shape) == tuple(shape), "%s must have shape %s, not %s" % (what, tuple(shape), tuple(t.shape)))
+    if dense:
+        _require(t.is_contiguous(), "%s must be contiguous" % what)
+
+
+def _bytes_from_start(t):
+    """Bytes of t's storage from its first element on: all a kernel given t.data_ptr() may reach."""
+    return t.untyped_storage().nbytes() - t.storage_offset() * t.element_size()
+
+
+def _check_routing(topk_idx, topk_weights):
+    """topk_idx int64 [T, K] on a CUDA device; topk_weights None or fp32 [T, K] beside it."""
+    _require(isinstance(topk_idx, torch.Tensor) and topk_idx.dim() == 2, "topk_idx must be a [T, K] tensor")
+    _check_tensor(topk_idx, "topk_idx", topk_idx.device, torch.int64)
+    if topk_weights is not None:
+        _check_tensor(topk_weights, "topk_weights", topk_idx.device, torch.float32, topk_idx.shape)
+    return topk_idx.shape
+
+
+def _check_scales_out(out_scales, rows, hidden, fmt, device):
+    """A caller's scale array: on the device, of the format's element type, and
+    holding ep_scale_bytes(rows, hidden, fmt) bytes from its first element."""
+    nbytes = int(_lib.load().ep_scale_bytes(rows, hidden, fmt))
+    _require(nbytes >= 0, "scale format")
+    dtype = torch.uint8 if fmt & EP_SF_UE8M0 else torch.float32
+    _check_tensor(out_scales, "out_scales", device, dtype, dense=False)
+    _require(_bytes_from_start(out_scales) >= nbytes,
+             "out_scales holds %d bytes, the format needs %d" % (_bytes_from_start(out_scales), nbytes))
+
+
 def workspace_bytes(num_tokens, num_topk, num_experts, expert_alignment):
     return int(_lib.load().ep_workspace_bytes(num_tokens, num_topk, num_experts, expert_alignment))
 
@@ -92,7 +147,7 @@ class Layout:
         T, K, E, A = num_tokens, num_topk, num_experts, expert_alignment
         if capacity is None:
             capacity = capacity_rows(T, K, E, A)
-        dev = torch.device(device)
+        dev = _handle_device(device)
         i32 = dict(dtype=torch.int32, device=dev)
         self.num_tokens, self.num_topk, self.num_experts = T, K, E
         self.num_ranks, self.expert_alignment = num_ranks, A
@@ -141,8 +196,7 @@ class Layout:
 def _set_recv_stats(lay, stats):
     """Point the handle at the caller's running per-expert receive counts (or at none)."""
     if stats is not None:
-        assert stats.dtype == torch.int32 and stats.is_contiguous() and stats.numel() == lay.num_experts
-        assert stats.device == lay.device
+        _check_tensor(stats, "cumulative_local_expert_recv_stats", lay.device, torch.int32, (lay.num_experts,))
     lay.cumulative_local_expert_recv_stats = stats       # kept alive with the handle
     lay.struct.cumulative_local_expert_recv_stats = _ptr(stats)
 
@@ -156,13 +210,10 @@ def layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment=1,
     when given, this call's per-expert receive counts are added to it (§2.1).
     """
     L = _lib.load()
-    assert topk_idx.dtype == torch.int64 and topk_idx.dim() == 2 and topk_idx.is_contiguous()
-    T, K = topk_idx.shape
-    if topk_weights is not None:
-        assert topk_weights.dtype == torch.float32 and topk_weights.shape == (T, K)
-        assert topk_weights.is_contiguous()
+    T, K = _check_routing(topk_idx, topk_weights)
     if out is not None:
-        assert (out.num_tokens, out.num_topk, out.num_experts) == (T, K, num_experts), "layout size mismatch"
+        _require((out.num_tokens, out.num_topk, out.num_experts) == (T, K, num_experts), "layout size mismatch")
+        _require(out.device == topk_idx.device, "the layout handle is on another device")
     lay = out if out is not None else Layout(T, K, num_experts, num_ranks, expert_alignment,
                                              topk_idx.device, capacity, num_max_tokens_per_rank)
     _set_recv_stats(lay, cumulative_local_expert_recv_stats)
@@ -179,12 +230,8 @@ def ll_layout(topk_idx, topk_weights, num_experts, num_ranks, num_max_dispatch_t
     pairs first (token-major, k-minor), the rest padding.  Returns a ``Layout``
     (capacity E*S) usable by ``dispatch`` and ``combine``."""
     L = _lib.load()
-    assert topk_idx.dtype == torch.int64 and topk_idx.dim() == 2 and topk_idx.is_contiguous()
-    T, K = topk_idx.shape
+    T, K = _check_routing(topk_idx, topk_weights)
     E, R, M = num_experts, num_ranks, num_max_dispatch_tokens_per_rank
-    if topk_weights is not None:
-        assert topk_weights.dtype == torch.float32 and topk_weights.shape == (T, K)
-        assert topk_weights.is_contiguous()
     if out is None:
         nbytes = int(L.ep_ll_workspace_bytes(T, K, E, R, M))
         if nbytes == 0:
@@ -192,7 +239,8 @@ def ll_layout(topk_idx, topk_weights, num_experts, num_ranks, num_max_dispatch_t
         out = Layout(T, K, E, R, 1, topk_idx.device, capacity=E * R * M, num_max_tokens_per_rank=M,
                      workspace_nbytes=nbytes)
     else:
-        assert (out.num_tokens, out.num_topk, out.num_experts) == (T, K, E), "layout size mismatch"
+        _require((out.num_tokens, out.num_topk, out.num_experts) == (T, K, E), "layout size mismatch")
+        _require(out.device == topk_idx.device, "the layout handle is on another device")
     _set_recv_stats(out, cumulative_local_expert_recv_stats)
     _check(L.ep_ll_layout(_ptr(topk_idx), _ptr(topk_weights), T, K, E, R, M, out.ref(), _stream(topk_idx.device)),
            "ep_ll_layout")
@@ -216,7 +264,7 @@ class RankLayout:
         T, K, E, R = num_tokens, num_topk, num_experts, num_ranks
         if capacity is None:
             capacity = T * R
-        dev = torch.device(device)
+        dev = _handle_device(device)
         i32 = dict(dtype=torch.int32, device=dev)
         self.num_tokens, self.num_topk, self.num_experts, self.num_ranks = T, K, E, R
         self.expert_alignment = expert_alignment
@@ -261,13 +309,11 @@ def rank_layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment
     receive form; §3.1 num_tokens_per_rank / is_token_in_rank /
     num_tokens_per_expert).  ``out`` may be a ``RankLayout`` of the same sizes."""
     L = _lib.load()
-    assert topk_idx.dtype == torch.int64 and topk_idx.dim() == 2 and topk_idx.is_contiguous()
-    T, K = topk_idx.shape
-    if topk_weights is not None:
-        assert topk_weights.dtype == torch.float32 and topk_weights.shape == (T, K)
-        assert topk_weights.is_contiguous()
+    T, K = _check_routing(topk_idx, topk_weights)
     if out is not None:
-        assert (out.num_tokens, out.num_topk, out.num_experts, out.num_ranks) == (T, K, num_experts, num_ranks)
+        _require((out.num_tokens, out.num_topk, out.num_experts, out.num_ranks) == (T, K, num_experts, num_ranks),
+                 "layout size mismatch")
+        _require(out.device == topk_idx.device, "the layout handle is on another device")
     lay = out if out is not None else RankLayout(T, K, num_experts, num_ranks, expert_alignment,
                                                  topk_idx.device, capacity)
     lay.expert_alignment = expert_alignment
@@ -276,6 +322,35 @@ def rank_layout(topk_idx, topk_weights, num_experts, num_ranks, expert_alignment
                             _ptr(lay.num_recv_tokens_per_expert), _ptr(lay.recv_topk_idx),
                             _ptr(lay.recv_topk_weights), lay.ref(), _stream(topk_idx.device)), "ep_rank_layout")
     return lay
+
+
+def _dispatch_buffers(lay, x, x_scales, cast_to_fp8, out, out_scales, scale_fmt):
+    """Check dispatch's tensors against the handle and allocate the outputs
+    not given; returns (H, fp8_in, fp8_out, recv_x, recv_scales)."""
+    dev, T = lay.device, lay.num_tokens
+    _require(isinstance(x, torch.Tensor) and x.dim() == 2 and x.shape[0] == T, "x must be a [T, H] tensor")
+    _check_tensor(x, "x", dev)
+    H = x.shape[1]
+    fp8_in = x.dtype == torch.float8_e4m3fn
+    _require(fp8_in or x.dtype == torch.bfloat16, "x must be bfloat16 or float8_e4m3fn, not %s" % x.dtype)
+    if fp8_in:
+        _require(x_scales is not None, "FP8 input needs x_scales")
+        _check_tensor(x_scales, "x_scales", dev, torch.float32, (T, H // 128))
+    fp8_out = fp8_in or bool(cast_to_fp8)
+    out_dtype = torch.float8_e4m3fn if fp8_out else torch.bfloat16
+    cap = max(lay.capacity, 1)
+    if out is None:
+        out = torch.empty((cap, H), dtype=out_dtype, device=dev)
+    else:
+        _check_tensor(out, "out", dev, out_dtype)
+        _require(out.dim() == 2 and out.shape[1] == H and out.shape[0] >= lay.capacity,
+                 "out must be [rows >= capacity %d, H %d], not %s" % (lay.capacity, H, tuple(out.shape)))
+    if fp8_out:
+        if out_scales is None:
+            out_scales = scale_tensor(cap, H, scale_fmt, dev)
+        else:
+            _check_scales_out(out_scales, lay.capacity, H, scale_fmt, dev)
+    return H, fp8_in, fp8_out, out, out_scales
 
 
 def dispatch(lay, x, x_scales=None, cast_to_fp8=False, do_zero_padding=False, out=None, out_scales=None,
@@ -289,16 +364,7 @@ def dispatch(lay, x, x_scales=None, cast_to_fp8=False, do_zero_padding=False, ou
     ``scale_format()``, asks for another form of the cast's scales).
     """
     L = _lib.load()
-    assert x.dim() == 2 and x.is_contiguous() and x.shape[0] == lay.num_tokens
-    H = x.shape[1]
-    fp8_in = x.dtype == torch.float8_e4m3fn
-    assert fp8_in or x.dtype == torch.bfloat16
-    fp8_out = fp8_in or cast_to_fp8
-    cap = max(lay.capacity, 1)
-    if out is None:
-        out = torch.empty((cap, H), dtype=torch.float8_e4m3fn if fp8_out else torch.bfloat16, device=x.device)
-    if fp8_out and out_scales is None:
-        out_scales = scale_tensor(cap, H, scale_fmt, x.device)
+    H, fp8_in, fp8_out, out, out_scales = _dispatch_buffers(lay, x, x_scales, cast_to_fp8, out, out_scales, scale_fmt)
     _check(L.ep_dispatch(lay.ref(), _ptr(x), EP_DTYPE_FP8_E4M3 if fp8_in else EP_DTYPE_BF16,
                          _ptr(x_scales if fp8_in else None), H, int(bool(cast_to_fp8)), int(scale_fmt),
                          int(bool(do_zero_padding)), _ptr(out), _ptr(out_scales if fp8_out else None),
@@ -314,26 +380,15 @@ def layout_dispatch(topk_idx, topk_weights, x, num_experts, num_ranks, expert_al
     from topk_idx).  Same results as ``layout`` then ``dispatch``; returns
     ``(layout, recv_x)`` or ``(layout, (recv_x, recv_scales))`` for FP8 output."""
     L = _lib.load()
-    assert topk_idx.dtype == torch.int64 and topk_idx.dim() == 2 and topk_idx.is_contiguous()
-    T, K = topk_idx.shape
-    if topk_weights is not None:
-        assert topk_weights.dtype == torch.float32 and topk_weights.shape == (T, K)
-        assert topk_weights.is_contiguous()
-    assert x.dim() == 2 and x.is_contiguous() and x.shape[0] == T
+    T, K = _check_routing(topk_idx, topk_weights)
     if out_layout is not None:
-        assert (out_layout.num_tokens, out_layout.num_topk, out_layout.num_experts) == (T, K, num_experts)
+        _require((out_layout.num_tokens, out_layout.num_topk, out_layout.num_experts) == (T, K, num_experts),
+                 "layout size mismatch")
+        _require(out_layout.device == topk_idx.device, "the layout handle is on another device")
     lay = out_layout if out_layout is not None else Layout(T, K, num_experts, num_ranks, expert_alignment,
                                                            topk_idx.device, capacity, num_max_tokens_per_rank)
     _set_recv_stats(lay, cumulative_local_expert_recv_stats)
-    H = x.shape[1]
-    fp8_in = x.dtype == torch.float8_e4m3fn
-    assert fp8_in or x.dtype == torch.bfloat16
-    fp8_out = fp8_in or cast_to_fp8
-    cap = max(lay.capacity, 1)
-    if out is None:
-        out = torch.empty((cap, H), dtype=torch.float8_e4m3fn if fp8_out else torch.bfloat16, device=x.device)
-    if fp8_out and out_scales is None:
-        out_scales = scale_tensor(cap, H, scale_fmt, x.device)
+    H, fp8_in, fp8_out, out, out_scales = _dispatch_buffers(lay, x, x_scales, cast_to_fp8, out, out_scales, scale_fmt)
     _check(L.ep_layout_dispatch(_ptr(topk_idx), _ptr(topk_weights), T, K, num_experts, num_ranks,
                                 expert_alignment, num_max_tokens_per_rank, lay.ref(), _ptr(x),
                                 EP_DTYPE_FP8_E4M3 if fp8_in else EP_DTYPE_BF16, _ptr(x_scales if fp8_in else None),
@@ -349,24 +404,28 @@ def combine(lay, y, topk_weights=None, bias=None, out=None):
     0, 1 or 2 output biases); the fp32 sum starts from bias0 (+ bias1).
     """
     L = _lib.load()
-    assert y.dtype == torch.bfloat16 and y.dim() == 2 and y.is_contiguous()
-    H = y.shape[1]
-    if topk_weights is not None:
-        assert topk_weights.dtype == torch.float32 and topk_weights.is_contiguous()
+    dev, T = lay.device, lay.num_tokens
     if bias is None:
         biases = (None, None)
     elif isinstance(bias, torch.Tensor):
         biases = (bias, None)
     else:
-        assert len(bias) == 2, "bias is a tensor or a pair of tensors"
         biases = tuple(bias)
+        _require(len(biases) == 2, "bias is a tensor or a pair of tensors")
+    _require(isinstance(y, torch.Tensor) and y.dim() == 2, "y must be a [rows, H] tensor")
+    _check_tensor(y, "y", dev, torch.bfloat16)
+    H = y.shape[1]
+    if topk_weights is not None:
+        _check_tensor(topk_weights, "topk_weights", dev, torch.float32, (T, lay.num_topk))
     for b in biases:
         if b is not None:
-            assert b.dtype == torch.bfloat16 and b.is_contiguous() and b.shape == (lay.num_tokens, H)
+            _check_tensor(b, "bias", dev, torch.bfloat16, (T, H))
     if out is None:
-        out = torch.empty((lay.num_tokens, H), dtype=torch.bfloat16, device=y.device)
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    else:
+        _check_tensor(out, "out", dev, torch.bfloat16, (T, H))
     _check(L.ep_combine(lay.ref(), _ptr(y), H, _ptr(topk_weights), _ptr(biases[0]), _ptr(biases[1]),
-                        _ptr(out), _stream(y.device)), "ep_combine")
+                        _ptr(out), _stream(dev)), "ep_combine")
     return out
 
 
@@ -374,12 +433,17 @@ def cast_fp8(x, out=None, out_scales=None, scale_fmt=0):
     """bf16 [T, H] -> (float8_e4m3fn [T, H], scales [T, groups]) (§4.2); fp32
     scales per 128-column block unless ``scale_fmt`` (EP_SF_* bits) says otherwise."""
     L = _lib.load()
-    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+    _require(isinstance(x, torch.Tensor) and x.dim() == 2, "x must be a [T, H] tensor")
+    _check_tensor(x, "x", x.device, torch.bfloat16)
     T, H = x.shape
     if out is None:
         out = torch.empty((T, H), dtype=torch.float8_e4m3fn, device=x.device)
+    else:
+        _check_tensor(out, "out", x.device, torch.float8_e4m3fn, (T, H))
     if out_scales is None:
         out_scales = scale_tensor(T, H, scale_fmt, x.device)
+    else:
+        _check_scales_out(out_scales, T, H, scale_fmt, x.device)
     _check(L.ep_cast_fp8(_ptr(x), T, H, int(scale_fmt), _ptr(out), _ptr(out_scales), _stream(x.device)),
            "ep_cast_fp8")
     return out, out_scales
