@@ -202,6 +202,21 @@ def algorithmic_bytes_rank(cfg, rows, N):
     return dict(layout=layout_b, dispatch=dispatch_b, combine=combine_b, N=N, Np=rows, pad_rows=0)
 
 
+def workload_config(cfg, form, world, nbytes, topk_idx):
+    """The `config` keys that name the workload; both arms print them, so the
+    reference line describes exactly the work of ours."""
+    T, H, E, K, R, A = (cfg[k] for k in ("T", "H", "E", "K", "R", "A"))
+    M = cfg["max_tokens_per_rank"] or T // R
+    shape = {"expand": "",
+             "rank": " layout=per-rank (one row per token and rank reached, unweighted combine)",
+             "ll": " layout=ll (fixed slab of R*%d rows per expert)" % M}[form]
+    return {"workload": "%s: T=%d H=%d E=%d top-%d R=%d align=%d zero_pad=%s%s%s" % (
+                cfg["name"], T, H, E, K, R, A, cfg["zero_pad"], " fp8-cast" if cfg["fp8"] else "", shape),
+            "global_batch": T * world, "parallelism": "replicas x%d (R=%d virtual ranks per GPU)" % (world, R),
+            "pairs": nbytes["N"], "recv_rows": nbytes["Np"], "pad_rows": nbytes["pad_rows"],
+            "load": workload.load_stats(topk_idx, E)}
+
+
 # --------------------------------------------------------------------------
 # our implementation
 # --------------------------------------------------------------------------
@@ -391,17 +406,12 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "fp8-e4m3/bf16" if fp8 else "bf16",
         "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
-        "config": {"workload": "%s: T=%d H=%d E=%d top-%d R=%d align=%d zero_pad=%s%s%s" % (
-            cfg["name"], T, H, E, K, R, A, cfg["zero_pad"], " fp8-cast" if fp8 else "",
-            " layout=per-rank (one row per token and rank reached, unweighted combine)" if per_rank else
-            (" layout=ll (fixed slab of R*%d rows per expert)" % M) if slab else ""),
-            "global_batch": T * world, "parallelism": "replicas x%d (R=%d virtual ranks per GPU)" % (world, R),
-            "l2": ("flushed by a 256 MiB write before every step, outside the timed events" if args.flush else
-                   "not flushed: the inputs each step reads (x and the expert-output rows, %.0f MB) exceed "
-                   "the 126 MB L2" % ((T + nbytes["Np"] - nbytes["pad_rows"]) * H * 2 / 1e6)),
-            "launch": "one CUDA graph per step" if args.graph else "stream launches with programmatic dependent launch",
-            "pairs": nbytes["N"], "recv_rows": nbytes["Np"], "pad_rows": nbytes["pad_rows"],
-            "load": workload.load_stats(inp["topk_idx"], E)},
+        "config": dict(
+            workload_config(cfg, args.layout, world, nbytes, inp["topk_idx"]),
+            l2=("flushed by a 256 MiB write before every step, outside the timed events" if args.flush else
+                "not flushed: the inputs each step reads (x and the expert-output rows, %.0f MB) exceed "
+                "the 126 MB L2" % ((T + nbytes["Np"] - nbytes["pad_rows"]) * H * 2 / 1e6)),
+            launch="one CUDA graph per step" if args.graph else "stream launches with programmatic dependent launch"),
         "ms_per_step_median": round(ms_median, 5),
         # the count_bytes convention: one row copy in dispatch and one row read in
         # combine per receive row that holds data
@@ -547,6 +557,14 @@ def run_reference(args, rank, world):
     form = args.layout
     full = oracle_step_inputs(cfg, inp, form)
     import oracle
+    olay = oracle.step_layout(inp, cfg, form)
+    if form == "rank":
+        nbytes = algorithmic_bytes_rank(cfg, int(olay["off"][-1]), int((inp["topk_idx"] >= 0).sum()))
+    elif form == "ll":
+        nbytes = algorithmic_bytes(cfg, olay["cnt"], 1, slab=cfg["R"] * (cfg["max_tokens_per_rank"] or
+                                                                       cfg["T"] // cfg["R"]))
+    else:
+        nbytes = algorithmic_bytes(cfg, olay["cnt"], cfg["A"])
     for _ in range(args.warmup):
         oracle.step(full, cfg, form)
     ts = []
@@ -560,9 +578,8 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp8-e4m3/bf16" if cfg["fp8"] else "bf16",
             "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
-            "config": {"workload": cfg["name"] + ("" if args.tokens is None else " T=%d" % cfg["T"]) +
-                                   ("" if form == "expand" else " layout=" + form),
-                       "global_batch": cfg["T"]},
+            "config": dict(workload_config(cfg, form, world, nbytes, inp["topk_idx"]),
+                           l2="not applicable: the oracle runs on the host cores"),
             "impl": "reference",
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": "the full %s workload per step (single-threaded C oracle)" % cfg["name"]},

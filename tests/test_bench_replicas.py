@@ -105,3 +105,28 @@ def test_algorithmic_bytes_accounting():
     rank = bench.algorithmic_bytes_rank(cfg, rows=20000, N=N)
     assert rank["dispatch"] == T * 2 * H + 20000 * 2 * H + T * cfg["R"] * 4
     assert rank["combine"] == 20000 * 2 * H + T * 2 * H + T * cfg["R"] * 4
+
+
+@pytest.mark.parametrize("form", ["expand", "rank", "ll"])
+def test_reference_line_names_our_workload(form):
+    """The reference arm prints the workload keys of `config` from the same
+    function as our arm, with the oracle's own pair and receive-row counts."""
+    import argparse
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    import oracle
+    import workload
+    args = argparse.Namespace(workload="tiny", tokens=None, layout=form, steps=1, warmup=0)
+    line = bench.run_reference(args, 0, 1)
+    cfg = workload.config("tiny")
+    inp = workload.inputs(cfg)
+    lay = oracle.step_layout(inp, cfg, form)
+    c = line["config"]
+    assert line["impl"] == "reference" and c["workload"].startswith("tiny: T=128 H=256 E=16 top-4 R=2")
+    assert c["pairs"] == int((inp["topk_idx"] >= 0).sum())
+    assert c["recv_rows"] == int(lay["off"][-1])
+    expect = bench.workload_config(cfg, form, 1, {"N": c["pairs"], "Np": c["recv_rows"], "pad_rows": c["pad_rows"]},
+                                   inp["topk_idx"])
+    assert {k: c[k] for k in expect} == expect
+    assert np.isfinite(line["value"]) and line["value"] > 0
