@@ -251,3 +251,25 @@ def test_c_client_builds_and_links(lib, tmp_path):
          "tests/c_abi_client.c", "-o", str(exe), "-L", os.path.dirname(build.LIB), "-lep_b200",
          "-L", "/usr/local/cuda/lib64", "-lcudart"], tmp_path)
     assert exe.exists()
+
+
+def test_oracle_and_kernels_share_no_code():
+    """The oracle is built from its own C file with system headers only and
+    imports nothing of the package; the kernels include nothing of the oracle.
+    The only module both sides use is workload/ (seeded inputs)."""
+    import re
+    odir = os.path.join(ROOT, "oracle")
+    for fn in os.listdir(odir):
+        if not fn.endswith((".c", ".h", ".py")):
+            continue
+        src = open(os.path.join(odir, fn)).read()
+        assert not re.search(r"^\s*(import|from)\s+combine_ep_layout_11_b200", src, re.M), fn
+        for inc in re.findall(r'#include\s*([<"][^>"]+[>"])', src):
+            assert inc.startswith("<"), (fn, inc)              # system headers only
+    build_src = open(os.path.join(odir, "build.py")).read()
+    assert "csrc" not in build_src and "include" not in build_src   # no -I into the kernels' headers
+    cdir = os.path.join(ROOT, "combine_ep_layout_11_b200", "csrc")
+    for fn in os.listdir(cdir):
+        src = open(os.path.join(cdir, fn)).read()
+        for inc in re.findall(r'#include\s*"([^"]+)"', src):
+            assert inc == "ep_b200.h" or os.path.exists(os.path.join(cdir, inc)), (fn, inc)
