@@ -84,6 +84,19 @@ MUTANTS = {
     "routing_start_exclusive": ("if (e >= local_start && e < local_end)",
                                 "if (e > local_start && e < local_end)"),
     "dispatch_no_zero_padding": ("if (do_zero_padding)\n        for", "if (0)\n        for"),
+    "dispatch_previous_token_row": ("x + t * row_bytes, (size_t)row_bytes);",
+                                    "x + (t > 0 ? t - 1 : 0) * row_bytes, (size_t)row_bytes);"),
+    "dequant_divides": ("out[t * H + j] = v * s;", "out[t * H + j] = v / s;"),
+    "dequant_first_block_scale": ("float s = scales[t * ng + j / group];", "float s = scales[t * ng];"),
+    "ue8m0_decode_off_by_one": ("out[i] = ldexpf(1.0f, (int)b[i] - 127);", "out[i] = ldexpf(1.0f, (int)b[i] - 126);"),
+    "e4m3_subnormal_exponent": ("return ldexp((double)m / 8.0, -6);", "return ldexp((double)m / 8.0, -7);"),
+    "e4m3_saturates_to_nan": ("return (uint8_t)(sign | 0x7e);\n    /* largest", "return (uint8_t)(sign | 0x7f);\n    /* largest"),
+    "cast_amax_clamp_1e-3": ("if (amax < 1e-4f)\n                amax = 1e-4f;", "if (amax < 1e-3f)\n                amax = 1e-3f;"),
+    "layout_accepts_minus_two": (
+        "an expert id in [0, E) */\n    for (int64_t i = 0; i < T * K; i++)\n        if (topk_idx[i] < -1 ||",
+        "an expert id in [0, E) */\n    for (int64_t i = 0; i < T * K; i++)\n        if (topk_idx[i] < -2 ||"),
+    "routing_end_inclusive": ("if (e >= local_start && e < local_end)", "if (e >= local_start && e <= local_end)"),
+    "stats_added_twice": ("stats[e] += cnt[e];", "stats[e] += 2 * cnt[e];"),
 }
 
 
