@@ -1,12 +1,14 @@
 """Planted mistakes in the oracle must each fail at least one pin.
 
-Each case below makes one or more edits to a copy of ``oracle/ep_oracle.c`` (the committed source is
+Each C case below makes one or more edits to a copy of ``oracle/ep_oracle.c`` (the committed source is
 never touched), builds it into a temporary library, routes the oracle through it
-and runs the pins until one fails.  A mistake that no pin catches means a pin is
+and runs the pins until one fails; each Python case swaps a faulty version in
+for one of the oracle's own Python functions.  A mistake that no pin catches means a pin is
 missing.  Mistakes that would write out of bounds in the mutated C code are not
 planted.
 """
 
+import numpy as np
 import pytest
 
 import oracle
@@ -136,3 +138,44 @@ def test_pins_catch_planted_mistake(name, source, tmp_path):
 def test_unmutated_oracle_passes_all_pins():
     caught_by, exc = _run_pins()
     assert caught_by is None, "%s: %s" % (caught_by, exc)
+
+
+# The oracle's own Python arithmetic (the column-major scale placement) gets
+# planted mistakes too, swapped in for the function the pins call.
+def _col_major_unpadded_ld(scales):
+    scales = np.asarray(scales)
+    return np.ascontiguousarray(scales.T)                      # ld = rows: no 16-byte rounding
+
+
+def _col_major_pads_to_16_elements(scales):
+    scales = np.asarray(scales)
+    rows, G = scales.shape
+    ld = (rows + 15) // 16 * 16                                # 16 elements instead of 16 bytes
+    out = np.zeros((G, ld), scales.dtype)
+    out[:, :rows] = scales.T
+    return out
+
+
+def _col_major_groups_reversed(scales):
+    scales = np.asarray(scales)
+    rows, G = scales.shape
+    per16 = 16 // scales.dtype.itemsize
+    ld = (rows + per16 - 1) // per16 * per16
+    out = np.zeros((G, ld), scales.dtype)
+    out[:, :rows] = scales.T[::-1]
+    return out
+
+
+PY_MUTANTS = {
+    "col_major_unpadded_ld": ("scales_col_major", _col_major_unpadded_ld),
+    "col_major_pads_to_16_elements": ("scales_col_major", _col_major_pads_to_16_elements),
+    "col_major_groups_reversed": ("scales_col_major", _col_major_groups_reversed),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_pins_catch_planted_python_mistake(name, monkeypatch):
+    fn_name, fn = PY_MUTANTS[name]
+    monkeypatch.setattr(oracle, fn_name, fn)
+    caught_by, _ = _run_pins()
+    assert caught_by is not None, "no pin caught the planted mistake %r" % name
