@@ -184,7 +184,7 @@ def algorithmic_bytes(cfg, cnt, A, slab=0):
     pad = (Np - N) if cfg["zero_pad"] else 0
     nb = H // 128
     out_row = (H + 4 * nb) if cfg["fp8"] else 2 * H
-    layout_b = T * K * 8 * 2 + T * K * 4 * 2 + Np * 12 + E * 8      # idx read twice, weights, slots, maps
+    layout_b = T * K * (8 + 4 + 4) + Np * 12 + E * 8     # idx and weights read, slots written, row maps, counts
     dispatch_b = T * 2 * H + (N + pad) * out_row + T * K * 4
     combine_b = N * 2 * H + T * K * 8 + T * 2 * H
     return dict(layout=layout_b, dispatch=dispatch_b, combine=combine_b, N=N, Np=Np, pad_rows=Np - N)

@@ -94,6 +94,8 @@ def test_algorithmic_bytes_accounting():
     Np = int(((cnt + A - 1) // A * A).sum())
     b = bench.algorithmic_bytes(cfg, cnt, A)
     assert (b["N"], b["Np"], b["pad_rows"]) == (N, Np, Np - N)
+    # layout: topk_idx and weights read once, one slot written per entry, 12 B per receive row, E counts
+    assert b["layout"] == T * K * (8 + 4 + 4) + Np * 12 + E * 8
     assert b["dispatch"] == T * 2 * H + Np * 2 * H + T * K * 4
     assert b["combine"] == N * 2 * H + T * 2 * H + T * K * 8
     fp8 = dict(cfg, fp8=True)
