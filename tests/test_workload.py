@@ -56,3 +56,21 @@ def test_expert_outputs_range():
     f = np.abs((y.astype(np.uint32) << 16).view(np.float32))
     assert f.min() >= 2.0 ** -7 and f.max() < 16.0
     assert np.array_equal(y, workload.expert_outputs(cfg, 64))
+
+
+@pytest.mark.parametrize("name,pairs,rows", [
+    ("tiny", 512, 512),
+    ("prefill_bf16", 32768, 56576),
+    ("fp8_dispatch", 32768, 56576),
+    ("decode", 29418, 29418),
+    ("large_prefill", 131072, 153472),
+])
+def test_realised_workload_sizes(name, pairs, rows):
+    """The seeded inputs are fixed: the pair and receive-row counts every
+    reported figure was measured on (the oracle's layout of each workload)."""
+    import oracle
+    cfg = workload.config(name)
+    inp = workload.inputs(cfg, with_x=False)
+    lay = oracle.layout(inp["topk_idx"], inp["topk_weights"], cfg["E"], cfg["R"], cfg["A"])
+    assert int((inp["topk_idx"] >= 0).sum()) == pairs
+    assert int(lay["off"][-1]) == rows
