@@ -143,6 +143,24 @@ int prepare_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, cons
 
 }  // namespace
 
+namespace ep {
+
+int layout_call(const int64_t* topk_idx, const float* topk_weights, int T, int K, int E, int R, int A,
+                int num_max_tokens_per_rank, ep_layout_t* layout, cudaStream_t s, bool clear_header) {
+    LayoutArgs a;
+    int rc = prepare_layout(topk_idx, topk_weights, T, K, E, R, A, num_max_tokens_per_rank, layout, &a);
+    if (rc != EP_OK) return rc;
+    if (T == 0) return empty_layout(layout, s);   // clears the header itself
+    int sms = 0;
+    if ((rc = device_sms(&sms)) != EP_OK) return rc;
+    // only now, with every check passed, may the call touch the workspace
+    if (clear_header && cudaMemsetAsync(layout->workspace, 0, sizeof(WsHeader), s) != cudaSuccess)
+        return EP_ERR_CUDA;
+    return launch_layout(a, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+}  // namespace ep
+
 extern "C" {
 
 int ep_version(void) { return EP_B200_VERSION; }
@@ -173,15 +191,8 @@ int64_t ep_capacity_rows(int num_tokens, int num_topk, int num_experts, int expe
 int ep_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
               int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
               ep_layout_t* layout, void* stream) {
-    ep::LayoutArgs a;
-    int rc = prepare_layout(topk_idx, topk_weights, num_tokens, num_topk, num_experts, num_ranks,
-                            expert_alignment, num_max_tokens_per_rank, layout, &a);
-    if (rc != EP_OK) return rc;
-    cudaStream_t s = (cudaStream_t)stream;
-    if (num_tokens == 0) return empty_layout(layout, s);
-    int sms = 0;
-    if ((rc = device_sms(&sms)) != EP_OK) return rc;
-    return ep::launch_layout(a, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    return ep::layout_call(topk_idx, topk_weights, num_tokens, num_topk, num_experts, num_ranks, expert_alignment,
+                           num_max_tokens_per_rank, layout, (cudaStream_t)stream, false);
 }
 
 size_t ep_rank_workspace_bytes(int num_tokens, int num_ranks, int num_experts) {

@@ -105,6 +105,12 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 
 cudaError_t launch_selftest_wait(WsHeader* hdr, uint64_t timeout_ns, cudaStream_t s);
 
+// ep_layout's argument checks, then its launch on `s`.  With clear_header the
+// workspace header words are zeroed on the stream first, but only once every
+// check has passed: a rejected call enqueues nothing (ep_abi.cu).
+int layout_call(const int64_t* topk_idx, const float* topk_weights, int T, int K, int E, int R, int A,
+                int num_max_tokens_per_rank, ep_layout_t* layout, cudaStream_t s, bool clear_header);
+
 // Per-token-per-rank layout (ep_rank_layout.cu).  Workspace: the expand-layout
 // workspace of the [T, R] (token, rank) table (E' = K' = R, A = 1), scratch
 // targets for the layout kernel's per-row weight and local-expert writes

@@ -55,10 +55,11 @@ int ep_layout_no_alloc(const int64_t* topk_idx, const float* topk_weights, int n
     ep_layout_t tmp = *layout;
     tmp.workspace = ws;
     tmp.workspace_bytes = kStaticScratchBytes;
-    // the barrier counter and the pending flags must start at zero
-    if (cudaMemsetAsync(ws, 0, sizeof(ep::WsHeader), (cudaStream_t)stream) != cudaSuccess) return EP_ERR_CUDA;
-    rc = ep_layout(topk_idx, topk_weights, num_tokens, num_topk, num_experts, num_ranks, expert_alignment,
-                   num_max_tokens_per_rank, &tmp, stream);
+    // ep_layout's checks first; only a call that passes them clears the
+    // header words that must start at zero (the barrier counter, the pending
+    // flags) and launches, so a rejected call leaves the shared array as it was
+    rc = ep::layout_call(topk_idx, topk_weights, num_tokens, num_topk, num_experts, num_ranks, expert_alignment,
+                         num_max_tokens_per_rank, &tmp, (cudaStream_t)stream, true);
     if (rc == EP_OK) *layout = tmp;
     return rc;
 }

@@ -368,12 +368,22 @@ int ep_cast_fp8(const void* x, int num_tokens, int hidden, int scale_format, voi
  * provides every input and output array.  It calls no cudaMalloc or cudaFree.
  *
  *   - Sizes whose workspace (ep_workspace_bytes) exceeds 4 MiB are rejected
- *     with EP_ERR_UNSUPPORTED, before anything is enqueued.
+ *     with EP_ERR_UNSUPPORTED, and every other argument error is returned as
+ *     ep_layout returns it; a rejected call enqueues nothing and leaves the
+ *     array as it was.
  *   - Every GPU that loads the library holds the 4 MiB until the process exits.
  *   - All calls on a device share the one array and it keeps the last call's
- *     contents (each call clears the words that must start at zero).  Calls
- *     whose work overlaps on the GPU - from other streams or threads, or a
- *     dispatch or combine of an older handle still pending - race on it.
+ *     contents (each accepted call clears the words that must start at zero).
+ *     Calls whose work overlaps on the GPU - from other streams or threads, or
+ *     a dispatch or combine of an older handle still pending - race on it.
+ *   - Each accepted call also replaces what every earlier no-alloc handle on
+ *     that device reads from the array: the list of padding rows, their
+ *     number and the device status word.  After a later ep_layout_no_alloc,
+ *     an older no-alloc handle is still valid for ep_dispatch with
+ *     do_zero_padding = 0 and for ep_combine (their arrays are the caller's),
+ *     but ep_dispatch with do_zero_padding = 1 would zero the later call's
+ *     padding rows and ep_get_status would report the later call's flags.
+ *     Use only the most recent no-alloc handle for those two.
  *   - The first call on a device looks up the array's device address with that
  *     device current (cudaGetSymbolAddress) and caches it; make that first call
  *     before any stream capture.
