@@ -2,11 +2,15 @@
 
 One step = the whole hot path over one batch: ep_layout (one kernel),
 ep_dispatch (with the fused FP8 cast for the FP8 workload) and ep_combine, on
-the default workload "prefill_bf16": T = 4096 tokens,
-H = 7168 bf16, 256 experts, top-8, R = 8 virtual ranks, expert_alignment 128,
-zero padding, skewed (Zipf s = 1.2 bias) gate.  Inputs are seeded synthetic
-(workload/), resident in HBM before timing; the combine input ("expert
-outputs") is the dispatched receive buffer itself (identity experts).
+the default workload "large_prefill", the largest one-GPU configuration:
+T = 16384 tokens, H = 7168 bf16, 256 experts, top-8, R = 64 virtual ranks
+(4 experts each), expert_alignment 128, zero padding, heavily skewed (Zipf
+s = 1.5 bias, two hot experts take about 20 % of the pairs) gate, weighted
+combine.  Inputs are seeded synthetic (workload/), resident in HBM before
+timing; the combine input ("expert outputs") is the dispatched receive buffer
+itself (identity experts).  After the headline, the same measurement runs on
+every other workload (tiny, prefill_bf16, fp8_dispatch, decode) and is
+reported under "per_workload" (one GPU only).
 
 Timing: W warm-up steps, then K steps; before every step L2 is flushed by
 writing a 256 MiB buffer (outside the timed events); each step is timed with
@@ -43,11 +47,13 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=10)
-    p.add_argument("--workload", default="prefill_bf16", choices=sorted(workload.WORKLOADS))
+    p.add_argument("--workload", default="large_prefill", choices=sorted(workload.WORKLOADS))
     p.add_argument("--tokens", type=int, default=None,
                    help="override the workload's token count T (a multiple of its rank count)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-per-workload", dest="per_workload", action="store_false",
+                   help="time only the headline workload (by default the others follow it on one GPU)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--fused", action="store_true",
@@ -202,9 +208,18 @@ def algorithmic_bytes_rank(cfg, rows, N):
     return dict(layout=layout_b, dispatch=dispatch_b, combine=combine_b, N=N, Np=rows, pad_rows=0)
 
 
+def l2_statement(cfg, nbytes):
+    """How the workload relates to the 126 MB L2: a property of the work, the
+    same for both arms (the GPU arm's own flush is reported beside `config`)."""
+    read_mb = (cfg["T"] + nbytes["Np"] - nbytes["pad_rows"]) * cfg["H"] * 2 / 1e6
+    if read_mb > 126:
+        return "inputs larger than L2: each step reads x and the expert-output rows, %.0f MB > 126 MB" % read_mb
+    return "inputs fit in L2 (%.1f MB per step)" % read_mb
+
+
 def workload_config(cfg, form, world, nbytes, topk_idx):
-    """The `config` keys that name the workload; both arms print them, so the
-    reference line describes exactly the work of ours."""
+    """The `config` keys that name the workload; both arms print exactly these,
+    so the reference line describes exactly the work of ours."""
     T, H, E, K, R, A = (cfg[k] for k in ("T", "H", "E", "K", "R", "A"))
     M = cfg["max_tokens_per_rank"] or T // R
     shape = {"expand": "",
@@ -214,128 +229,140 @@ def workload_config(cfg, form, world, nbytes, topk_idx):
                 cfg["name"], T, H, E, K, R, A, cfg["zero_pad"], " fp8-cast" if cfg["fp8"] else "", shape),
             "global_batch": T * world, "parallelism": "replicas x%d (R=%d virtual ranks per GPU)" % (world, R),
             "pairs": nbytes["N"], "recv_rows": nbytes["Np"], "pad_rows": nbytes["pad_rows"],
-            "load": workload.load_stats(topk_idx, E)}
+            "load": workload.load_stats(topk_idx, E), "l2": l2_statement(cfg, nbytes)}
+
+
+def form_bytes(cfg, form, cnt_or_rows, n_pairs):
+    """Algorithmic bytes of one step of `form` on `cfg`: cnt_or_rows is the
+    per-expert pair counts (expand, ll) or the receive-row count (rank)."""
+    if form == "rank":
+        return algorithmic_bytes_rank(cfg, cnt_or_rows, n_pairs)
+    if form == "ll":
+        return algorithmic_bytes(cfg, cnt_or_rows, 1, slab=cfg["R"] * (cfg["max_tokens_per_rank"] or
+                                                                       cfg["T"] // cfg["R"]))
+    return algorithmic_bytes(cfg, cnt_or_rows, cfg["A"])
 
 
 # --------------------------------------------------------------------------
 # our implementation
 # --------------------------------------------------------------------------
-def run_ours(args, rank, world, local_rank):
-    import torch
-    import combine_ep_layout_11_b200 as ep
-    from combine_ep_layout_11_b200 import build as lib_build
-    if rank == 0 or not os.path.exists(lib_build.LIB):
-        lib_build.build()
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        import datetime
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+class Step:
+    """One workload set up on the device: inputs resident in HBM, the handle,
+    the receive and output buffers, and the calls of one step."""
 
-    cfg = bench_config(args)
-    inp = workload.inputs(cfg)
-    T, H, K, E, R, A = cfg["T"], cfg["H"], cfg["K"], cfg["E"], cfg["R"], cfg["A"]
-    idx = torch.from_numpy(inp["topk_idx"]).to(dev)
-    w = torch.from_numpy(inp["topk_weights"]).to(dev)
-    x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
-    per_rank = args.layout == "rank"
-    slab = args.layout == "ll"
-    M = cfg["max_tokens_per_rank"] or T // R
-    if args.layout != "expand" and args.fused:
-        raise SystemExit("--fused applies to the expand layout only")
-    if per_rank:
-        lay = ep.RankLayout(T, K, E, R, A, dev)
-    elif slab:
-        lay = ep.ll_layout(idx, w, E, R, M)
-    else:
-        lay = ep.Layout(T, K, E, R, A, dev, num_max_tokens_per_rank=cfg["max_tokens_per_rank"])
-    cw = None if per_rank else w            # V1's combine is a plain sum over the ranks
-    cap = lay.capacity
-    fp8 = cfg["fp8"]
-    recv = torch.empty((cap, H), dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16, device=dev)
-    recv_s = torch.empty((cap, H // 128), dtype=torch.float32, device=dev) if fp8 else None
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def dispatch():
+    def __init__(self, args, cfg, ep, torch, dev):
+        self.args, self.cfg, self.ep, self.torch, self.dev = args, cfg, ep, torch, dev
+        self.inp = inp = workload.inputs(cfg)
+        T, H, K, E, R, A = cfg["T"], cfg["H"], cfg["K"], cfg["E"], cfg["R"], cfg["A"]
+        self.idx = torch.from_numpy(inp["topk_idx"]).to(dev)
+        self.w = torch.from_numpy(inp["topk_weights"]).to(dev)
+        self.x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+        self.form = args.layout
+        self.per_rank = self.form == "rank"
+        self.slab = self.form == "ll"
+        self.M = cfg["max_tokens_per_rank"] or T // R
+        if self.form != "expand" and args.fused:
+            raise SystemExit("--fused applies to the expand layout only")
+        if self.per_rank:
+            self.lay = ep.RankLayout(T, K, E, R, A, dev)
+        elif self.slab:
+            self.lay = ep.ll_layout(self.idx, self.w, E, R, self.M)
+        else:
+            self.lay = ep.Layout(T, K, E, R, A, dev, num_max_tokens_per_rank=cfg["max_tokens_per_rank"])
+        self.cw = None if self.per_rank else self.w          # V1's combine is a plain sum over the ranks
+        cap = self.lay.capacity
+        self.fp8 = fp8 = cfg["fp8"]
+        self.recv = torch.empty((cap, H), dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16, device=dev)
+        self.recv_s = torch.empty((cap, H // 128), dtype=torch.float32, device=dev) if fp8 else None
+        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.stream = torch.cuda.current_stream(dev)
+        # expert outputs for combine: identity experts (bf16), or seeded outputs for FP8
+        self.do_layout(self.idx, self.w)
+        self.dispatch()
+        torch.cuda.synchronize(dev)
         if fp8:
-            ep.dispatch(lay, x, cast_to_fp8=True, do_zero_padding=cfg["zero_pad"], out=recv, out_scales=recv_s)
+            self.y = torch.from_numpy(workload.expert_outputs(cfg, cap).view(np.int16)).to(dev).view(torch.bfloat16)
         else:
-            ep.dispatch(lay, x, do_zero_padding=cfg["zero_pad"], out=recv)
-
-    def do_layout(d_idx, d_w):
-        if per_rank:
-            ep.rank_layout(d_idx, d_w, E, R, A, out=lay)
-        elif slab:
-            ep.ll_layout(d_idx, d_w, E, R, M, out=lay)
+            self.y = self.recv.clone()
+        if self.per_rank:
+            self.nbytes = form_bytes(cfg, "rank", self.lay.num_recv_rows(), int((self.idx >= 0).sum()))
         else:
-            ep.layout(d_idx, d_w, E, R, A, cfg["max_tokens_per_rank"], out=lay)
+            self.nbytes = form_bytes(cfg, self.form, self.lay.num_recv_tokens_per_expert.cpu().numpy(), None)
 
-    # expert outputs for combine: identity experts (bf16), or seeded outputs for FP8
-    do_layout(idx, w)
-    dispatch()
-    torch.cuda.synchronize(dev)
-    if fp8:
-        y = torch.from_numpy(workload.expert_outputs(cfg, cap).view(np.int16)).to(dev).view(torch.bfloat16)
-    else:
-        y = recv.clone()
-    if per_rank:
-        nbytes = algorithmic_bytes_rank(cfg, lay.num_recv_rows(), int((idx >= 0).sum()))
-    elif slab:
-        nbytes = algorithmic_bytes(cfg, lay.num_recv_tokens_per_expert.cpu().numpy(), 1, slab=R * M)
-    else:
-        nbytes = algorithmic_bytes(cfg, lay.num_recv_tokens_per_expert.cpu().numpy(), A)
+    def dispatch(self):
+        cfg = self.cfg
+        if self.fp8:
+            self.ep.dispatch(self.lay, self.x, cast_to_fp8=True, do_zero_padding=cfg["zero_pad"], out=self.recv,
+                             out_scales=self.recv_s)
+        else:
+            self.ep.dispatch(self.lay, self.x, do_zero_padding=cfg["zero_pad"], out=self.recv)
 
-    def step(evs=None):
+    def do_layout(self, d_idx, d_w):
+        cfg, ep = self.cfg, self.ep
+        if self.per_rank:
+            ep.rank_layout(d_idx, d_w, cfg["E"], cfg["R"], cfg["A"], out=self.lay)
+        elif self.slab:
+            ep.ll_layout(d_idx, d_w, cfg["E"], cfg["R"], self.M, out=self.lay)
+        else:
+            ep.layout(d_idx, d_w, cfg["E"], cfg["R"], cfg["A"], cfg["max_tokens_per_rank"], out=self.lay)
+
+    def step(self, evs=None):
+        cfg, ep, stream = self.cfg, self.ep, self.stream
         if evs:
             evs[0].record(stream)
-        if not args.fused:
-            do_layout(idx, w)
+        if not self.args.fused:
+            self.do_layout(self.idx, self.w)
             if evs:
                 evs[1].record(stream)
-            dispatch()
+            self.dispatch()
         else:
-            ep.layout_dispatch(idx, w, x, E, R, A, cfg["max_tokens_per_rank"], cast_to_fp8=fp8,
-                               do_zero_padding=cfg["zero_pad"], out_layout=lay, out=recv, out_scales=recv_s)
+            ep.layout_dispatch(self.idx, self.w, self.x, cfg["E"], cfg["R"], cfg["A"], cfg["max_tokens_per_rank"],
+                               cast_to_fp8=self.fp8, do_zero_padding=cfg["zero_pad"], out_layout=self.lay,
+                               out=self.recv, out_scales=self.recv_s)
             if evs:
                 evs[1].record(stream)
         if evs:
             evs[2].record(stream)
-        ep.combine(lay, y, cw, out=out)
+        ep.combine(self.lay, self.y, self.cw, out=self.out)
         if evs:
             evs[3].record(stream)
 
+    def check(self):
+        """Device status clean; with identity experts and weights summing to one,
+        combine(dispatch(x)) gives x back."""
+        torch = self.torch
+        torch.cuda.synchronize(self.dev)
+        code, flags = self.ep.get_status(self.lay)
+        assert code == 0, "device status %d (flags %d)" % (code, flags)
+        if not self.fp8 and self.cfg["drop"] == 0 and not self.per_rank:
+            has = (self.idx >= 0).any(dim=1)
+            assert torch.equal(self.out[has].float(), self.x[has].float()), "combine(dispatch(x)) != x"
+
+
+def time_steps(st, args, flush, dist, dev, clocks=None):
+    """W warm-up steps, then K timed steps (one event pair around each; no
+    events between the kernels), then K more with events between the calls
+    for the per-kernel split.  Returns the timings in ms."""
+    torch = st.torch
     for _ in range(args.warmup):
         flush.zero_()
-        step()
-    torch.cuda.synchronize(dev)
-    code, flags = ep.get_status(lay)
-    assert code == 0, "device status %d (flags %d)" % (code, flags)
-    if not fp8 and cfg["drop"] == 0 and not per_rank:   # identity experts, weights summing to 1: x again
-        has = (idx >= 0).any(dim=1)
-        assert torch.equal(out[has].float(), x[has].float()), "combine(dispatch(x)) != x"
-
+        st.step()
+    st.check()
     # optionally one step captured as a CUDA graph (the calls allocate nothing
     # and only enqueue work, so they capture as they are)
-    run_step = step
+    run_step, graph = st.step, None
     if args.graph:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, capture_error_mode="thread_local"):
-            step()
+            st.step()
         torch.cuda.synchronize(dev)
         for _ in range(3):
             flush.zero_()
             graph.replay()
         torch.cuda.synchronize(dev)
         run_step = graph.replay
-
-    # timed region: K steps, one event pair around each step (no events between
-    # the kernels, so each launch may overlap its predecessor's tail)
+    stream = st.stream
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    clocks = ClockSampler(local_rank) if (rank == 0 and not args.no_clocks) else None
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -355,20 +382,86 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     clock_info = clocks.stop() if clocks else None
     step_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    ms_per_step = max_over_ranks(np.mean(step_ms), dist, dev)
-    ms_median = max_over_ranks(float(np.median(step_ms)), dist, dev)
     # per-kernel breakdown: the same K steps again with events between the kernels
     evk = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     for i in range(args.steps):
         if args.flush:
             flush.zero_()
-        step(evk[i])
+        st.step(evk[i])
     torch.cuda.synchronize(dev)
+    st.check()
     per = np.array([[evk[i][j].elapsed_time(evk[i][j + 1]) for j in range(3)] for i in range(args.steps)])
+    del graph
+    return dict(ms_mean=float(np.mean(step_ms)), ms_median=float(np.median(step_ms)),
+                kernel_ms=per.mean(axis=0), wall=wall, clocks=clock_info)
+
+
+def kernel_summary(st, args, k_ms, peak):
+    """Per-kernel times, the dominant kernel's achieved bandwidth and its roofline fraction."""
+    nb = st.nbytes
+    if not args.fused:
+        top_kernel = "dispatch_cast_kernel" if st.fp8 else "dispatch_copy_kernel"
+        top_bytes, top_ms = nb["dispatch"], k_ms[1]
+        kernels_us = {"layout": round(k_ms[0] * 1e3, 2), "dispatch": round(k_ms[1] * 1e3, 2)}
+    else:
+        top_kernel = "layout_kernel+dispatch_cast_kernel" if st.fp8 else "layout_dispatch_kernel"
+        top_bytes, top_ms = nb["layout"] + nb["dispatch"], k_ms[0] + k_ms[1]
+        kernels_us = {"layout_dispatch": round(top_ms * 1e3, 2)}
+    kernels_us["combine"] = round(k_ms[2] * 1e3, 2)
+    disp_gbs = top_bytes / (top_ms * 1e-3) / 1e9
+    return dict(top_kernel=top_kernel, top_bytes=top_bytes, disp_gbs=disp_gbs, kernels_us=kernels_us,
+                combine_gbs=nb["combine"] / (k_ms[2] * 1e-3) / 1e9, frac=disp_gbs / peak)
+
+
+def step_bytes(nb):
+    return nb["layout"] + nb["dispatch"] + nb["combine"]
+
+
+def per_workload_entry(st, args, tm, peak):
+    """One line of `per_workload`: a whole-step and per-kernel summary."""
+    ks = kernel_summary(st, args, tm["kernel_ms"], peak)
+    ms = tm["ms_mean"]
+    total = step_bytes(st.nbytes)
+    return {"workload": workload_config(st.cfg, args.layout, 1, st.nbytes, st.inp["topk_idx"])["workload"],
+            "ms_per_step": round(ms, 5), "ms_per_step_median": round(tm["ms_median"], 5),
+            "tokens_per_s": round(st.cfg["T"] / (ms * 1e-3), 1),
+            "hbm_gbs": round(total / (ms * 1e-3) / 1e9, 1),
+            "hbm_frac_of_measured": round(total / (ms * 1e-3) / 1e9 / peak, 4),
+            "hbm_frac_of_nominal_8tbs": round(total / (ms * 1e-3) / 1e9 / 8000.0, 4),
+            "algorithmic_bytes_per_step": total,
+            "kernels_us": ks["kernels_us"],
+            "dispatch": {"kernel": ks["top_kernel"], "gbs": round(ks["disp_gbs"], 1), "frac": round(ks["frac"], 4)},
+            "combine_gbs": round(ks["combine_gbs"], 1),
+            "gpu_launches_per_step": 2 if (args.fused and not st.fp8) else 3}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import combine_ep_layout_11_b200 as ep
+    from combine_ep_layout_11_b200 import build as lib_build
+    if rank == 0 or not os.path.exists(lib_build.LIB):
+        lib_build.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    cfg = bench_config(args)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    st = Step(args, cfg, ep, torch, dev)
+    T, H = cfg["T"], cfg["H"]
+    clocks = ClockSampler(local_rank) if (rank == 0 and not args.no_clocks) else None
+    tm = time_steps(st, args, flush, dist, dev, clocks)
+    ms_per_step = max_over_ranks(tm["ms_mean"], dist, dev)
+    ms_median = max_over_ranks(tm["ms_median"], dist, dev)
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush, do_layout, per_rank)
+        e2e = run_e2e(args, ep, torch, dev, st.inp, cfg, st.lay, st.y, st.fp8, st.recv, st.recv_s, flush,
+                      st.do_layout, st.per_rank)
         e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dist, dev)
 
     if rank != 0:
@@ -378,20 +471,11 @@ def run_ours(args, rank, world, local_rank):
         return None
 
     peak, peak_kind = measured_peaks()
+    nbytes, fp8 = st.nbytes, st.fp8
     payload_rows = nbytes["Np"] - nbytes["pad_rows"]
-    k_ms = per.mean(axis=0)   # layout, dispatch, combine (fused: layout+dispatch, -, combine)
-    total_bytes = nbytes["layout"] + nbytes["dispatch"] + nbytes["combine"]
-    if not args.fused:
-        top_kernel = "dispatch_cast_kernel" if fp8 else "dispatch_copy_kernel"
-        top_bytes, top_ms = nbytes["dispatch"], k_ms[1]
-        kernels_us = {"layout": round(k_ms[0] * 1e3, 2), "dispatch": round(k_ms[1] * 1e3, 2)}
-    else:
-        top_kernel = "layout_kernel+dispatch_cast_kernel" if fp8 else "layout_dispatch_kernel"
-        top_bytes, top_ms = nbytes["layout"] + nbytes["dispatch"], k_ms[0] + k_ms[1]
-        kernels_us = {"layout_dispatch": round(top_ms * 1e3, 2)}
-    kernels_us["combine"] = round(k_ms[2] * 1e3, 2)
-    kernels_us["note"] = "second pass with events between the calls"
-    disp_gbs = top_bytes / (top_ms * 1e-3) / 1e9
+    ks = kernel_summary(st, args, tm["kernel_ms"], peak)
+    total_bytes = step_bytes(nbytes)
+    kernels_us = dict(ks["kernels_us"], note="second pass with events between the calls")
     value = job_throughput(T, world, ms_per_step)
     line = {
         "metric": METRIC,
@@ -406,12 +490,10 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "fp8-e4m3/bf16" if fp8 else "bf16",
         "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
-        "config": dict(
-            workload_config(cfg, args.layout, world, nbytes, inp["topk_idx"]),
-            l2=("flushed by a 256 MiB write before every step, outside the timed events" if args.flush else
-                "not flushed: the inputs each step reads (x and the expert-output rows, %.0f MB) exceed "
-                "the 126 MB L2" % ((T + nbytes["Np"] - nbytes["pad_rows"]) * H * 2 / 1e6)),
-            launch="one CUDA graph per step" if args.graph else "stream launches with programmatic dependent launch"),
+        "config": workload_config(cfg, args.layout, world, nbytes, st.inp["topk_idx"]),
+        "l2_flush": ("a 256 MiB write before every step, outside the timed events" if args.flush else
+                     "none (the step's inputs exceed L2)"),
+        "launch": "one CUDA graph per step" if args.graph else "stream launches with programmatic dependent launch",
         "ms_per_step_median": round(ms_median, 5),
         # the count_bytes convention: one row copy in dispatch and one row read in
         # combine per receive row that holds data
@@ -422,28 +504,43 @@ def run_ours(args, rank, world, local_rank):
         "hbm_frac_of_nominal_8tbs": round(total_bytes / (ms_per_step * 1e-3) / 1e9 / 8000.0, 4),
         "algorithmic_bytes_per_step": total_bytes,
         "kernels_us": kernels_us,
-        "kernels_gbs": {"dispatch": round(disp_gbs, 1),
-                        "combine": round(nbytes["combine"] / (k_ms[2] * 1e-3) / 1e9, 1)},
-        "roofline": {"bound": "hbm", "kernel": top_kernel,
-                     "achieved": round(disp_gbs, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(disp_gbs / peak, 4),
-                     "traffic": ncu_traffic(top_kernel, cfg["name"] + ("" if args.layout == "expand"
-                                                                       else "/" + args.layout)),
-                     "algorithmic_bytes_per_launch": top_bytes},
+        "kernels_gbs": {"dispatch": round(ks["disp_gbs"], 1), "combine": round(ks["combine_gbs"], 1)},
+        "roofline": {"bound": "hbm", "kernel": ks["top_kernel"],
+                     "achieved": round(ks["disp_gbs"], 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(ks["frac"], 4),
+                     "traffic": ncu_traffic(ks["top_kernel"], cfg["name"] + ("" if args.layout == "expand"
+                                                                             else "/" + args.layout)),
+                     "algorithmic_bytes_per_launch": ks["top_bytes"]},
         "gpu_launches": args.steps * (2 if (args.fused and not fp8) else 3),
-        "wall_s_timed_region": round(wall, 4),
+        "wall_s_timed_region": round(tm["wall"], 4),
     }
-    if clock_info:
-        line["clocks"] = clock_info
+    if tm["clocks"]:
+        line["clocks"] = tm["clocks"]
     if e2e:
         line["e2e"] = {"value": round(job_throughput(T, world, e2e["ms_per_step"]), 1), "unit": "tokens/s",
                        "ms_per_step": round(e2e["ms_per_step"], 4),
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                       "how": "%d steps through the public API from pinned host buffers, uploads, calls and "
-                              "downloads pipelined over three streams, timed from the first upload to the "
-                              "last download; no L2 flush (each step moves > 1 GB)" % e2e["steps"]}
+                       "how": "%d steps through the public API from pinned host buffers: every step uploads "
+                              "topk_idx, topk_weights and x and downloads the combined output; the expert "
+                              "outputs (the combine input) stay resident on the device, as a GPU expert layer "
+                              "produces them there; uploads, calls and downloads pipelined over three streams, "
+                              "timed from the first upload to the last download; no L2 flush (each step moves "
+                              "more than L2 holds)" % e2e["steps"]}
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, inp, args.layout)
+        line["cpu_baseline"] = cpu_baseline(cfg, st.inp, args.layout)
+    if world == 1 and args.per_workload and args.tokens is None:
+        # every other workload, same measurement, one at a time (buffers freed in between)
+        del st, e2e
+        torch.cuda.empty_cache()
+        entries = {}
+        for name in sorted(workload.WORKLOADS, key=lambda n: workload.WORKLOADS[n]["index"]):
+            if name == cfg["name"]:
+                continue
+            other = Step(args, workload.config(name), ep, torch, dev)
+            entries[name] = per_workload_entry(other, args, time_steps(other, args, flush, None, dev), peak)
+            del other
+            torch.cuda.empty_cache()
+        line["per_workload"] = entries
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -559,12 +656,9 @@ def run_reference(args, rank, world):
     import oracle
     olay = oracle.step_layout(inp, cfg, form)
     if form == "rank":
-        nbytes = algorithmic_bytes_rank(cfg, int(olay["off"][-1]), int((inp["topk_idx"] >= 0).sum()))
-    elif form == "ll":
-        nbytes = algorithmic_bytes(cfg, olay["cnt"], 1, slab=cfg["R"] * (cfg["max_tokens_per_rank"] or
-                                                                       cfg["T"] // cfg["R"]))
+        nbytes = form_bytes(cfg, form, int(olay["off"][-1]), int((inp["topk_idx"] >= 0).sum()))
     else:
-        nbytes = algorithmic_bytes(cfg, olay["cnt"], cfg["A"])
+        nbytes = form_bytes(cfg, form, olay["cnt"], None)
     for _ in range(args.warmup):
         oracle.step(full, cfg, form)
     ts = []
@@ -578,8 +672,7 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp8-e4m3/bf16" if cfg["fp8"] else "bf16",
             "data": "synthetic (seeded; workload/ generator, seed %d)" % cfg["seed"],
-            "config": dict(workload_config(cfg, form, world, nbytes, inp["topk_idx"]),
-                           l2="not applicable: the oracle runs on the host cores"),
+            "config": workload_config(cfg, form, world, nbytes, inp["topk_idx"]),
             "impl": "reference",
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": "the full %s workload per step (single-threaded C oracle)" % cfg["name"]},

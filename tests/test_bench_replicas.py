@@ -130,5 +130,20 @@ def test_reference_line_names_our_workload(form):
     assert c["recv_rows"] == int(lay["off"][-1])
     expect = bench.workload_config(cfg, form, 1, {"N": c["pairs"], "Np": c["recv_rows"], "pad_rows": c["pad_rows"]},
                                    inp["topk_idx"])
-    assert {k: c[k] for k in expect} == expect
+    assert c == expect                      # the same keys and values as our arm's config
     assert np.isfinite(line["value"]) and line["value"] > 0
+
+
+def test_default_workload_is_the_largest_one_gpu_configuration(monkeypatch):
+    """With no flags the bench times large_prefill (T = 16384, R = 64), the
+    largest configuration that fits one GPU, and follows it with the others."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workload
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    args = bench.parse()
+    assert args.workload == "large_prefill" and args.per_workload and args.gpus == 1
+    assert args.warmup >= 3
+    cfg = bench.bench_config(args)
+    assert max(workload.WORKLOADS, key=lambda n: workload.WORKLOADS[n]["T"]) == "large_prefill"
+    assert (cfg["T"], cfg["H"], cfg["E"], cfg["K"], cfg["R"], cfg["A"]) == (16384, 7168, 256, 8, 64, 128)
