@@ -8,6 +8,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <cstddef>
+
 #include "ep_b200.h"
 
 namespace ep {
@@ -25,18 +27,26 @@ constexpr uint32_t kDevTimeout = EP_DEV_TIMEOUT;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // ---------------------------------------------------------------------------
-// Workspace: [0, 256) header words, then the (chunk x expert) count table,
-// the padding prefix and the list of padding rows.
+// Workspace: [0, 256) header words, then the (chunk x expert) count table, the
+// padding prefix and the list of padding rows.
 // ---------------------------------------------------------------------------
-// `bar_count` and `pending` must be zero before the first ep_layout on a
-// workspace; every ep_layout leaves them at zero again.
+// Every word before `bar_gen` must be zero before the first ep_layout on a
+// workspace; the layout and dispatch kernels leave them at zero again (apart
+// from the status word and num_pad, which the next layout rewrites), and the
+// host clears them (kHeaderClearBytes) where a call skips the layout kernel.
 struct WsHeader {
-    uint32_t status;     // EP_DEV_* bits of the last ep_layout and what followed it
-    uint32_t bar_count;  // grid barrier: CTAs arrived in the current generation
-    int32_t num_pad;     // padding rows (expert_offset[E] - pairs)
-    uint32_t pending;    // flags raised by CTAs before the barrier
-    uint32_t bar_gen;    // grid barrier generation
+    uint32_t status;      // EP_DEV_* bits of the last ep_layout and what followed it
+    int32_t num_pad;      // padding rows (expert_offset[E] - pairs)
+    uint32_t pending;     // flags raised by layout CTAs before the grid barrier
+    uint32_t tok_ticket;  // dispatch: next token-row ticket
+    uint32_t pad_ticket;  // dispatch: next padding ticket
+    uint32_t done;        // dispatch: CTAs finished (the last one resets the tickets)
+    uint32_t bar_count;   // layout grid barrier: CTAs arrived in the current generation
+    uint32_t reserved;
+    uint32_t bar_gen;     // layout grid barrier generation (any value will do)
 };
+constexpr size_t kHeaderClearBytes = offsetof(WsHeader, bar_gen);
+static_assert(sizeof(WsHeader) <= 256, "the header fits its 256 bytes");
 
 // Most chunks (CTAs of the layout kernel) a layout uses.
 constexpr int kMaxChunks = 256;
@@ -73,9 +83,9 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline WsLayout ws_layout(int T, int K, int E, int A) {
     (void)K;
+    (void)T;
     WsLayout w;
     w.table_off = 256;
-    (void)T;
     w.padpre_off = round_up(w.table_off + (size_t)kMaxChunks * round4(E) * 4, 256);
     w.padrows_off = round_up(w.padpre_off + ((size_t)E + 1) * 4, 256);
     w.total = round_up(w.padrows_off + (size_t)E * (size_t)(A > 1 ? A - 1 : 0) * 4 + 4, 256);

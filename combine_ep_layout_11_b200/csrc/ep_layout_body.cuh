@@ -280,10 +280,17 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
         if (key >= 0 && lane == __ffs(peers) - 1) my[key] += __popc(peers);
         __syncwarp();
     };
-    // the first rounds load together and keep their expert ids in registers
+    // the first rounds load together and keep their expert ids (and the
+    // weights the assign writes) in registers
     int keys[kKeyRounds];
+    float wts[kKeyRounds];
 #pragma unroll
     for (int r = 0; r < kKeyRounds; ++r) keys[r] = load_key(q0 + 32 * r + lane);
+#pragma unroll
+    for (int r = 0; r < kKeyRounds; ++r) {
+        const int64_t i = q0 + 32 * r + lane;
+        wts[r] = (!kRankKeys && a.topk_weights && i < q1) ? a.topk_weights[i] : 1.0f;
+    }
 #pragma unroll
     for (int r = 0; r < kKeyRounds; ++r)
         if (q0 + 32 * r < q1) count_round(keys[r]);
@@ -333,11 +340,18 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
             for (int q = tid % cols; q < cols; q += (cols < NT ? cols : NT)) {
                 int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
                 const int4* col = reinterpret_cast<const int4*>(a.table) + q;
-#pragma unroll 8
-                for (int cc = c_lo; cc < c_hi; ++cc) {
-                    const int4 v = __ldcg(col + (size_t)cc * cols);
-                    tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
-                    if (cc < c) { pre.x += v.x; pre.y += v.y; pre.z += v.z; pre.w += v.w; }
+                // up to 16 rows in flight at once (a group's whole range when
+                // C <= 128 and E <= 256), then summed
+                for (int r0 = c_lo; r0 < c_hi; r0 += 16) {
+                    int4 v[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        v[i] = r0 + i < c_hi ? __ldcg(col + (size_t)(r0 + i) * cols) : make_int4(0, 0, 0, 0);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        tot.x += v[i].x; tot.y += v[i].y; tot.z += v[i].z; tot.w += v[i].w;
+                        if (r0 + i < c) { pre.x += v[i].x; pre.y += v[i].y; pre.z += v[i].z; pre.w += v[i].w; }
+                    }
                 }
                 reinterpret_cast<int4*>(dst_tot + g * Ep)[q] = tot;
                 reinterpret_cast<int4*>(dst_pre + g * Ep)[q] = pre;
@@ -411,7 +425,7 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     {
         const int El = E / a.R;
         const uint32_t lt = lanemask_lt();
-        auto assign_round = [&](int64_t qb, int key) {
+        auto assign_round = [&](int64_t qb, int key, float wt) {
             const int64_t i = qb + lane;
             const uint32_t peers = __match_any_sync(0xffffffffu, key);
             int slot = -1;
@@ -425,7 +439,7 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
                 a.pair_slot[i] = slot;
                 if (slot >= 0 && (int64_t)slot < a.capacity) {
                     a.recv_src[slot] = (int32_t)(i / K);
-                    a.recv_w[slot] = a.topk_weights ? a.topk_weights[i] : 1.0f;
+                    a.recv_w[slot] = wt;
                     a.recv_lexp[slot] = key % El;
                     if (kRankKeys) write_rank_row(a, i, slot);
                 }
@@ -433,11 +447,12 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
         };
 #pragma unroll
         for (int r = 0; r < kKeyRounds; ++r)
-            if (q0 + 32 * r < q1) assign_round(q0 + 32 * r, keys[r]);
+            if (q0 + 32 * r < q1) assign_round(q0 + 32 * r, keys[r], wts[r]);
         bool unused = false;
         for (int64_t qb = q0 + 32 * kKeyRounds; qb < q1; qb += 32) {
             const int64_t i = qb + lane;
-            assign_round(qb, (i < q1) ? pair_key<kRankKeys>(a, i, unused) : -1);
+            const float wt = (!kRankKeys && a.topk_weights && i < q1) ? a.topk_weights[i] : 1.0f;
+            assign_round(qb, (i < q1) ? pair_key<kRankKeys>(a, i, unused) : -1, wt);
         }
     }
 
