@@ -53,6 +53,9 @@ SIGNATURES = {
     "ep_combine": (_i, [_LP, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "ep_cast_fp8": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "ep_get_status": (_i, [_LP, _vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "ep_source_offsets": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i64, _vp]),
+    "ep_dispatch_regions": (_i, [_LP, _vp, _vp, _vp, _i64, _vp, _i, _vp, _i64, _vp]),
+    "ep_combine_regions": (_i, [_LP, _vp, _vp, _vp, _i64, _i, _vp, _vp, _vp]),
     "ep_selftest_bounded_wait": (_i, [_LP, _u64, _vp]),
     "ep_status_string": (ctypes.c_char_p, [_i]),
     "ep_version": (_i, []),

@@ -460,3 +460,83 @@ def get_status(lay):
 def selftest_bounded_wait(lay, timeout_ns):
     _check(_lib.load().ep_selftest_bounded_wait(lay.ref(), int(timeout_ns), _stream(lay.device)),
            "ep_selftest_bounded_wait")
+
+
+# --------------------------------------------------------------------------
+# Several source groups (GPUs): receive regions as separate buffers
+# --------------------------------------------------------------------------
+def source_offsets(counts, num_ranks, expert_alignment, group):
+    """Host side of a dispatch from several source groups (§2.1 across ranks).
+
+    ``counts``: host int32 [G, E], row g = source group g's per-expert pair
+    counts (what an all-gather of every group's ``num_recv_tokens_per_expert``
+    delivers).  Returns ``(row_delta, region_rows, pad_list)`` for ``group``:
+    int32 [E], int64 [R] and int64 [P] numpy arrays (see ep_source_offsets)."""
+    import numpy as np
+    L = _lib.load()
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    _require(counts.ndim == 2, "counts must be [G, E]")
+    G, E = counts.shape
+    delta = np.zeros(E, np.int32)
+    rows = np.zeros(max(num_ranks, 1), np.int64)
+    npad = ctypes.c_int64(0)
+    args = (ctypes.c_void_p(counts.ctypes.data), G, E, num_ranks, expert_alignment, group,
+            ctypes.c_void_p(delta.ctypes.data), ctypes.c_void_p(rows.ctypes.data))
+    _check(L.ep_source_offsets(*args, None, 0, ctypes.byref(npad)), "ep_source_offsets")
+    pads = np.zeros(max(npad.value, 1), np.int64)
+    _check(L.ep_source_offsets(*args, ctypes.c_void_p(pads.ctypes.data), npad.value, ctypes.byref(npad)),
+           "ep_source_offsets")
+    return delta, rows[:num_ranks], pads[:npad.value]
+
+
+def _region_table(regions, device, H=None):
+    """Device int64 array of the regions' addresses; every region a bf16 [capacity, H] tensor."""
+    _require(len(regions) > 0, "no regions")
+    cap = regions[0].shape[0]
+    for r in regions:
+        _check_tensor(r, "region", device, torch.bfloat16)
+        _require(r.dim() == 2 and r.shape[0] == cap and (H is None or r.shape[1] == H),
+                 "every region must be bf16 [capacity, H] with one capacity")
+    return torch.tensor([r.data_ptr() for r in regions], dtype=torch.int64, device=device), int(cap)
+
+
+def _check_region_call(lay, topk_idx, row_delta, regions):
+    _require(isinstance(lay, Layout) and lay.expert_alignment == 1, "needs a handle of ep_layout with alignment 1")
+    _require(len(regions) == lay.num_ranks, "one region per rank (%d)" % lay.num_ranks)
+    _check_tensor(topk_idx, "topk_idx", lay.device, torch.int64, (lay.num_tokens, lay.num_topk))
+    _check_tensor(row_delta, "row_delta", lay.device, torch.int32, (lay.num_experts,))
+
+
+def dispatch_regions(lay, topk_idx, row_delta, regions, x, pad_list=None):
+    """Write this group's bf16 rows into the ranks' regions (list of R bf16
+    [capacity, H] tensors); ``pad_list``: int64 device tensor of padding rows to
+    zero-fill, or None.  ``row_delta``: int32 [E] device tensor from
+    ``source_offsets``."""
+    L = _lib.load()
+    _check_region_call(lay, topk_idx, row_delta, regions)
+    _check_tensor(x, "x", lay.device, torch.bfloat16, (lay.num_tokens, x.shape[-1] if x.dim() == 2 else -1))
+    table, cap = _region_table(regions, lay.device, x.shape[1])
+    n = 0
+    if pad_list is not None:
+        _check_tensor(pad_list, "pad_list", lay.device, torch.int64)
+        n = pad_list.numel()
+    _check(L.ep_dispatch_regions(lay.ref(), _ptr(topk_idx), _ptr(row_delta), _ptr(table), cap, _ptr(x),
+                                 x.shape[1], _ptr(pad_list) if n else None, n, _stream(lay.device)),
+           "ep_dispatch_regions")
+
+
+def combine_regions(lay, topk_idx, row_delta, regions, topk_weights=None, out=None):
+    """Ordered combine of this group's tokens, the rows read from the regions
+    (expert outputs, R bf16 [capacity, H] tensors).  Returns bf16 [T, H]."""
+    L = _lib.load()
+    _check_region_call(lay, topk_idx, row_delta, regions)
+    table, cap = _region_table(regions, lay.device)
+    H = regions[0].shape[1]
+    if topk_weights is not None:
+        _check_tensor(topk_weights, "topk_weights", lay.device, torch.float32, (lay.num_tokens, lay.num_topk))
+    if out is None:
+        out = torch.empty((lay.num_tokens, H), dtype=torch.bfloat16, device=lay.device)
+    _check_tensor(out, "out", lay.device, torch.bfloat16, (lay.num_tokens, H))
+    _check(L.ep_combine_regions(lay.ref(), _ptr(topk_idx), _ptr(row_delta), _ptr(table), cap, H,
+                                _ptr(topk_weights), _ptr(out), _stream(lay.device)), "ep_combine_regions")
+    return out

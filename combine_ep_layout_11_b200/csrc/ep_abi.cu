@@ -94,7 +94,7 @@ int prepare_layout(const int64_t* topk_idx, const float* topk_weights, int T, in
 
 // A layout of zero tokens: no kernels, just zero counts and offsets.
 int empty_layout(ep_layout_t* layout, cudaStream_t s) {
-    if (cudaMemsetAsync(layout->workspace, 0, sizeof(ep::WsHeader), s) != cudaSuccess ||
+    if (cudaMemsetAsync(layout->workspace, 0, ep::kHeaderClearBytes, s) != cudaSuccess ||
         cudaMemsetAsync(layout->num_recv_tokens_per_expert, 0, (size_t)layout->num_experts * 4, s) != cudaSuccess ||
         cudaMemsetAsync(layout->expert_offset, 0, (size_t)(layout->num_experts + 1) * 4, s) != cudaSuccess)
         return EP_ERR_CUDA;
@@ -147,14 +147,14 @@ namespace ep {
 
 int layout_call(const int64_t* topk_idx, const float* topk_weights, int T, int K, int E, int R, int A,
                 int num_max_tokens_per_rank, ep_layout_t* layout, cudaStream_t s, bool clear_header) {
-    LayoutArgs a;
+    LayoutArgs a{};
     int rc = prepare_layout(topk_idx, topk_weights, T, K, E, R, A, num_max_tokens_per_rank, layout, &a);
     if (rc != EP_OK) return rc;
     if (T == 0) return empty_layout(layout, s);   // clears the header itself
     int sms = 0;
     if ((rc = device_sms(&sms)) != EP_OK) return rc;
     // only now, with every check passed, may the call touch the workspace
-    if (clear_header && cudaMemsetAsync(layout->workspace, 0, sizeof(WsHeader), s) != cudaSuccess)
+    if (clear_header && cudaMemsetAsync(layout->workspace, 0, kHeaderClearBytes, s) != cudaSuccess)
         return EP_ERR_CUDA;
     return launch_layout(a, sms, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
@@ -234,7 +234,7 @@ int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_t
     cudaStream_t s = (cudaStream_t)stream;
     uint8_t* wsb = reinterpret_cast<uint8_t*>(layout->workspace);
     if (T == 0) {
-        if (cudaMemsetAsync(layout->workspace, 0, sizeof(ep::WsHeader), s) != cudaSuccess ||
+        if (cudaMemsetAsync(layout->workspace, 0, ep::kHeaderClearBytes, s) != cudaSuccess ||
             cudaMemsetAsync(layout->num_recv_tokens_per_expert, 0, (size_t)R * 4, s) != cudaSuccess ||
             cudaMemsetAsync(layout->expert_offset, 0, (size_t)(R + 1) * 4, s) != cudaSuccess ||
             (num_tokens_per_expert && cudaMemsetAsync(num_tokens_per_expert, 0, (size_t)E * 4, s) != cudaSuccess) ||
@@ -243,7 +243,7 @@ int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_t
             return EP_ERR_CUDA;
         return EP_OK;
     }
-    ep::LayoutArgs la;
+    ep::LayoutArgs la{};
     la.topk_idx = nullptr;   // keys come from src_idx
     la.topk_weights = nullptr;
     la.T = T; la.K = R; la.E = R; la.R = R; la.A = 1;
@@ -301,7 +301,7 @@ int ep_ll_layout(const int64_t* topk_idx, const float* topk_weights, int num_tok
         ep_ll_workspace_bytes(num_tokens, num_topk, num_experts, num_ranks, M))
         return EP_ERR_INVALID_ARG;
     ep_layout_t tmp = *layout;   // the handle changes only once every check has passed
-    ep::LayoutArgs a;
+    ep::LayoutArgs a{};
     int rc = prepare_layout(topk_idx, topk_weights, num_tokens, num_topk, num_experts, num_ranks, 1, M, &tmp, &a);
     if (rc != EP_OK) return rc;
     a.slab = (int)slab;
@@ -316,7 +316,7 @@ int ep_ll_layout(const int64_t* topk_idx, const float* topk_weights, int num_tok
 
 int64_t ep_scale_bytes(int64_t rows, int hidden, int scale_format) {
     if (rows < 0 || hidden <= 0 || hidden % 128 != 0) return -1;
-    ep::DispatchArgs a;
+    ep::DispatchArgs a{};
     a.nb = hidden / 128;
     if (!ep::set_scale_format(&a, scale_format, rows)) return -1;
     return (a.sf_col_major ? a.sf_ld : rows) * a.ng * a.sf_elem;
@@ -325,7 +325,7 @@ int64_t ep_scale_bytes(int64_t rows, int hidden, int scale_format) {
 int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales, int hidden,
                 int cast_to_fp8, int scale_format, int do_zero_padding, void* recv_x, void* recv_scales,
                 void* stream) {
-    ep::DispatchArgs a;
+    ep::DispatchArgs a{};
     int elem_bytes = 0;
     int rc = prepare_dispatch(layout, x, x_dtype, x_scales, hidden, cast_to_fp8, scale_format, do_zero_padding,
                               recv_x, recv_scales, &a, &elem_bytes);
@@ -344,8 +344,8 @@ int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int n
                        void* stream) {
     if (!layout) return EP_ERR_INVALID_ARG;
     ep_layout_t tmp = *layout;   // the handle changes only once every check has passed
-    ep::LayoutArgs la;
-    ep::DispatchArgs da;
+    ep::LayoutArgs la{};
+    ep::DispatchArgs da{};
     int elem_bytes = 0;
     int rc = prepare_layout(topk_idx, topk_weights, num_tokens, num_topk, num_experts, num_ranks,
                             expert_alignment, num_max_tokens_per_rank, &tmp, &la);
@@ -379,7 +379,7 @@ int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float
         !aligned(bias1, 16))
         return EP_ERR_INVALID_ARG;
     if (T == 0) return EP_OK;
-    ep::CombineArgs a;
+    ep::CombineArgs a{};
     a.y = reinterpret_cast<const uint16_t*>(y);
     a.pair_slot = layout->pair_slot;
     a.w = topk_weights;
@@ -395,6 +395,79 @@ int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float
     return ep::launch_combine(a, (cudaStream_t)stream) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
+// Checks shared by the two region calls: an expand handle of alignment 1 and
+// the routing it was made from.
+static int check_region_handle(const ep_layout_t* layout, const int64_t* topk_idx, const int32_t* row_delta,
+                               const void* regions, int64_t region_capacity) {
+    int rc = check_handle(layout);
+    if (rc != EP_OK) return rc;
+    if (layout->kind != EP_LAYOUT_EXPAND || layout->expert_alignment != 1) return EP_ERR_INVALID_ARG;
+    if (region_capacity < 0) return EP_ERR_INVALID_ARG;
+    if (layout->num_tokens > 0 && (!topk_idx || !row_delta || !regions)) return EP_ERR_INVALID_ARG;
+    if (!aligned(topk_idx, 8) || !aligned(row_delta, 4) || !aligned(regions, 8)) return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+int ep_dispatch_regions(const ep_layout_t* layout, const int64_t* topk_idx, const int32_t* row_delta,
+                        void* const* regions, int64_t region_capacity, const void* x, int hidden,
+                        const int64_t* pad_list, int64_t num_pad, void* stream) {
+    int rc = check_region_handle(layout, topk_idx, row_delta, regions, region_capacity);
+    if (rc != EP_OK) return rc;
+    if (num_pad < 0 || (num_pad > 0 && (!pad_list || !regions)) || !aligned(pad_list, 8)) return EP_ERR_INVALID_ARG;
+    const int T = layout->num_tokens, H = hidden;
+    if (H <= 0 || H % 8 != 0 || (T > 0 && !x) || !aligned(x, 16)) return EP_ERR_INVALID_ARG;
+    ep::DispatchArgs a{};
+    a.x = reinterpret_cast<const uint8_t*>(x);
+    a.pair_slot = layout->pair_slot;
+    a.hdr = header(layout);
+    a.status_hdr = header(layout);
+    a.T = T;
+    a.K = layout->num_topk;
+    a.H = H;
+    a.capacity = 0;            // no single receive buffer
+    a.zero_pad = num_pad > 0 ? 1 : 0;
+    if ((rc = device_sms(&a.sms)) != EP_OK) return rc;
+    a.topk_idx = topk_idx;
+    a.row_delta = row_delta;
+    a.regions = reinterpret_cast<uint8_t* const*>(regions);
+    a.region_capacity = region_capacity;
+    a.R = layout->num_ranks;
+    a.El = layout->num_experts / layout->num_ranks;
+    a.pad_list = pad_list;
+    a.num_pad_list = num_pad;
+    if (layout->num_tokens == 0 && num_pad == 0) return EP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    return ep::launch_dispatch_copy(a, 2, s, true) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+int ep_combine_regions(const ep_layout_t* layout, const int64_t* topk_idx, const int32_t* row_delta,
+                       const void* const* regions, int64_t region_capacity, int hidden, const float* topk_weights,
+                       void* out, void* stream) {
+    int rc = check_region_handle(layout, topk_idx, row_delta, regions, region_capacity);
+    if (rc != EP_OK) return rc;
+    const int H = hidden, T = layout->num_tokens;
+    if (H <= 0 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (T > 0 && !out) return EP_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || !aligned(topk_weights, 4)) return EP_ERR_INVALID_ARG;
+    if (T == 0) return EP_OK;
+    ep::CombineArgs a{};
+    a.pair_slot = layout->pair_slot;
+    a.w = topk_weights;
+    a.out = reinterpret_cast<uint16_t*>(out);
+    a.T = T;
+    a.K = layout->num_topk;
+    a.H = H;
+    a.status = header(layout);
+    a.topk_idx = topk_idx;
+    a.row_delta = row_delta;
+    a.regions = reinterpret_cast<const uint16_t* const*>(regions);
+    a.region_capacity = region_capacity;
+    a.R = layout->num_ranks;
+    a.El = layout->num_experts / layout->num_ranks;
+    if ((rc = device_sms(&a.sms)) != EP_OK) return rc;
+    return ep::launch_combine(a, (cudaStream_t)stream) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
 int ep_cast_fp8(const void* x, int num_tokens, int hidden, int scale_format, void* x_fp8, void* scales,
                 void* stream) {
     const int T = num_tokens, H = hidden;
@@ -404,7 +477,7 @@ int ep_cast_fp8(const void* x, int num_tokens, int hidden, int scale_format, voi
     if (!aligned(x, 16) || !aligned(x_fp8, 16) || !aligned(scales, 16)) return EP_ERR_INVALID_ARG;
     if (ep_scale_bytes(T, H, scale_format) < 0) return EP_ERR_INVALID_ARG;
     if (T == 0) return EP_OK;
-    ep::DispatchArgs a;
+    ep::DispatchArgs a{};
     a.x = reinterpret_cast<const uint8_t*>(x);
     a.x_scales = nullptr;
     a.recv = reinterpret_cast<uint8_t*>(x_fp8);

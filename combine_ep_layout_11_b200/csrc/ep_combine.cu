@@ -58,7 +58,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // V: 16-byte columns per lane per row (a row segment of V * 512 bytes per
 // item); KB: rows whose loads are issued together before they are summed;
 // kBias: the sum starts from the output bias (a.bias0 is set).
-template <int V, int kMinBlocks, int KB, bool kBias>
+// kRegions: the rows come from the regions of CombineArgs (ep_combine_regions),
+// each selected entry carrying its row's address instead of a receive row.
+template <int V, int kMinBlocks, int KB, bool kBias, bool kRegions = false>
 __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(CombineArgs a) {
     const int lane = threadIdx.x & 31;
     const int64_t gw = ((int64_t)blockIdx.x * kCombineThreads + threadIdx.x) >> 5;
@@ -73,40 +75,58 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
     pdl_launch_dependents();
 
     // the (slot, weight) of lane k for the warp's next item is loaded while the
-    // current item is processed, so no item starts with a dependent load
-    auto fetch = [&](int64_t it, int& slot, float& w) {
+    // current item is processed, so no item starts with a dependent load; with
+    // regions, also the address of the entry's row (slot then only marks it used)
+    auto fetch = [&](int64_t it, int& slot, float& w, const uint4*& rp) {
         slot = -1;
         w = 1.0f;
+        rp = nullptr;
         if (it < items && lane < K) {
             const int64_t t = it / nch;
             slot = a.pair_slot[t * K + lane];
             if (a.w) w = a.w[t * K + lane];
+            if (kRegions && slot >= 0) {
+                const int64_t e = a.topk_idx[t * K + lane];
+                const int64_t row = (e >= 0 && e < (int64_t)a.El * a.R) ? (int64_t)slot + a.row_delta[e] : -1;
+                if (row >= 0 && row < a.region_capacity)
+                    rp = reinterpret_cast<const uint4*>(a.regions[e / a.El]) + row * (a.H / 8);
+                slot = rp ? 0 : -1;
+            }
         }
     };
     int next_slot;
     float next_w;
-    fetch(gw, next_slot, next_w);
+    const uint4* next_rp;
+    fetch(gw, next_slot, next_w, next_rp);
     // per warp: the item's selected entries moved to the front, in ascending k
     __shared__ int2 packed[kCombineThreads / 32][32];
+    __shared__ const uint4* packed_rp[kRegions ? kCombineThreads / 32 : 1][32];
     int2* my_packed = packed[threadIdx.x >> 5];
+    const uint4** my_packed_rp = packed_rp[kRegions ? threadIdx.x >> 5 : 0];
     for (int64_t it = gw; it < items; it += nw) {
         const int64_t t = it / nch;
         const int ch = (int)(it % nch);
         int my_slot = next_slot;
         float my_w = next_w;
-        fetch(it + nw, next_slot, next_w);
-        if ((int64_t)my_slot >= a.capacity) my_slot = -1;
+        const uint4* my_rp = next_rp;
+        fetch(it + nw, next_slot, next_w, next_rp);
+        if (!kRegions && (int64_t)my_slot >= a.capacity) my_slot = -1;
         // compaction: lane k with a selected entry writes it to position
         // popc(selected below k); the loop below then runs over nsel entries
         // with no holes, in the same ascending-k order
         const uint32_t sel = __ballot_sync(0xffffffffu, lane < K && my_slot >= 0);
         const int nsel = __popc(sel);
-        if ((sel >> lane) & 1u) my_packed[__popc(sel & lanemask_lt())] = make_int2(my_slot, __float_as_int(my_w));
+        if ((sel >> lane) & 1u) {
+            const int pos = __popc(sel & lanemask_lt());
+            my_packed[pos] = make_int2(my_slot, __float_as_int(my_w));
+            if (kRegions) my_packed_rp[pos] = my_rp;
+        }
         __syncwarp();
         if (lane < nsel) {
             const int2 p = my_packed[lane];
             my_slot = p.x;
             my_w = __int_as_float(p.y);
+            if (kRegions) my_rp = my_packed_rp[lane];
         }
         __syncwarp();
         float acc[V][8];
@@ -135,13 +155,18 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
 #pragma unroll
             for (int kk = 0; kk < KB; ++kk) {
                 const int k = k0 + kk;
-                const int slot = __shfl_sync(0xffffffffu, my_slot, k & 31);
                 const bool use = k < nsel;
+                const uint4* row;
+                if (kRegions) {
+                    const uint64_t p = __shfl_sync(0xffffffffu, reinterpret_cast<uint64_t>(my_rp), k & 31);
+                    row = reinterpret_cast<const uint4*>(p);
+                } else {
+                    row = y + (int64_t)__shfl_sync(0xffffffffu, my_slot, k & 31) * HV;
+                }
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
                     const int col = ch * per_item + v * 32 + lane;
-                    rows[kk][v] = (use && col < HV) ? ld_stream_v4(y + (int64_t)slot * HV + col)
-                                                    : make_uint4(0, 0, 0, 0);
+                    rows[kk][v] = (use && col < HV) ? ld_stream_v4(row + col) : make_uint4(0, 0, 0, 0);
                 }
             }
             if (kBias && k0 == 0) {
@@ -192,7 +217,8 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
     // pairs measured on the prefill and decode workloads, expand and per-rank
     // handles, once the selected entries are packed (2-8 rows per batch,
     // 512 B - 4 KB per row and item)
-    auto kernel = a.bias0 ? combine_kernel<2, 2, 8, true> : combine_kernel<2, 2, 2, false>;
+    auto kernel = a.regions ? (a.bias0 ? combine_kernel<2, 2, 8, true, true> : combine_kernel<2, 2, 2, false, true>)
+                            : (a.bias0 ? combine_kernel<2, 2, 8, true> : combine_kernel<2, 2, 2, false>);
     int blocks_per_sm = 0;
     cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kernel, kCombineThreads, 0);
     if (err != cudaSuccess) return err;

@@ -7,6 +7,8 @@
 // through shared memory on the TMA engine: one bulk load per row segment into
 // a multi-stage ring guarded by mbarriers, then one bulk store per destination
 // row, issued by K different lanes so the K stores of a row go out together.
+// The copy kernel takes its rows by ticket from counters in the workspace, so
+// no SM idles while others finish a larger share.
 // Threads never touch the payload in the copy kernel; in the cast kernel they
 // read the staged bf16 row from shared memory, write the e4m3 row and its
 // scales to shared memory, and TMA stores those.
@@ -33,70 +35,167 @@ __device__ __forceinline__ void zero_smem(uint8_t* p, uint32_t bytes, int tid, i
 }
 
 // ---------------------------------------------------------------------------
-// Copy kernel: one warp per CTA, several CTAs per SM.
+// Copy kernel.  Work is handed out by tickets (atomic counters in the layout's
+// workspace header), not by a fixed stride: an ncu capture of a fixed split
+// showed the SMs active only 84 % of the kernel on average (some finished at
+// 67 %) while the rest worked through their share, so DRAM idled in the tail.
+// Two warps per CTA, several CTAs per SM:
+//   warp 0  token rows: a ring of `stages` row segments; it takes tickets
+//           (one row segment each) from tok_ticket, bulk-loads the segment
+//           and, once it lands, lanes k < K bulk-store it to receive rows
+//           pair_slot[t, k]; a stage is refilled once its stores have read it;
+//   warp 1  padding rows (do_zero_padding): bulk stores of a zeroed buffer of
+//           zero_bytes, 32 pieces per ticket from pad_ticket, concurrently
+//           with the token rows, so the zero writes fill the gaps of the copy
+//           stream instead of forming a tail of their own.
+// The CTA that finishes last resets the tickets for the next launch.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(32) dispatch_copy_kernel(DispatchArgs a, uint32_t row_bytes, uint32_t seg_bytes,
-                                                           int nseg, int stages) {
+constexpr int kCopyThreads = 64;
+constexpr uint32_t kZeroBytes = 2048;
+
+// After all of this CTA's work: count it finished; the last CTA of the grid
+// (every ticket drawn) sets the counters back to zero for the next launch.
+__device__ __forceinline__ void tickets_done(WsHeader* h) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&h->done, 1u) == gridDim.x - 1) {
+            h->tok_ticket = 0;
+            h->pad_ticket = 0;
+            __threadfence();
+            h->done = 0;
+        }
+    }
+}
+
+// kRegions: the destinations are rows of the regions in DispatchArgs (bf16
+// rows; ep_dispatch_regions) instead of the one receive buffer.
+template <bool kRegions>
+__device__ __forceinline__ uint8_t* region_row(const DispatchArgs& a, int64_t e, int32_t slot, uint32_t row_bytes) {
+    if (slot < 0 || e < 0 || e >= (int64_t)a.El * a.R) return nullptr;
+    const int64_t row = (int64_t)slot + a.row_delta[e];
+    if (row < 0 || row >= a.region_capacity) return nullptr;
+    return a.regions[e / a.El] + row * row_bytes;
+}
+
+template <bool kRegions>
+__global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArgs a, uint32_t row_bytes,
+                                                                     uint32_t seg_bytes, int nseg, int stages) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t stride = round_up_u32(seg_bytes, 128);
-    uint8_t* stage = smem;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stride);
-    int32_t* slots = reinterpret_cast<int32_t*>(full + stages);
-    const int lane = threadIdx.x;
+    uint8_t* ring = smem;
+    uint8_t* zero = ring + (size_t)stages * stride;
+    uint64_t* full = reinterpret_cast<uint64_t*>(zero + kZeroBytes);
+    uint8_t** dsts = reinterpret_cast<uint8_t**>(full + stages);     // [stages][32] (regions only)
+    int32_t* slots = reinterpret_cast<int32_t*>(dsts + (kRegions ? stages * 32 : 0));   // [stages][32]
+    uint32_t* stage_item = reinterpret_cast<uint32_t*>(slots + stages * 32);   // [stages]: item held
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int K = a.K;
+    WsHeader* h = a.status_hdr;
 
-    if (lane == 0) {
+    if (tid == 0) {
         for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
         fence_barrier_init();
     }
-    __syncwarp();
+    zero_smem(zero, kZeroBytes, tid, kCopyThreads);
+    __syncthreads();
     pdl_wait();
     pdl_launch_dependents();
 
-    const int64_t G = gridDim.x;
-    const int64_t items = (int64_t)a.T * nseg;
-    const int64_t first = blockIdx.x;
-    const int64_t n = first < items ? (items - first + G - 1) / G : 0;
+    if (warp == 1) {
+        // ---- padding rows: pieces of kZeroBytes, 32 per ticket ----
+        if (a.zero_pad) {
+            const uint32_t npiece = (row_bytes + kZeroBytes - 1) / kZeroBytes;
+            const int64_t pieces = (kRegions ? a.num_pad_list : (int64_t)a.hdr->num_pad) * npiece;
+            const int64_t tickets = (pieces + 31) / 32;
+            const uint32_t sf_bytes = (uint32_t)a.nb * 4u;   // e4m3 rows: their fp32 scale row
+            for (;;) {
+                uint32_t tk = 0;
+                if (lane == 0) tk = atomicAdd(&h->pad_ticket, 1u);
+                tk = __shfl_sync(0xffffffffu, tk, 0);
+                if ((int64_t)tk >= tickets) break;
+                const int64_t q = (int64_t)tk * 32 + lane;
+                if (q < pieces && kRegions) {
+                    const int64_t pr = q / npiece;
+                    const uint32_t off = (uint32_t)(q - pr * npiece) * kZeroBytes;
+                    const int64_t entry = a.pad_list[pr];
+                    const int64_t r = entry >> 32, row = entry & 0xffffffffll;
+                    if (r >= 0 && r < a.R && row < a.region_capacity)
+                        bulk_store(a.regions[r] + row * row_bytes + off, zero, min(kZeroBytes, row_bytes - off));
+                } else if (q < pieces) {
+                    const int64_t pr = q / npiece;
+                    const uint32_t off = (uint32_t)(q - pr * npiece) * kZeroBytes;
+                    const int32_t row = a.pad_rows[pr];
+                    if (row >= 0 && (int64_t)row < a.capacity) {
+                        bulk_store(a.recv + (int64_t)row * row_bytes + off, zero, min(kZeroBytes, row_bytes - off));
+                        if (a.recv_scales != nullptr && off == 0) {
+                            if (sf_bytes % 16u == 0 && sf_bytes <= kZeroBytes)
+                                bulk_store(a.recv_scales + (int64_t)row * a.nb, zero, sf_bytes);
+                            else
+                                for (int b = 0; b < a.nb; ++b) a.recv_scales[(int64_t)row * a.nb + b] = 0.0f;
+                        }
+                    }
+                }
+                bulk_commit();
+            }
+            bulk_wait_all<0>();
+        }
+        tickets_done(h);
+        return;
+    }
 
-    auto issue = [&](int64_t j) {
-        const int64_t item = first + j * G;
+    // ---- token rows: one ticket per (token, segment) item ----
+    const uint32_t items = (uint32_t)a.T * (uint32_t)nseg;
+    auto issue = [&](int s, uint32_t item) {
         const int64_t t = item / nseg;
         const uint32_t off = (uint32_t)(item % nseg) * seg_bytes;
         const uint32_t bytes = min(seg_bytes, row_bytes - off);
-        const int s = (int)(j % stages);
-        if (lane < K) slots[s * 32 + lane] = a.pair_slot[t * K + lane];
+        if (lane < K) {
+            const int32_t slot = a.pair_slot[t * K + lane];
+            if (kRegions) dsts[s * 32 + lane] = region_row<kRegions>(a, a.topk_idx[t * K + lane], slot, row_bytes);
+            else slots[s * 32 + lane] = slot;
+        }
         if (lane == 0) {
+            stage_item[s] = item;
             mbar_arrive_expect_tx(&full[s], bytes);
-            bulk_load(stage + (size_t)s * stride, a.x + t * row_bytes + off, bytes, &full[s]);
+            bulk_load(ring + (size_t)s * stride, a.x + t * row_bytes + off, bytes, &full[s]);
         }
     };
-
+    // the first `stages` tickets in one draw, then one ticket ahead of its use
+    uint32_t first = 0;
+    if (lane == 0) first = atomicAdd(&h->tok_ticket, (uint32_t)stages);
+    first = __shfl_sync(0xffffffffu, first, 0);
     int64_t issued = 0;
-    for (; issued < n && issued < stages; ++issued) issue(issued);
+    for (; issued < stages && first + issued < items; ++issued) issue((int)issued, first + (uint32_t)issued);
+    bool more = first + (uint32_t)stages < items;
+    uint32_t next = 0;
+    if (lane == 0 && more) next = atomicAdd(&h->tok_ticket, 1u);
 
-    for (int64_t j = 0; j < n; ++j) {
+    for (int64_t j = 0; j < issued; ++j) {
         const int s = (int)(j % stages);
         if (!mbar_wait(&full[s], (uint32_t)((j / stages) & 1))) {
             // A load never landed: report, wait a bounded time for the loads
             // still in flight so no copy outlives the CTA, and stop.
-            if (lane == 0) atomicOr(&a.status_hdr->status, kDevTimeout);
+            if (lane == 0) atomicOr(&h->status, kDevTimeout);
             for (int64_t jj = j + 1; jj < issued; ++jj)
                 mbar_wait(&full[jj % stages], (uint32_t)((jj / stages) & 1), 100000000ull);
-            bulk_wait_all<0>();
-            return;
+            break;
         }
         __syncwarp();
-        const int64_t item = first + j * G;
+        const uint32_t item = stage_item[s];
         const int64_t t = item / nseg;
         const int sg = (int)(item % nseg);
         const uint32_t off = (uint32_t)sg * seg_bytes;
         const uint32_t bytes = min(seg_bytes, row_bytes - off);
-        if (lane < K) {
+        if (lane < K && kRegions) {
+            uint8_t* dst = dsts[s * 32 + lane];
+            if (dst != nullptr) bulk_store(dst + off, ring + (size_t)s * stride, bytes);
+        } else if (lane < K) {
             const int32_t slot = slots[s * 32 + lane];
             if (slot >= 0 && (int64_t)slot < a.capacity)
-                bulk_store(a.recv + (int64_t)slot * row_bytes + off, stage + (size_t)s * stride, bytes);
+                bulk_store(a.recv + (int64_t)slot * row_bytes + off, ring + (size_t)s * stride, bytes);
         }
-        if (a.x_scales != nullptr && sg == 0) {
+        if (!kRegions && a.x_scales != nullptr && sg == 0) {
             // e4m3 input: carry the token's scale row to every destination
             for (int k = 0; k < K; ++k) {
                 const int32_t slot = slots[s * 32 + k];
@@ -107,31 +206,21 @@ __global__ void __launch_bounds__(32) dispatch_copy_kernel(DispatchArgs a, uint3
         }
         bulk_commit();
         // refill the stage of item j-1 (its stores have finished reading it)
-        if (j >= 1 && issued < n) {
+        if (j >= 1 && more) {
             bulk_wait_read<1>();
             __syncwarp();
-            issue(issued);
-            ++issued;
+            const uint32_t tk = __shfl_sync(0xffffffffu, next, 0);
+            if (tk < items) {
+                issue((int)((j - 1) % stages), tk);
+                ++issued;
+                if (lane == 0) next = atomicAdd(&h->tok_ticket, 1u);
+            } else {
+                more = false;
+            }
         }
     }
     bulk_wait_all<0>();
-
-    if (!a.zero_pad) return;
-    // padding rows: bulk stores from a zeroed stage
-    __syncwarp();
-    zero_smem(stage, stride, lane, 32);
-    __syncwarp();
-    const int64_t pitems = (int64_t)a.hdr->num_pad * nseg;
-    for (int64_t q = first * 32 + lane; q < pitems; q += G * 32) {
-        const int32_t row = a.pad_rows[q / nseg];
-        const uint32_t off = (uint32_t)(q % nseg) * seg_bytes;
-        if (row < 0 || (int64_t)row >= a.capacity) continue;
-        bulk_store(a.recv + (int64_t)row * row_bytes + off, stage, min(seg_bytes, row_bytes - off));
-        if (a.recv_scales != nullptr && off == 0)
-            for (int b = 0; b < a.nb; ++b) a.recv_scales[(int64_t)row * a.nb + b] = 0.0f;
-    }
-    bulk_commit();
-    bulk_wait_all<0>();
+    tickets_done(h);
 }
 
 // ---------------------------------------------------------------------------
@@ -215,9 +304,39 @@ __device__ __forceinline__ void copy_word(uint8_t* dst, const uint8_t* src, int 
         *dst = *src;
 }
 
+// Barrier 1 over the cast warps only (barrier 0, __syncthreads, also waits
+// for the padding warp and is used once, at the end).
+__device__ __forceinline__ void cast_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCastThreads) : "memory"); }
+__device__ __forceinline__ bool cast_sync_or(bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n"
+        " .reg .pred q, r;\n"
+        " setp.ne.u32 q, %1, 0;\n"
+        " bar.red.or.pred r, 1, %2, q;\n"
+        " selp.u32 %0, 1, 0, r;\n"
+        "}\n"
+        : "=r"(r)
+        : "r"((uint32_t)p), "n"(kCastThreads)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Cast warps 0..7 and one padding warp.  With a handle (a.status_hdr set) the
+// token rows come by ticket, as in the copy kernel, and the padding warp
+// zero-fills the padding rows and their scales meanwhile; the plain cast
+// (ep_cast_fp8: no workspace, no padding) takes rows blockIdx.x, + grid, ...
+// Warp 0 draws the items and issues every bulk copy; the item of each input
+// stage is published through the stage's mbarrier (a load completing it, or a
+// plain arrival with kNoItem when the work has run out).
 template <bool kPerRow, bool kPow2>
-__global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArgs a, int stages) {
+__global__ void __launch_bounds__(kCastThreads + 32) dispatch_cast_kernel(DispatchArgs a, int stages) {
     constexpr int kWarps = kCastThreads / 32;
+    constexpr uint32_t kNoItem = 0xffffffffu;
     extern __shared__ __align__(128) uint8_t smem[];
     const int H = a.H, nb = a.nb, K = a.K, ng = a.ng, elem = a.sf_elem;
     const uint32_t in_stride = round_up_u32(2u * H, 128);
@@ -225,9 +344,11 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
     const uint32_t out_stride = round_up_u32(out_bytes, 128);
     uint8_t* in = smem;
     uint8_t* out = smem + (size_t)stages * in_stride;
-    uint64_t* full = reinterpret_cast<uint64_t*>(out + 2 * (size_t)out_stride);
-    int32_t* slots = reinterpret_cast<int32_t*>(full + stages);
-    int32_t* oslots = slots + stages * 32;                         // [2][32] slots of each output stage
+    uint8_t* zero = out + 2 * (size_t)out_stride;                   // kZeroBytes of zeros
+    uint64_t* full = reinterpret_cast<uint64_t*>(zero + kZeroBytes);
+    int32_t* slots = reinterpret_cast<int32_t*>(full + stages);      // [stages][32]
+    uint32_t* stage_item = reinterpret_cast<uint32_t*>(slots + stages * 32);   // [stages]
+    int32_t* oslots = reinterpret_cast<int32_t*>(stage_item + stages);         // [2][32] slots of each output stage
     float* bmax = reinterpret_cast<float*>(oslots + 2 * 32);        // per-row scales: block maxima
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t* sf = reinterpret_cast<uint8_t*>(a.recv_scales);
@@ -235,48 +356,115 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
     const bool bulk_scales = !a.sf_col_major && (sf_row_bytes % 16u) == 0;
     const int sf_word = sf_row_bytes % 8u == 0 ? 8 : sf_row_bytes % 4u == 0 ? 4 : sf_row_bytes % 2u == 0 ? 2 : 1;
     const int sf_words = (int)sf_row_bytes / sf_word;
+    WsHeader* h = a.status_hdr;
+    const bool tickets = h != nullptr;
 
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
         fence_barrier_init();
     }
+    zero_smem(zero, kZeroBytes, tid, kCastThreads + 32);
     __syncthreads();
     pdl_wait();
     pdl_launch_dependents();
 
-    const int64_t G = gridDim.x;
-    const int64_t first = blockIdx.x;
-    const int64_t n = first < a.T ? (a.T - first + G - 1) / G : 0;
-
-    // warp 0 only
-    auto issue = [&](int64_t j) {
-        const int64_t t = first + j * G;
-        const int s = (int)(j % stages);
-        if (lane < K) slots[s * 32 + lane] = a.pair_slot ? a.pair_slot[t * K + lane] : (int32_t)t;
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&full[s], 2u * H);
-            bulk_load(in + (size_t)s * in_stride, a.x + t * 2 * H, 2u * H, &full[s]);
+    if (warp == kWarps) {
+        // ---- padding rows and their scales: pieces of kZeroBytes, 32 per ticket ----
+        if (tickets && a.zero_pad) {
+            const uint32_t npiece = ((uint32_t)H + kZeroBytes - 1) / kZeroBytes;
+            const int64_t pieces = (int64_t)a.hdr->num_pad * npiece;
+            const int64_t ntk = (pieces + 31) / 32;
+            for (;;) {
+                uint32_t tk = 0;
+                if (lane == 0) tk = atomicAdd(&h->pad_ticket, 1u);
+                tk = __shfl_sync(0xffffffffu, tk, 0);
+                if ((int64_t)tk >= ntk) break;
+                const int64_t q = (int64_t)tk * 32 + lane;
+                if (q < pieces) {
+                    const int64_t pr = q / npiece;
+                    const uint32_t off = (uint32_t)(q - pr * npiece) * kZeroBytes;
+                    const int32_t row = a.pad_rows[pr];
+                    if (row >= 0 && (int64_t)row < a.capacity) {
+                        bulk_store(a.recv + (int64_t)row * H + off, zero, min(kZeroBytes, (uint32_t)H - off));
+                        if (off == 0) {
+                            if (bulk_scales)
+                                bulk_store(sf + (int64_t)row * sf_row_bytes, zero, sf_row_bytes);
+                            else if (a.sf_col_major)
+                                for (int g = 0; g < ng; ++g) copy_scale(sf, sf_offset(a, row, g), zero, g, elem);
+                            else
+                                for (int wd = 0; wd < sf_words; ++wd)
+                                    copy_word(sf + (int64_t)row * sf_row_bytes + wd * sf_word, zero + wd * sf_word,
+                                              sf_word);
+                        }
+                    }
+                }
+                bulk_commit();
+            }
+            bulk_wait_all<0>();
         }
+        if (tickets) tickets_done(h);
+        else __syncthreads();
+        return;
+    }
+
+    // ---- token rows (cast warps) ----
+    const uint32_t items = (uint32_t)a.T;
+    const uint32_t G = gridDim.x;
+    // warp 0: the CTA's items.  Tickets: the first `stages` in one draw (plus
+    // one more, held in `next`), then one drawn ahead of each use.  Without a
+    // handle: blockIdx.x, blockIdx.x + G, ...
+    uint32_t next = 0, draws = 0;
+    auto draw = [&]() -> uint32_t {
+        if (!tickets) return blockIdx.x + (draws++) * G;
+        const uint32_t t = __shfl_sync(0xffffffffu, next, 0);
+        if (lane == 0) next = atomicAdd(&h->tok_ticket, 1u);
+        return t;
+    };
+    // fill stage s with `item`, or mark it the end of this CTA's work
+    auto issue = [&](int s, uint32_t item) {
+        if (item >= items) {
+            if (lane == 0) {
+                stage_item[s] = kNoItem;
+                mbar_arrive(&full[s]);
+            }
+            return false;
+        }
+        if (lane < K) slots[s * 32 + lane] = a.pair_slot ? a.pair_slot[(int64_t)item * K + lane] : (int32_t)item;
+        if (lane == 0) {
+            stage_item[s] = item;
+            mbar_arrive_expect_tx(&full[s], 2u * H);
+            bulk_load(in + (size_t)s * in_stride, a.x + (int64_t)item * 2 * H, 2u * H, &full[s]);
+        }
+        return true;
     };
 
-    int64_t issued = 0;
-    if (warp == 0)
-        for (; issued < n && issued < stages; ++issued) issue(issued);
+    bool more = true;   // warp 0: a refill may still find work
+    if (warp == 0) {
+        uint32_t first = 0;
+        if (tickets) {
+            if (lane == 0) first = atomicAdd(&h->tok_ticket, (uint32_t)stages + 1u);
+            first = __shfl_sync(0xffffffffu, first, 0);
+            next = first + (uint32_t)stages;
+        }
+        for (int s = 0; s < stages && more; ++s) more = issue(s, tickets ? first + (uint32_t)s : draw());
+    }
 
-    for (int64_t j = 0; j < n; ++j) {
+    for (int64_t j = 0;; ++j) {
         const int s = (int)(j % stages);
         const int o = (int)(j & 1);
         if (warp == 0) bulk_wait_read<1>();   // output stage o: stores of item j-2 done reading
         const bool landed = mbar_wait(&full[s], (uint32_t)((j / stages) & 1));
-        if (__syncthreads_or(!landed)) {
-            if (tid == 0 && a.status_hdr != nullptr) atomicOr(&a.status_hdr->status, kDevTimeout);
+        if (cast_sync_or(!landed)) {
+            if (tid == 0 && h != nullptr) atomicOr(&h->status, kDevTimeout);
             if (warp == 0) {
-                for (int64_t jj = j; jj < issued; ++jj)
+                for (int64_t jj = j; jj < j + stages; ++jj)
                     mbar_wait(&full[jj % stages], (uint32_t)((jj / stages) & 1), 100000000ull);
                 bulk_wait_all<0>();
             }
-            return;
+            break;
         }
+        const uint32_t item = stage_item[s];
+        if (item == kNoItem) break;
         const uint8_t* src = in + (size_t)s * in_stride;
         uint8_t* dst = out + (size_t)o * out_stride;
         uint8_t* dst_sf = dst + H;   // this row's ng scales, elem bytes each
@@ -285,7 +473,7 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
                 const float m = block_amax(*reinterpret_cast<const uint2*>(src + (size_t)b * 256 + lane * 8));
                 if (lane == 0) bmax[b] = m;
             }
-            __syncthreads();
+            cast_sync();
             float m = 0.0f;
             for (int b = lane; b < nb; b += 32) m = fmaxf(m, bmax[b]);
             const float sc = make_scale<kPow2>(warp_max(m));
@@ -302,12 +490,12 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
                 if (lane == 0) put_scale(dst_sf, b, sc, elem);
             }
         }
-        // column-major scales are stored by every warp below; they read the
-        // item's slots from oslots[o], a copy that the refill of input stage s
-        // cannot overwrite (it lives as long as output stage o)
+        // column-major scales are stored by every cast warp below; they read
+        // the item's slots from oslots[o], a copy that the refill of input
+        // stage s cannot overwrite (it lives as long as output stage o)
         if (a.sf_col_major && warp == 0 && lane < K) oslots[o * 32 + lane] = slots[s * 32 + lane];
         fence_proxy_async_smem();
-        __syncthreads();
+        cast_sync();
         if (a.sf_col_major) {
             for (int q = tid; q < K * ng; q += kCastThreads) {
                 const int k = q / ng, g = q - k * ng;
@@ -323,9 +511,7 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
                     if (bulk_scales) bulk_store(sf + (int64_t)slot * sf_row_bytes, dst_sf, sf_row_bytes);
                 }
             }
-            if (a.sf_col_major) {
-                // stored by all warps above
-            } else if (!bulk_scales) {
+            if (!a.sf_col_major && !bulk_scales) {
                 for (int q = lane; q < K * sf_words; q += 32) {
                     const int k = q / sf_words, wd = q - k * sf_words;
                     const int32_t slot = slots[s * 32 + k];
@@ -334,37 +520,15 @@ __global__ void __launch_bounds__(kCastThreads) dispatch_cast_kernel(DispatchArg
                 }
             }
             bulk_commit();
-            if (issued < n) {
+            if (more) {
                 __syncwarp();
-                issue(issued);   // into stage s: every thread finished reading it before the barrier
-                ++issued;
+                more = issue(s, draw());   // into stage s: every cast thread finished reading it before the barrier
             }
         }
     }
     if (warp == 0) bulk_wait_all<0>();
-
-    if (!a.zero_pad) return;
-    __syncthreads();
-    uint8_t* zero = out;   // output stage 0, zeroed: an e4m3 row of zeros followed by zero scales
-    zero_smem(zero, out_stride, tid, kCastThreads);
-    __syncthreads();
-    if (warp == 0) {
-        const int64_t npad = a.hdr->num_pad;
-        for (int64_t q = first * 32 + lane; q < npad; q += G * 32) {
-            const int32_t row = a.pad_rows[q];
-            if (row < 0 || (int64_t)row >= a.capacity) continue;
-            bulk_store(a.recv + (int64_t)row * H, zero, (uint32_t)H);
-            if (bulk_scales)
-                bulk_store(sf + (int64_t)row * sf_row_bytes, zero + H, sf_row_bytes);
-            else if (a.sf_col_major)
-                for (int g = 0; g < ng; ++g) copy_scale(sf, sf_offset(a, row, g), zero + H, g, elem);
-            else
-                for (int wd = 0; wd < sf_words; ++wd)
-                    copy_word(sf + (int64_t)row * sf_row_bytes + wd * sf_word, zero + H + wd * sf_word, sf_word);
-        }
-        bulk_commit();
-        bulk_wait_all<0>();
-    }
+    if (tickets) tickets_done(h);
+    else __syncthreads();
 }
 
 template <bool kPerRow, bool kPow2>
@@ -373,39 +537,41 @@ cudaError_t launch_cast_variant(const DispatchArgs& a, cudaStream_t s) {
     const uint32_t in_stride = round_up_u32(2u * a.H, 128);
     const uint32_t out_stride = round_up_u32((uint32_t)a.H + 4u * a.nb, 128);
     const int stages = 3;   // H <= 16384: at most 130 KB of stages
-    const size_t smem = (size_t)stages * in_stride + 2 * (size_t)out_stride + (size_t)stages * 8 +
-                        (size_t)stages * 32 * 4 + 2 * 32 * 4 + (size_t)a.nb * 4;
+    const size_t smem = (size_t)stages * in_stride + 2 * (size_t)out_stride + kZeroBytes + (size_t)stages * 8 +
+                        (size_t)stages * 33 * 4 + 2 * 32 * 4 + (size_t)a.nb * 4;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     int ctas_per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, kernel, kCastThreads, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, kernel, kCastThreads + 32, smem);
     if (err != cudaSuccess) return err;
     if (ctas_per_sm > 4) ctas_per_sm = 4;
     if (ctas_per_sm < 1) ctas_per_sm = 1;
-    return launch_pdl(kernel, dim3(a.sms * ctas_per_sm), dim3(kCastThreads), smem, s, false, a, stages);
+    return launch_pdl(kernel, dim3(a.sms * ctas_per_sm), dim3(kCastThreads + 32), smem, s, false, a, stages);
 }
 
 }  // namespace
 
-cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStream_t s) {
+cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStream_t s, bool regions) {
     const uint32_t row_bytes = (uint32_t)a.H * (uint32_t)elem_bytes;
     const int nseg = (int)((row_bytes + kMaxSegBytes - 1) / kMaxSegBytes);
     const uint32_t seg_bytes = round_up_u32((row_bytes + nseg - 1) / nseg, 16);
     const uint32_t stride = round_up_u32(seg_bytes, 128);
-    // about 56 KB of stages per CTA, 2..8 stages, 4 CTAs (warps) per SM
-    int stages = (int)((57344u + stride - 1) / stride);
-    stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
-    const size_t smem = (size_t)stages * stride + (size_t)stages * 8 + (size_t)stages * 32 * 4;
-    cudaError_t err =
-        cudaFuncSetAttribute(dispatch_copy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // three row stages of at most 16 KB, up to four CTAs per SM: a sweep of
+    // 2-4 stages, 3-4 CTAs per SM and 2-4 KB zero buffers on the prefill,
+    // large-prefill and decode workloads put every setting within 2 %
+    const int stages = 3;
+    const size_t smem = (size_t)stages * stride + kZeroBytes + (size_t)stages * 8 + (size_t)stages * 33 * 4 +
+                        (regions ? (size_t)stages * 32 * 8 : 0);
+    auto kernel = regions ? dispatch_copy_kernel<true> : dispatch_copy_kernel<false>;
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     int ctas_per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, dispatch_copy_kernel, 32, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, kernel, kCopyThreads, smem);
     if (err != cudaSuccess) return err;
     if (ctas_per_sm > 4) ctas_per_sm = 4;
     if (ctas_per_sm < 1) ctas_per_sm = 1;
     const int grid = a.sms * ctas_per_sm;
-    return launch_pdl(dispatch_copy_kernel, dim3(grid), dim3(32), smem, s, false, a, row_bytes, seg_bytes, nseg, stages);
+    return launch_pdl(kernel, dim3(grid), dim3(kCopyThreads), smem, s, false, a, row_bytes, seg_bytes, nseg, stages);
 }
 
 cudaError_t launch_dispatch_cast(const DispatchArgs& a, cudaStream_t s) {

@@ -73,14 +73,25 @@ struct DispatchArgs {
     int sf_elem;
     int sf_col_major;
     int64_t sf_ld;
+    // Regions (ep_dispatch_regions; bf16 rows): pair (t, k) with expert
+    // e = topk_idx[t, k] goes to regions[e / El], row pair_slot[t, k] +
+    // row_delta[e]; padding rows come from pad_list ((r << 32) | row).
+    const int64_t* topk_idx;
+    const int32_t* row_delta;
+    uint8_t* const* regions;
+    int64_t region_capacity;
+    int El, R;
+    const int64_t* pad_list;
+    int64_t num_pad_list;
 };
 
 // Fill the sf_* fields for `rows` output rows; returns false for an invalid
 // format (unknown bits, UE8M0 without power-of-two rounding).
 bool set_scale_format(DispatchArgs* a, int scale_format, int64_t rows);
 
-// bf16 -> bf16 or e4m3 -> e4m3 row scatter through TMA bulk copies.
-cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStream_t s);
+// bf16 -> bf16 or e4m3 -> e4m3 row scatter through TMA bulk copies; with
+// `regions`, bf16 rows into the regions of DispatchArgs.
+cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStream_t s, bool regions = false);
 // bf16 -> e4m3 scatter with the per-128-column cast fused in.
 cudaError_t launch_dispatch_cast(const DispatchArgs& a, cudaStream_t s);
 
@@ -98,6 +109,14 @@ struct CombineArgs {
     int T, K, H;
     int64_t capacity;
     int sms;
+    // Regions (ep_combine_regions): the row of pair (t, k) with expert
+    // e = topk_idx[t, k] is regions[e / El] row pair_slot[t, k] + row_delta[e]
+    // (rows below region_capacity); y and capacity are then unused.
+    const int64_t* topk_idx;
+    const int32_t* row_delta;
+    const uint16_t* const* regions;
+    int64_t region_capacity;
+    int El, R;
 };
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);

@@ -350,6 +350,68 @@ int ep_combine(const ep_layout_t* layout, const void* y, int hidden, const float
 int ep_cast_fp8(const void* x, int num_tokens, int hidden, int scale_format, void* x_fp8, void* scales,
                 void* stream);
 
+/*
+ * Expert parallelism over G source groups (one per GPU in a multi-GPU run),
+ * §2.1 dispatch() / §2.2 combine() across ranks: each group g runs ep_layout
+ * on its own tokens with expert_alignment 1; the groups exchange their
+ * per-expert counts (an all-gather of num_recv_tokens_per_expert); then every
+ * group writes its rows straight into the destination ranks' receive regions
+ * (separate buffers, one per rank: on several GPUs, peer pointers).  The
+ * regions then hold exactly the rows one ep_layout over the concatenated batch
+ * (group 0's tokens, then group 1's, ...) with alignment A would give, region r
+ * being that layout's rows [off[r*E/R], off[(r+1)*E/R]).
+ *
+ * ep_source_offsets (a pure host function): from counts, host int32 [G][E]
+ * (row g = group g's num_recv_tokens_per_expert), for group `group`:
+ *   row_delta    host int32 [E] out: group `group`'s pair (t, k) with expert e
+ *                goes to region e / (E/R), row pair_slot[t, k] + row_delta[e]
+ *                (pair_slot of its own alignment-1 ep_layout)
+ *   region_rows  host int64 [R] out or NULL: rows region r holds, padding included
+ *   pad_list     host int64 [pad_list_capacity] out or NULL: every padding row
+ *                of every region, (r << 32) | row, in ascending order
+ *   num_pad      out (required with pad_list): the number of padding rows
+ * Returns EP_ERR_CAPACITY (after filling what fits) when pad_list is too short,
+ * EP_ERR_UNSUPPORTED when the rows exceed 2^31 - 1.
+ */
+int ep_source_offsets(const int32_t* counts, int num_groups, int num_experts, int num_ranks, int expert_alignment,
+                      int group, int32_t* row_delta, int64_t* region_rows, int64_t* pad_list,
+                      int64_t pad_list_capacity, int64_t* num_pad);
+
+/*
+ * Dispatch of one source group's bf16 rows into the regions (§2.1).
+ *   layout         the group's handle from ep_layout with expert_alignment 1
+ *                  (EP_ERR_INVALID_ARG otherwise); its num_ranks R and
+ *                  num_experts E give the regions' experts (E/R each)
+ *   topk_idx       device int64 [T, K]: the routing that layout was made from
+ *   row_delta      device int32 [E]: ep_source_offsets' row_delta for this group
+ *   regions        device array of R device pointers, 16-byte aligned: region r's
+ *                  bf16 rows [region_capacity, H] (on several GPUs, peer memory
+ *                  mapped into this process)
+ *   region_capacity rows each region holds (at least ep_source_offsets'
+ *                  region_rows); a row at or past it is not written
+ *   x              device bf16 [T, H], 16-byte aligned; H % 8 == 0
+ *   pad_list, num_pad  device int64 [num_pad] ((r << 32) | row) or NULL / 0:
+ *                  the padding rows this call zero-fills (give them to one call,
+ *                  e.g. the last group's)
+ * Rows go out as TMA bulk stores from shared memory: plain stores, no
+ * multicast.  No kernel reads a region.  The handle's workspace serves the
+ * work tickets, so one call per handle at a time.
+ */
+int ep_dispatch_regions(const ep_layout_t* layout, const int64_t* topk_idx, const int32_t* row_delta,
+                        void* const* regions, int64_t region_capacity, const void* x, int hidden,
+                        const int64_t* pad_list, int64_t num_pad, void* stream);
+
+/*
+ * Combine of one source group's tokens from the regions (§2.2): as ep_combine,
+ * with the row of pair (t, k) read from region topk_idx[t, k] / (E/R), row
+ * pair_slot[t, k] + row_delta[topk_idx[t, k]] (rows at or past
+ * region_capacity are skipped).  Arguments as for ep_dispatch_regions and
+ * ep_combine (no biases); regions hold the expert outputs, bf16.
+ */
+int ep_combine_regions(const ep_layout_t* layout, const int64_t* topk_idx, const int32_t* row_delta,
+                       const void* const* regions, int64_t region_capacity, int hidden, const float* topk_weights,
+                       void* out, void* stream);
+
 /* Size of the library-owned workspace behind ep_layout_no_alloc. */
 #define EP_NO_ALLOC_SCRATCH_BYTES ((size_t)4 << 20)
 
