@@ -356,12 +356,17 @@ int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int n
     *layout = tmp;
     cudaStream_t s = (cudaStream_t)stream;
     if (num_tokens == 0) return empty_layout(layout, s);
-    cudaError_t err;
-    if (cast_to_fp8) {
-        err = ep::launch_layout(la, da.sms, s);
-        if (err == cudaSuccess) err = ep::launch_dispatch_cast(da, s);
-    } else {
-        err = ep::launch_layout_dispatch(la, da, elem_bytes, s);
+    // the layout kernel, then the dispatch kernel launched behind it; x is an
+    // input of this call, so the layout kernel has waited for its producer and
+    // the copy kernel may load its first rows while the layout runs
+    cudaError_t err = ep::launch_layout(la, da.sms, s);
+    if (err == cudaSuccess) {
+        if (cast_to_fp8) {
+            err = ep::launch_dispatch_cast(da, s);
+        } else {
+            da.early = 1;
+            err = ep::launch_dispatch_copy(da, elem_bytes, s);
+        }
     }
     return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }

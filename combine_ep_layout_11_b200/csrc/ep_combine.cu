@@ -71,8 +71,11 @@ __global__ void __launch_bounds__(kCombineThreads, kMinBlocks) combine_kernel(Co
     const int64_t items = (int64_t)a.T * nch;
     const int K = a.K;
     const uint4* y = reinterpret_cast<const uint4*>(a.y);
+    // the next grid in the stream is not let in early (no launch_dependents):
+    // its CTAs would sit resident beside this bandwidth-bound kernel, which
+    // measured slower (dispatch -> combine: 765 against 733 us per
+    // large-prefill step); it starts when this grid ends
     pdl_wait();
-    pdl_launch_dependents();
 
     // the (slot, weight) of lane k for the warp's next item is loaded while the
     // current item is processed, so no item starts with a dependent load; with

@@ -23,6 +23,7 @@ namespace {
 
 constexpr uint32_t kMaxSegBytes = 16384;   // one bulk copy per row segment
 constexpr int kCastThreads = 256;
+constexpr int kCastOutStages = 2;          // e4m3 rows (and their scales) in flight per cast CTA
 
 __host__ __device__ __forceinline__ uint32_t round_up_u32(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
@@ -99,8 +100,42 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
     }
     zero_smem(zero, kZeroBytes, tid, kCopyThreads);
     __syncthreads();
+
+    // token rows: one ticket per (token, segment) item; the row of a stage is
+    // loaded by load_row, its destinations by load_slots
+    const uint32_t items = (uint32_t)a.T * (uint32_t)nseg;
+    auto load_row = [&](int s, uint32_t item) {
+        const int64_t t = item / nseg;
+        const uint32_t off = (uint32_t)(item % nseg) * seg_bytes;
+        const uint32_t bytes = min(seg_bytes, row_bytes - off);
+        if (lane == 0) {
+            stage_item[s] = item;
+            mbar_arrive_expect_tx(&full[s], bytes);
+            bulk_load(ring + (size_t)s * stride, a.x + t * row_bytes + off, bytes, &full[s]);
+        }
+    };
+    auto load_slots = [&](int s, uint32_t item) {
+        const int64_t t = item / nseg;
+        if (lane < K) {
+            const int32_t slot = a.pair_slot[t * K + lane];
+            if (kRegions) dsts[s * 32 + lane] = region_row<kRegions>(a, a.topk_idx[t * K + lane], slot, row_bytes);
+            else slots[s * 32 + lane] = slot;
+        }
+    };
+    // the first `stages` tickets in one draw (the counters are not written by
+    // the preceding grid, and x is complete when a.early is set)
+    uint32_t first = 0;
+    int64_t issued = 0;
+    if (warp == 0) {
+        if (lane == 0) first = atomicAdd(&h->tok_ticket, (uint32_t)stages);
+        first = __shfl_sync(0xffffffffu, first, 0);
+        if (a.early)
+            for (; issued < stages && first + issued < items; ++issued) load_row((int)issued, first + (uint32_t)issued);
+    }
+    // no launch_dependents: a successor's CTAs resident beside this kernel
+    // slowed the step (765 against 733 us at large prefill); it starts when
+    // this grid ends
     pdl_wait();
-    pdl_launch_dependents();
 
     if (warp == 1) {
         // ---- padding rows: pieces of kZeroBytes, 32 per ticket ----
@@ -144,29 +179,17 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
         return;
     }
 
-    // ---- token rows: one ticket per (token, segment) item ----
-    const uint32_t items = (uint32_t)a.T * (uint32_t)nseg;
+    // ---- token rows (warp 0) ----
     auto issue = [&](int s, uint32_t item) {
-        const int64_t t = item / nseg;
-        const uint32_t off = (uint32_t)(item % nseg) * seg_bytes;
-        const uint32_t bytes = min(seg_bytes, row_bytes - off);
-        if (lane < K) {
-            const int32_t slot = a.pair_slot[t * K + lane];
-            if (kRegions) dsts[s * 32 + lane] = region_row<kRegions>(a, a.topk_idx[t * K + lane], slot, row_bytes);
-            else slots[s * 32 + lane] = slot;
-        }
-        if (lane == 0) {
-            stage_item[s] = item;
-            mbar_arrive_expect_tx(&full[s], bytes);
-            bulk_load(ring + (size_t)s * stride, a.x + t * row_bytes + off, bytes, &full[s]);
-        }
+        load_slots(s, item);
+        load_row(s, item);
     };
-    // the first `stages` tickets in one draw, then one ticket ahead of its use
-    uint32_t first = 0;
-    if (lane == 0) first = atomicAdd(&h->tok_ticket, (uint32_t)stages);
-    first = __shfl_sync(0xffffffffu, first, 0);
-    int64_t issued = 0;
-    for (; issued < stages && first + issued < items; ++issued) issue((int)issued, first + (uint32_t)issued);
+    if (a.early) {
+        for (int64_t j = 0; j < issued; ++j) load_slots((int)j, first + (uint32_t)j);
+    } else {
+        for (; issued < stages && first + issued < items; ++issued) issue((int)issued, first + (uint32_t)issued);
+    }
+    // then one ticket drawn ahead of its use
     bool more = first + (uint32_t)stages < items;
     uint32_t next = 0;
     if (lane == 0 && more) next = atomicAdd(&h->tok_ticket, 1u);
@@ -344,12 +367,12 @@ __global__ void __launch_bounds__(kCastThreads + 32) dispatch_cast_kernel(Dispat
     const uint32_t out_stride = round_up_u32(out_bytes, 128);
     uint8_t* in = smem;
     uint8_t* out = smem + (size_t)stages * in_stride;
-    uint8_t* zero = out + 2 * (size_t)out_stride;                   // kZeroBytes of zeros
+    uint8_t* zero = out + kCastOutStages * (size_t)out_stride;      // kZeroBytes of zeros
     uint64_t* full = reinterpret_cast<uint64_t*>(zero + kZeroBytes);
     int32_t* slots = reinterpret_cast<int32_t*>(full + stages);      // [stages][32]
     uint32_t* stage_item = reinterpret_cast<uint32_t*>(slots + stages * 32);   // [stages]
-    int32_t* oslots = reinterpret_cast<int32_t*>(stage_item + stages);         // [2][32] slots of each output stage
-    float* bmax = reinterpret_cast<float*>(oslots + 2 * 32);        // per-row scales: block maxima
+    int32_t* oslots = reinterpret_cast<int32_t*>(stage_item + stages);   // [kCastOutStages][32] slots per output stage
+    float* bmax = reinterpret_cast<float*>(oslots + kCastOutStages * 32);  // per-row scales: block maxima
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t* sf = reinterpret_cast<uint8_t*>(a.recv_scales);
     const uint32_t sf_row_bytes = (uint32_t)ng * (uint32_t)elem;
@@ -365,8 +388,7 @@ __global__ void __launch_bounds__(kCastThreads + 32) dispatch_cast_kernel(Dispat
     }
     zero_smem(zero, kZeroBytes, tid, kCastThreads + 32);
     __syncthreads();
-    pdl_wait();
-    pdl_launch_dependents();
+    pdl_wait();   // no launch_dependents, as in the copy kernel
 
     if (warp == kWarps) {
         // ---- padding rows and their scales: pieces of kZeroBytes, 32 per ticket ----
@@ -451,8 +473,9 @@ __global__ void __launch_bounds__(kCastThreads + 32) dispatch_cast_kernel(Dispat
 
     for (int64_t j = 0;; ++j) {
         const int s = (int)(j % stages);
-        const int o = (int)(j & 1);
-        if (warp == 0) bulk_wait_read<1>();   // output stage o: stores of item j-2 done reading
+        const int o = (int)(j % kCastOutStages);
+        // output stage o: the stores of item j - kCastOutStages are done reading it
+        if (warp == 0) bulk_wait_read<kCastOutStages - 1>();
         const bool landed = mbar_wait(&full[s], (uint32_t)((j / stages) & 1));
         if (cast_sync_or(!landed)) {
             if (tid == 0 && h != nullptr) atomicOr(&h->status, kDevTimeout);
@@ -537,8 +560,8 @@ cudaError_t launch_cast_variant(const DispatchArgs& a, cudaStream_t s) {
     const uint32_t in_stride = round_up_u32(2u * a.H, 128);
     const uint32_t out_stride = round_up_u32((uint32_t)a.H + 4u * a.nb, 128);
     const int stages = 3;   // H <= 16384: at most 130 KB of stages
-    const size_t smem = (size_t)stages * in_stride + 2 * (size_t)out_stride + kZeroBytes + (size_t)stages * 8 +
-                        (size_t)stages * 33 * 4 + 2 * 32 * 4 + (size_t)a.nb * 4;
+    const size_t smem = (size_t)stages * in_stride + kCastOutStages * (size_t)out_stride + kZeroBytes +
+                        (size_t)stages * 8 + (size_t)stages * 33 * 4 + kCastOutStages * 32 * 4 + (size_t)a.nb * 4;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     int ctas_per_sm = 0;

@@ -83,6 +83,11 @@ struct DispatchArgs {
     int El, R;
     const int64_t* pad_list;
     int64_t num_pad_list;
+    // Copy kernel: 1 when x is known to be complete before the grid that
+    // precedes the kernel has finished (ep_layout_dispatch: x is an input of
+    // the same call, so the layout kernel waited for its producer); the first
+    // row loads are then issued before waiting for that grid.
+    int early;
 };
 
 // Fill the sf_* fields for `rows` output rows; returns false for an invalid
@@ -95,8 +100,6 @@ cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStre
 // bf16 -> e4m3 scatter with the per-128-column cast fused in.
 cudaError_t launch_dispatch_cast(const DispatchArgs& a, cudaStream_t s);
 
-// Layout and bf16 / e4m3 row scatter in one cooperative kernel (ep_fused.cu).
-cudaError_t launch_layout_dispatch(LayoutArgs la, DispatchArgs da, int elem_bytes, cudaStream_t s);
 
 struct CombineArgs {
     const uint16_t* y;         // bf16 [capacity][H]

@@ -96,6 +96,12 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// 16-byte load through L2 only (the table rows were written by other CTAs).
+__device__ __forceinline__ int4 ld_cg_v4(const int4* p) {
+    int4 v;
+    asm volatile("ld.global.cg.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -343,12 +349,14 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
                 // up to 16 rows in flight at once (a group's whole range when
                 // C <= 128 and E <= 256), then summed
                 for (int r0 = c_lo; r0 < c_hi; r0 += 16) {
+                    // sixteen unconditional loads (rows past the range re-read
+                    // the last row and are dropped), issued back to back
                     int4 v[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        v[i] = r0 + i < c_hi ? __ldcg(col + (size_t)(r0 + i) * cols) : make_int4(0, 0, 0, 0);
+                    for (int i = 0; i < 16; ++i) v[i] = ld_cg_v4(col + (size_t)min(r0 + i, c_hi - 1) * cols);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
+                        if (r0 + i >= c_hi) continue;
                         tot.x += v[i].x; tot.y += v[i].y; tot.z += v[i].z; tot.w += v[i].w;
                         if (r0 + i < c) { pre.x += v[i].x; pre.y += v[i].y; pre.z += v[i].z; pre.w += v[i].w; }
                     }

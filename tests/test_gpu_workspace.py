@@ -65,7 +65,7 @@ def test_reused_workspace_across_inputs_and_zero_token_calls(ep):
         ref = oracle.layout(idx, w, E, R, A)
         check_layout(lay, ref)
         assert int(words[1]) == int(ref["off"][-1]) - int((idx >= 0).sum())   # num_pad
-        assert (words[2], words[3], words[4], words[5], words[6]) == (0, 0, 0, 0, 0)
+        assert (words[2:8] == 0).all()                    # pending, tickets, barrier count
         # a call with no tokens on the same handle: counts and offsets zeroed, generation kept
         rc = lib.ep_layout(None, None, 0, K, E, R, A, 0, lay.ref(), stream)
         assert rc == 0
@@ -111,8 +111,9 @@ def test_dispatch_tickets_reset(ep, fp8):
 
 
 def test_fused_call_advances_the_generation(ep):
-    """ep_layout_dispatch runs the same layout body: one generation per call,
-    tickets untouched (the fused kernel splits its work by chunk)."""
+    """ep_layout_dispatch runs the layout kernel and then the ticketed copy
+    kernel (whose first row loads start while the layout runs): one
+    generation per call, every ticket back at zero, the same bytes twice."""
     T, K, E, R, A, H = 2048, 8, 64, 4, 16, 512
     idx, w, x = _rand(T, K, E, H, 21)
     lay, recv = ep.layout_dispatch(to_dev(idx), to_dev(w), to_dev_bf16(x), E, R, A, do_zero_padding=True)
@@ -122,5 +123,5 @@ def test_fused_call_advances_the_generation(ep):
     assert np.array_equal(bf16_bits(recv[:Np]), oracle.dispatch_rows(x, ref, True)[:Np])
     lay2, recv2 = ep.layout_dispatch(to_dev(idx), to_dev(w), to_dev_bf16(x), E, R, A, do_zero_padding=True,
                                      out_layout=lay, out=recv)
-    assert _words(lay)[8] == 2 and (_words(lay)[2:7] == 0).all()
+    assert _words(lay)[8] == 2 and (_words(lay)[2:8] == 0).all()
     assert np.array_equal(bf16_bits(recv2[:Np]), oracle.dispatch_rows(x, ref, True)[:Np])
