@@ -111,10 +111,13 @@ def test_shapes_fp8(ep, T, K, E, R, A, H, fused):
     _full(ep, idx, w, x, E, R, A, fp8=True, fused=fused)
 
 
+@pytest.mark.parametrize("H", [1024, 640, 128], ids=["sf32B", "sf20B", "sf4B"])
 @pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
-def test_fp8_input_passthrough(ep, fused):
-    """(e4m3, scales) input is dispatched as is: rows and scale rows move together."""
-    T, K, E, R, A, H = 200, 8, 64, 4, 16, 1024
+def test_fp8_input_passthrough(ep, fused, H):
+    """(e4m3, scales) input is dispatched as is: rows and scale rows move together.
+    The padding rows' scales are zeroed by a bulk store when the scale row is a
+    multiple of 16 bytes (H = 1024: 32 B), else by plain stores (20 B, 4 B)."""
+    T, K, E, R, A = 200, 8, 64, 4, 16
     idx, w, x = _rand(T, K, E, H, seed=11)
     q, s = oracle.cast_fp8(x)
     ref = oracle.layout(idx, w, E, R, A)

@@ -96,3 +96,43 @@ def test_regions_reject_an_aligned_handle(ep):
     delta = torch.zeros(cfg["E"], dtype=torch.int32, device=DEV)
     with pytest.raises(ep.EpError):
         ep.dispatch_regions(lay, idx, delta, regions, to_dev_bf16(inp["x"]))
+
+
+def test_regions_with_two_segment_rows(ep):
+    """bf16 rows of 32 KB (H = 16384) travel as two bulk segments; padding
+    rows are zeroed in 2 KB pieces; G = 3 groups of ragged sizes."""
+    rng = np.random.default_rng(5)
+    T, K, E, R, A, H = 96, 4, 16, 4, 8, 16384
+    idx_h = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int64)
+    idx_h[rng.random(idx_h.shape) < 0.15] = -1
+    w_h = rng.random((T, K)).astype(np.float32)
+    x_h = workload.to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
+    ref = oracle.layout(idx_h, w_h, E, R, A)
+    off = ref["off"].astype(np.int64)
+    El = E // R
+    cuts = [0, 40, 44, 96]                     # groups of 40, 4 and 52 tokens
+    groups = []
+    for g in range(3):
+        sl = slice(cuts[g], cuts[g + 1])
+        idx, w = to_dev(idx_h[sl]), to_dev(w_h[sl])
+        groups.append((sl, idx, w, to_dev_bf16(x_h[sl]), ep.layout(idx, w, E, R, 1)))
+    counts = np.stack([lay.num_recv_tokens_per_expert.cpu().numpy() for (_, _, _, _, lay) in groups])
+    offs = [ep.source_offsets(counts, R, A, g) for g in range(3)]
+    cap = int(offs[0][1].max())
+    regions = [torch.full((cap, H), 7.0, dtype=torch.bfloat16, device=DEV) for _ in range(R)]
+    for g, (sl, idx, w, x, lay) in enumerate(groups):
+        pads = offs[g][2]
+        ep.dispatch_regions(lay, idx, to_dev(offs[g][0]), regions, x, pad_list=to_dev(pads) if g == 0 else None)
+    torch.cuda.synchronize()
+    exp = oracle.dispatch_rows(x_h, ref, True)
+    for r in range(R):
+        lo, hi = int(off[r * El]), int(off[(r + 1) * El])
+        assert np.array_equal(bf16_bits(regions[r][:hi - lo]), exp[lo:hi]), "region %d" % r
+    y = workload.expert_outputs(dict(seed=9, H=H), int(off[-1]))
+    yreg = [torch.zeros((cap, H), dtype=torch.bfloat16, device=DEV) for _ in range(R)]
+    for r in range(R):
+        lo, hi = int(off[r * El]), int(off[(r + 1) * El])
+        yreg[r][:hi - lo] = to_dev_bf16(y[lo:hi])
+    for g, (sl, idx, w, x, lay) in enumerate(groups):
+        out = ep.combine_regions(lay, idx, to_dev(offs[g][0]), yreg, w)
+        assert np.array_equal(bf16_bits(out), oracle.combine(y, ref["pair_slot"][sl], w_h[sl]))
