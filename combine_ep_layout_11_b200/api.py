@@ -489,33 +489,52 @@ def source_offsets(counts, num_ranks, expert_alignment, group):
     return delta, rows[:num_ranks], pads[:npad.value]
 
 
-def _region_table(regions, device, H=None):
-    """Device int64 array of the regions' addresses; every region a bf16 [capacity, H] tensor."""
-    _require(len(regions) > 0, "no regions")
-    cap = regions[0].shape[0]
-    for r in regions:
-        _check_tensor(r, "region", device, torch.bfloat16)
-        _require(r.dim() == 2 and r.shape[0] == cap and (H is None or r.shape[1] == H),
-                 "every region must be bf16 [capacity, H] with one capacity")
-    return torch.tensor([r.data_ptr() for r in regions], dtype=torch.int64, device=device), int(cap)
+class RegionTable:
+    """The regions of a dispatch / combine across source groups: R bf16
+    [capacity, H] tensors of one capacity and width, and the device array of
+    their addresses the kernels index.  Build it once and pass it to every
+    call (``dispatch_regions`` / ``combine_regions`` also take the list and
+    build a table per call, which costs a host-to-device copy)."""
+
+    def __init__(self, regions):
+        _require(len(regions) > 0, "no regions")
+        device = regions[0].device
+        cap, H = regions[0].shape[0], regions[0].shape[-1]
+        for r in regions:
+            _check_tensor(r, "region", device, torch.bfloat16)
+            _require(r.dim() == 2 and tuple(r.shape) == (cap, H),
+                     "every region must be bf16 [capacity, H] with one capacity and width")
+        self.regions = list(regions)         # kept alive with the table
+        self.device = device
+        self.capacity, self.hidden = int(cap), int(H)
+        self.table = torch.tensor([r.data_ptr() for r in regions], dtype=torch.int64, device=device)
+
+    def __len__(self):
+        return len(self.regions)
 
 
-def _check_region_call(lay, topk_idx, row_delta, regions):
+def _region_table(regions):
+    return regions if isinstance(regions, RegionTable) else RegionTable(regions)
+
+
+def _check_region_call(lay, topk_idx, row_delta, table):
     _require(isinstance(lay, Layout) and lay.expert_alignment == 1, "needs a handle of ep_layout with alignment 1")
-    _require(len(regions) == lay.num_ranks, "one region per rank (%d)" % lay.num_ranks)
+    _require(len(table) == lay.num_ranks, "one region per rank (%d)" % lay.num_ranks)
+    _require(table.device == lay.device, "the regions are on another device")
     _check_tensor(topk_idx, "topk_idx", lay.device, torch.int64, (lay.num_tokens, lay.num_topk))
     _check_tensor(row_delta, "row_delta", lay.device, torch.int32, (lay.num_experts,))
 
 
 def dispatch_regions(lay, topk_idx, row_delta, regions, x, pad_list=None):
-    """Write this group's bf16 rows into the ranks' regions (list of R bf16
-    [capacity, H] tensors); ``pad_list``: int64 device tensor of padding rows to
-    zero-fill, or None.  ``row_delta``: int32 [E] device tensor from
-    ``source_offsets``."""
+    """Write this group's bf16 rows into the ranks' regions (a ``RegionTable``,
+    or a list of R bf16 [capacity, H] tensors); ``pad_list``: int64 device
+    tensor of padding rows to zero-fill, or None.  ``row_delta``: int32 [E]
+    device tensor from ``source_offsets``."""
     L = _lib.load()
-    _check_region_call(lay, topk_idx, row_delta, regions)
-    _check_tensor(x, "x", lay.device, torch.bfloat16, (lay.num_tokens, x.shape[-1] if x.dim() == 2 else -1))
-    table, cap = _region_table(regions, lay.device, x.shape[1])
+    rt = _region_table(regions)
+    _check_region_call(lay, topk_idx, row_delta, rt)
+    _check_tensor(x, "x", lay.device, torch.bfloat16, (lay.num_tokens, rt.hidden))
+    table, cap = rt.table, rt.capacity
     n = 0
     if pad_list is not None:
         _check_tensor(pad_list, "pad_list", lay.device, torch.int64)
@@ -527,11 +546,12 @@ def dispatch_regions(lay, topk_idx, row_delta, regions, x, pad_list=None):
 
 def combine_regions(lay, topk_idx, row_delta, regions, topk_weights=None, out=None):
     """Ordered combine of this group's tokens, the rows read from the regions
-    (expert outputs, R bf16 [capacity, H] tensors).  Returns bf16 [T, H]."""
+    (expert outputs: a ``RegionTable`` or a list of R bf16 [capacity, H]
+    tensors).  Returns bf16 [T, H]."""
     L = _lib.load()
-    _check_region_call(lay, topk_idx, row_delta, regions)
-    table, cap = _region_table(regions, lay.device)
-    H = regions[0].shape[1]
+    rt = _region_table(regions)
+    _check_region_call(lay, topk_idx, row_delta, rt)
+    table, cap, H = rt.table, rt.capacity, rt.hidden
     if topk_weights is not None:
         _check_tensor(topk_weights, "topk_weights", lay.device, torch.float32, (lay.num_tokens, lay.num_topk))
     if out is None:

@@ -180,9 +180,11 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
     }
 
     // ---- token rows (warp 0) ----
+    // the row's bulk load goes out first: it does not need the slots, which
+    // are read only when the row has landed
     auto issue = [&](int s, uint32_t item) {
-        load_slots(s, item);
         load_row(s, item);
+        load_slots(s, item);
     };
     if (a.early) {
         for (int64_t j = 0; j < issued; ++j) load_slots((int)j, first + (uint32_t)j);

@@ -51,11 +51,12 @@ def _run(ep, name, G, pad_on_last=True):
     rows = offs[0][1]
     cap = int(rows.max()) + 3
     regions = [torch.full((cap, H), -1.0, dtype=torch.bfloat16, device=DEV) for _ in range(R)]
+    table = ep.RegionTable(regions)          # built once, used by every group's call
     for g, (sl, idx, w, x, lay) in enumerate(groups):
         delta, rows_g, pads = offs[g]
         assert np.array_equal(rows_g, rows)
         last = g == G - 1
-        ep.dispatch_regions(lay, idx, to_dev(delta), regions, x,
+        ep.dispatch_regions(lay, idx, to_dev(delta), table, x,
                             pad_list=to_dev(pads) if (last and pad_on_last and len(pads)) else None)
     torch.cuda.synchronize()
     exp = oracle.dispatch_rows(x_h, ref, True)
