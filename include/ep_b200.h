@@ -302,9 +302,12 @@ int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const flo
  * Layout and dispatch in one call, as V2's dispatch() derives its layout from
  * topk_idx itself (§2.1; §3.1's V1/V2 comparison).  Arguments and results are
  * exactly those of ep_layout followed by ep_dispatch on the same handle; the
- * handle is then reusable by ep_combine and by further ep_dispatch calls.  One
- * kernel for bf16 or e4m3 input (its token-row reads overlap the layout work);
- * with cast_to_fp8 the layout and the casting dispatch run as two kernels.
+ * handle is then reusable by ep_combine and by further ep_dispatch calls.  Two
+ * kernels: the layout, then the dispatch, launched behind it with programmatic
+ * dependent launch.  x is an input of this call, so x must be complete when
+ * the call is made (as for every input).  For bf16 or e4m3 rows, the dispatch
+ * kernel may then load its first rows of x while the layout kernel still
+ * runs.
  */
 int ep_layout_dispatch(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,
                        int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,

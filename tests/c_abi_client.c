@@ -10,9 +10,12 @@
  * [T, K]), <dir>/x.bin (bf16 bits [T, H]) and <dir>/y.bin (bf16 bits
  * [capacity, H], the expert outputs).  Runs ep_layout, ep_dispatch (zero
  * padding) and ep_combine (weighted) on a caller-allocated workspace, then
- * ep_layout_no_alloc on the same inputs, and writes pair_slot.bin,
- * expert_offset.bin, recv.bin (the first expert_offset[E] rows), out.bin and
- * pair_slot_no_alloc.bin.  Exit status 0 on success; any library or CUDA
+ * ep_layout_no_alloc on the same inputs, then one source group into R
+ * separately allocated regions (ep_layout with alignment 1,
+ * ep_source_offsets, ep_dispatch_regions with the padding list,
+ * ep_combine_regions), and writes pair_slot.bin, expert_offset.bin, recv.bin
+ * (the first expert_offset[E] rows), out.bin, pair_slot_no_alloc.bin,
+ * regions.bin (the regions' rows one after the other) and out_regions.bin.  Exit status 0 on success; any library or CUDA
  * error prints its status string and exits 1.
  */
 #include <cuda_runtime_api.h>
@@ -157,6 +160,64 @@ int main(int argc, char** argv)
     check_ep(ep_get_status(&lay2, NULL, &flags), "ep_get_status (no-alloc)");
     check_cuda(cudaMemcpy(h_slot, lay2.pair_slot, (size_t)T * K * 4, cudaMemcpyDeviceToHost), "D2H slots 2");
     write_file(dir, "pair_slot_no_alloc.bin", h_slot, (size_t)T * K * 4);
+
+    /* one source group into R separately allocated regions: an alignment-1
+       layout of the same tokens, the offsets from its counts, then dispatch
+       and combine over a device table of region addresses */
+    ep_layout_t lay3 = lay;
+    const int64_t cap1 = ep_capacity_rows(T, K, E, 1);
+    lay3.pair_slot = (int32_t*)dev_alloc((size_t)T * K * 4);
+    lay3.num_recv_tokens_per_expert = (int32_t*)dev_alloc((size_t)E * 4);
+    lay3.expert_offset = (int32_t*)dev_alloc((size_t)(E + 1) * 4);
+    lay3.recv_src_token = (int32_t*)dev_alloc((size_t)cap1 * 4);
+    lay3.recv_weight = (float*)dev_alloc((size_t)cap1 * 4);
+    lay3.recv_local_expert = (int32_t*)dev_alloc((size_t)cap1 * 4);
+    lay3.capacity = cap1;
+    lay3.workspace_bytes = ep_workspace_bytes(T, K, E, 1);
+    lay3.workspace = dev_alloc(lay3.workspace_bytes);
+    check_cuda(cudaMemset(lay3.workspace, 0, lay3.workspace_bytes), "workspace 3 zero-fill");
+    check_ep(ep_layout(d_idx, d_w, T, K, E, R, 1, 0, &lay3, NULL), "ep_layout (alignment 1)");
+    int32_t* h_cnt = (int32_t*)malloc((size_t)E * 4);
+    check_cuda(cudaMemcpy(h_cnt, lay3.num_recv_tokens_per_expert, (size_t)E * 4, cudaMemcpyDeviceToHost), "D2H cnt");
+    int32_t* h_delta = (int32_t*)malloc((size_t)E * 4);
+    int64_t* h_rows = (int64_t*)malloc((size_t)R * 8);
+    int64_t npad = 0;
+    check_ep(ep_source_offsets(h_cnt, 1, E, R, A, 0, h_delta, h_rows, NULL, 0, &npad), "ep_source_offsets");
+    int64_t* h_pads = (int64_t*)malloc((size_t)(npad > 0 ? npad : 1) * 8);
+    check_ep(ep_source_offsets(h_cnt, 1, E, R, A, 0, h_delta, h_rows, h_pads, npad, &npad), "ep_source_offsets");
+    int64_t rcap = 1;
+    for (int r = 0; r < R; ++r) rcap = h_rows[r] > rcap ? h_rows[r] : rcap;
+    void** h_reg = (void**)malloc((size_t)R * sizeof(void*));
+    void** h_yreg = (void**)malloc((size_t)R * sizeof(void*));
+    int64_t base = 0;
+    for (int r = 0; r < R; ++r) {
+        h_reg[r] = dev_alloc((size_t)rcap * H * 2);
+        h_yreg[r] = dev_alloc((size_t)rcap * H * 2);
+        /* the expert outputs of region r: its rows of the single receive order */
+        check_cuda(cudaMemcpy(h_yreg[r], h_y + (size_t)base * H, (size_t)h_rows[r] * H * 2, cudaMemcpyHostToDevice),
+                   "H2D y region");
+        base += h_rows[r];
+    }
+    void* d_reg = dev_copy(h_reg, (size_t)R * sizeof(void*));
+    void* d_yreg = dev_copy(h_yreg, (size_t)R * sizeof(void*));
+    void* d_delta = dev_copy(h_delta, (size_t)E * 4);
+    void* d_pads = dev_copy(h_pads, (size_t)(npad > 0 ? npad : 1) * 8);
+    void* d_out2 = dev_alloc((size_t)T * H * 2);
+    check_ep(ep_dispatch_regions(&lay3, d_idx, (const int32_t*)d_delta, (void* const*)d_reg, rcap, d_x, H,
+                                 (const int64_t*)d_pads, npad, NULL), "ep_dispatch_regions");
+    check_ep(ep_combine_regions(&lay3, d_idx, (const int32_t*)d_delta, (const void* const*)d_yreg, rcap, H, d_w,
+                                d_out2, NULL), "ep_combine_regions");
+    check_ep(ep_get_status(&lay3, NULL, &flags), "ep_get_status (regions)");
+    uint16_t* h_regs = (uint16_t*)malloc((size_t)(base > 0 ? base : 1) * H * 2);
+    int64_t at = 0;
+    for (int r = 0; r < R; ++r) {
+        check_cuda(cudaMemcpy(h_regs + (size_t)at * H, h_reg[r], (size_t)h_rows[r] * H * 2, cudaMemcpyDeviceToHost),
+                   "D2H region");
+        at += h_rows[r];
+    }
+    write_file(dir, "regions.bin", h_regs, (size_t)base * H * 2);
+    check_cuda(cudaMemcpy(h_out, d_out2, (size_t)T * H * 2, cudaMemcpyDeviceToHost), "D2H out 2");
+    write_file(dir, "out_regions.bin", h_out, (size_t)T * H * 2);
 
     printf("ok rows=%lld\n", (long long)rows);
     return 0;

@@ -1,7 +1,7 @@
 """The C ABI from a plain C program (tests/c_abi_client.c: no torch, device
 memory from cudaMalloc): ep_layout, ep_dispatch with zero padding, the weighted
-ep_combine and ep_layout_no_alloc on seeded inputs, every result compared with
-the oracle ("DeepEP 测试目标 API 系统性参考" §2.1 / §2.2)."""
+ep_combine, ep_layout_no_alloc and the region calls of one source group on
+seeded inputs, every result compared with the oracle ("DeepEP 测试目标 API 系统性参考" §2.1 / §2.2)."""
 import os
 import subprocess
 
@@ -52,3 +52,8 @@ def test_c_client_matches_oracle(client, tmp_path, T, K, E, R, A, H):
     assert np.array_equal(out, oracle.combine(y, ref["pair_slot"], w))
     slots2 = np.fromfile(str(tmp_path / "pair_slot_no_alloc.bin"), np.int32).reshape(T, K)
     assert np.array_equal(slots2, ref["pair_slot"])
+    # the regions, one after the other, are the receive rows; their combine is the same
+    regions = np.fromfile(str(tmp_path / "regions.bin"), np.uint16).reshape(Np, H)
+    assert np.array_equal(regions, oracle.dispatch_rows(x, ref, True)[:Np])
+    out2 = np.fromfile(str(tmp_path / "out_regions.bin"), np.uint16).reshape(T, H)
+    assert np.array_equal(out2, oracle.combine(y, ref["pair_slot"], w))
