@@ -47,8 +47,10 @@ int prepare_layout(const int64_t* topk_idx, const float* topk_weights, int T, in
         !aligned(layout->recv_local_expert, 4) || !aligned(layout->workspace, 256) ||
         !aligned(layout->cumulative_local_expert_recv_stats, 4))
         return EP_ERR_INVALID_ARG;
+    // the layout's own part is the minimum; the scale staging area behind it
+    // is optional (see prepare_dispatch)
     const ep::WsLayout ws = ep::ws_layout(T, K, E, A);
-    if (layout->workspace_bytes < ws.total) return EP_ERR_INVALID_ARG;
+    if (layout->workspace_bytes < ws.base_total) return EP_ERR_INVALID_ARG;
 
     layout->num_tokens = T;
     layout->num_topk = K;
@@ -137,6 +139,16 @@ int prepare_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, cons
     a->nb = fp8_out ? H / 128 : 0;
     a->zero_pad = do_zero_padding ? 1 : 0;
     if (!ep::set_scale_format(a, scale_format, layout->capacity)) return EP_ERR_INVALID_ARG;
+    // column-major per-block scales go through the staging area when the
+    // handle's workspace holds it (per-row scales are K words per token: one
+    // store each is cheaper than a second kernel)
+    if (cast_to_fp8 && a->sf_col_major && a->ng > 1 && layout->kind == EP_LAYOUT_EXPAND &&
+        layout->workspace_bytes >= ws.total) {
+        a->sf_stage = reinterpret_cast<uint8_t*>(layout->workspace) + ws.stage_off;
+        a->sf_stage_ld = (int64_t)ep::round_up((size_t)a->ng * a->sf_elem, 16);
+        a->recv_src = layout->recv_src_token;
+        a->num_rows = layout->expert_offset + layout->num_experts;
+    }
     *elem_bytes = fp8_in ? 1 : 2;
     return device_sms(&a->sms);
 }
@@ -287,7 +299,7 @@ size_t ep_ll_workspace_bytes(int num_tokens, int num_topk, int num_experts, int 
     const int64_t slab = (int64_t)num_ranks * num_max_dispatch_tokens_per_rank;
     if (slab > INT_MAX - 1) return 0;
     // the padding-row list holds up to E * slab rows: the expand sizing with A = slab + 1
-    return ep::ws_layout(num_tokens, num_topk, num_experts, (int)(slab + 1)).total;
+    return ep::ws_layout(num_tokens, num_topk, num_experts, (int)(slab + 1)).base_total;
 }
 
 int ep_ll_layout(const int64_t* topk_idx, const float* topk_weights, int num_tokens, int num_topk,

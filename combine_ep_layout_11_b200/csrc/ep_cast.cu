@@ -125,7 +125,7 @@ __device__ __forceinline__ bool cast_sync_or(bool p) {
 // stage is published through the stage's mbarrier (a load completing it, or a
 // plain arrival with kNoItem when the work has run out).
 template <bool kPerRow, bool kPow2>
-__global__ void __launch_bounds__(kCastThreads + 32) dispatch_cast_kernel(DispatchArgs a, int stages) {
+__global__ void __launch_bounds__(kCastThreads + 32, 4) dispatch_cast_kernel(DispatchArgs a, int stages) {
     constexpr int kWarps = kCastThreads / 32;
     constexpr uint32_t kNoItem = 0xffffffffu;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -149,6 +149,8 @@ __global__ void __launch_bounds__(kCastThreads + 32) dispatch_cast_kernel(Dispat
     const int sf_words = (int)sf_row_bytes / sf_word;
     WsHeader* h = a.status_hdr;
     const bool tickets = h != nullptr;
+    uint8_t* const sf_stage = a.sf_stage;
+    const bool scattered_sf = a.sf_col_major && sf_stage == nullptr;
 
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
@@ -179,8 +181,10 @@ __global__ void __launch_bounds__(kCastThreads + 32) dispatch_cast_kernel(Dispat
                         if (off == 0) {
                             if (bulk_scales)
                                 bulk_store(sf + (int64_t)row * sf_row_bytes, zero, sf_row_bytes);
-                            else if (a.sf_col_major)
-                                for (int g = 0; g < ng; ++g) copy_scale(sf, sf_offset(a, row, g), zero, g, elem);
+                            else if (a.sf_col_major) {
+                                if (scattered_sf)   // staged: the second kernel writes them
+                                    for (int g = 0; g < ng; ++g) copy_scale(sf, sf_offset(a, row, g), zero, g, elem);
+                            }
                             else
                                 for (int wd = 0; wd < sf_words; ++wd)
                                     copy_word(sf + (int64_t)row * sf_row_bytes + wd * sf_word, zero + wd * sf_word,
@@ -281,13 +285,13 @@ __global__ void __launch_bounds__(kCastThreads + 32) dispatch_cast_kernel(Dispat
                 if (lane == 0) put_scale(dst_sf, b, sc, elem);
             }
         }
-        // column-major scales are stored by every cast warp below; they read
-        // the item's slots from oslots[o], a copy that the refill of input
-        // stage s cannot overwrite (it lives as long as output stage o)
-        if (a.sf_col_major && warp == 0 && lane < K) oslots[o * 32 + lane] = slots[s * 32 + lane];
+        // unstaged column-major scales are stored by every cast warp below;
+        // they read the item's slots from oslots[o], a copy that the refill of
+        // input stage s cannot overwrite (it lives as long as output stage o)
+        if (scattered_sf && warp == 0 && lane < K) oslots[o * 32 + lane] = slots[s * 32 + lane];
         fence_proxy_async_smem();
         cast_sync();
-        if (a.sf_col_major) {
+        if (scattered_sf) {
             for (int q = tid; q < K * ng; q += kCastThreads) {
                 const int k = q / ng, g = q - k * ng;
                 const int32_t slot = oslots[o * 32 + k];
@@ -302,6 +306,11 @@ __global__ void __launch_bounds__(kCastThreads + 32) dispatch_cast_kernel(Dispat
                     if (bulk_scales) bulk_store(sf + (int64_t)slot * sf_row_bytes, dst_sf, sf_row_bytes);
                 }
             }
+            // staged column-major scales: the token's scale row, once (the
+            // bytes past ng * elem up to the 16-byte stride are not read back)
+            // (stage_item[s] still holds the item: the refill comes below)
+            if (sf_stage != nullptr && lane == 0)
+                bulk_store(sf_stage + (int64_t)stage_item[s] * a.sf_stage_ld, dst_sf, (uint32_t)a.sf_stage_ld);
             if (!a.sf_col_major && !bulk_scales) {
                 for (int q = lane; q < K * sf_words; q += 32) {
                     const int k = q / sf_words, wd = q - k * sf_words;
@@ -320,6 +329,45 @@ __global__ void __launch_bounds__(kCastThreads + 32) dispatch_cast_kernel(Dispat
     if (warp == 0) bulk_wait_all<0>();
     if (tickets) tickets_done(h);
     else __syncthreads();
+}
+
+// Column-major scales from the staging area: thread i takes receive row i
+// (grid-stride) and writes its ng scales, so each store instruction of a warp
+// covers 32 consecutive rows of one scale column (128 bytes of fp32, 32 of
+// UE8M0) instead of 32 scattered words.  Padding rows (recv_src < 0) get zero
+// scales when the dispatch zero-fills padding, and are left alone otherwise.
+__global__ void __launch_bounds__(256) scale_colmajor_kernel(DispatchArgs a) {
+    pdl_wait();   // the cast kernel's staged rows and the layout's recv_src
+    const int64_t n = *a.num_rows;
+    const int64_t rows = n < a.capacity ? n : a.capacity;
+    const int ng = a.ng, elem = a.sf_elem;
+    const int chunks = (int)(a.sf_stage_ld / 16);
+    uint8_t* sf = reinterpret_cast<uint8_t*>(a.recv_scales);
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; row < rows; row += stride) {
+        const int32_t src = a.recv_src[row];
+        const bool real = src >= 0 && src < a.T;
+        if (!real && !a.zero_pad) continue;
+        const uint4* staged = reinterpret_cast<const uint4*>(a.sf_stage + (real ? (int64_t)src * a.sf_stage_ld : 0));
+#pragma unroll 2
+        for (int c = 0; c < chunks; ++c) {
+            const uint4 v = real ? staged[c] : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            if (elem == 4) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int g = c * 4 + j;
+                    if (g < ng) reinterpret_cast<uint32_t*>(sf)[(int64_t)g * a.sf_ld + row] = w[j];
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int g = c * 16 + j;
+                    if (g < ng) sf[(int64_t)g * a.sf_ld + row] = (uint8_t)(w[j >> 2] >> (8 * (j & 3)));
+                }
+            }
+        }
+    }
 }
 
 template <bool kPerRow, bool kPow2>
@@ -347,8 +395,15 @@ cudaError_t launch_cast_variant(const DispatchArgs& a, cudaStream_t s) {
 
 cudaError_t launch_dispatch_cast(const DispatchArgs& a, cudaStream_t s) {
     const bool per_row = (a.sf_format & EP_SF_PER_ROW) != 0, pow2 = (a.sf_format & EP_SF_POW2) != 0;
-    if (per_row) return pow2 ? launch_cast_variant<true, true>(a, s) : launch_cast_variant<true, false>(a, s);
-    return pow2 ? launch_cast_variant<false, true>(a, s) : launch_cast_variant<false, false>(a, s);
+    cudaError_t err;
+    if (per_row) err = pow2 ? launch_cast_variant<true, true>(a, s) : launch_cast_variant<true, false>(a, s);
+    else err = pow2 ? launch_cast_variant<false, true>(a, s) : launch_cast_variant<false, false>(a, s);
+    if (err != cudaSuccess || a.sf_stage == nullptr) return err;
+    // one thread per receive row, at most eight CTAs of 256 per SM (grid-stride beyond)
+    int64_t ctas = (a.capacity + 255) / 256;
+    if (ctas > (int64_t)a.sms * 8) ctas = (int64_t)a.sms * 8;
+    if (ctas < 1) ctas = 1;
+    return launch_pdl(scale_colmajor_kernel, dim3((unsigned)ctas), dim3(256), 0, s, false, a);
 }
 
 bool set_scale_format(DispatchArgs* a, int scale_format, int64_t rows) {

@@ -72,23 +72,30 @@ inline Chunking chunking(int T, int K, int max_chunks, int target_pairs) {
 
 __host__ __device__ inline int round4(int x) { return (x + 3) / 4 * 4; }
 
+// Bytes per token of the scale staging area: one row of up to 128 fp32
+// scales (H <= 16384 for the cast).
+constexpr size_t kStageRowBytes = 512;
+
 struct WsLayout {
     size_t table_off;    // int32 [kMaxChunks][round4(E)]: per-chunk expert counts
     size_t padpre_off;   // int32 [E+1]: exclusive prefix of padding rows per expert
     size_t padrows_off;  // int32 [E*(A-1)]: receive row of every padding row
-    size_t total;
+    size_t base_total;   // what the layout itself needs
+    size_t stage_off;    // [T][kStageRowBytes]: the FP8 dispatch's per-token scale rows
+    size_t total;        // with the staging area
 };
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline WsLayout ws_layout(int T, int K, int E, int A) {
     (void)K;
-    (void)T;
     WsLayout w;
     w.table_off = 256;
     w.padpre_off = round_up(w.table_off + (size_t)kMaxChunks * round4(E) * 4, 256);
     w.padrows_off = round_up(w.padpre_off + ((size_t)E + 1) * 4, 256);
-    w.total = round_up(w.padrows_off + (size_t)E * (size_t)(A > 1 ? A - 1 : 0) * 4 + 4, 256);
+    w.base_total = round_up(w.padrows_off + (size_t)E * (size_t)(A > 1 ? A - 1 : 0) * 4 + 4, 256);
+    w.stage_off = w.base_total;
+    w.total = w.stage_off + (size_t)(T > 0 ? T : 0) * kStageRowBytes;
     return w;
 }
 

@@ -73,6 +73,17 @@ struct DispatchArgs {
     int sf_elem;
     int sf_col_major;
     int64_t sf_ld;
+    // Column-major scales through the staging area of an expand handle's
+    // workspace (when it holds one): the cast kernel bulk-stores each token's
+    // scale row to sf_stage + t * sf_stage_ld, then a second kernel writes the
+    // column-major array receive row by receive row, scale (row, g) =
+    // staged[recv_src[row]][g] (zero for padding rows), so that a warp's
+    // stores cover consecutive rows.  nullptr: one store per scale from the
+    // cast kernel.
+    uint8_t* sf_stage;
+    int64_t sf_stage_ld;
+    const int32_t* recv_src;
+    const int32_t* num_rows;   // device word: receive rows in use (expert_offset[E])
     // Regions (ep_dispatch_regions; bf16 rows): pair (t, k) with expert
     // e = topk_idx[t, k] goes to regions[e / El], row pair_slot[t, k] +
     // row_delta[e]; padding rows come from pad_list ((r << 32) | row).

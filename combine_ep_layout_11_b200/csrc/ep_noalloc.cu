@@ -46,8 +46,10 @@ int ep_layout_no_alloc(const int64_t* topk_idx, const float* topk_weights, int n
                        int num_experts, int num_ranks, int expert_alignment, int num_max_tokens_per_rank,
                        ep_layout_t* layout, void* stream) {
     if (!layout) return EP_ERR_INVALID_ARG;
-    const size_t need = ep_workspace_bytes(num_tokens, num_topk, num_experts, expert_alignment);
-    if (need == 0) return EP_ERR_INVALID_ARG;
+    if (ep_workspace_bytes(num_tokens, num_topk, num_experts, expert_alignment) == 0) return EP_ERR_INVALID_ARG;
+    // the layout's own part; the dispatch uses the scale staging area behind
+    // it only where the array has room for it
+    const size_t need = ep::ws_layout(num_tokens, num_topk, num_experts, expert_alignment).base_total;
     if (need > kStaticScratchBytes) return EP_ERR_UNSUPPORTED;
     void* ws = nullptr;
     int rc = scratch_address(&ws);

@@ -32,7 +32,7 @@ RankWsLayout rank_ws_layout(int T, int R, int E) {
     RankWsLayout w;
     w.expand = ws_layout(T, R, R, 1);
     const size_t n = (size_t)(T > 0 ? T : 0) * (size_t)R;
-    w.scratch_w_off = w.expand.total;
+    w.scratch_w_off = w.expand.base_total;
     w.scratch_lexp_off = round_up(w.scratch_w_off + n * 4, 256);
     w.counts_off = round_up(w.scratch_lexp_off + n * 4, 256);
     w.total = round_up(w.counts_off + (size_t)E * 4, 256);

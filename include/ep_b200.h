@@ -135,7 +135,13 @@ extern "C" {
  *   workspace                  ep_workspace_bytes() bytes, 256-byte aligned,
  *                              zero-filled by the caller before its first use
  *                              (every later ep_layout leaves it ready again);
- *                              holds the device status word and scan scratch.
+ *                              holds the device status word and scan scratch,
+ *                              and last a staging area of 512 bytes per token
+ *                              for ep_dispatch's column-major FP8 scales.  A
+ *                              workspace of ep_workspace_bytes() - 512 * T
+ *                              bytes (the layout's own part) is accepted too:
+ *                              ep_dispatch then stores column-major scales one
+ *                              by one, which is slower (see ep_dispatch).
  *                              One workspace serves one call at a time.
  *   cumulative_local_expert_recv_stats [E] int32 or NULL (§2.1 dispatch() and
  *                              §3.3 low_latency_dispatch() argument of that
@@ -173,7 +179,8 @@ typedef struct ep_layout_t {
 #define EP_LAYOUT_PER_RANK 1   /* ep_rank_layout: one row per (token, rank) reached */
 #define EP_LAYOUT_LL_SLAB 2    /* ep_ll_layout: a fixed slab of rows per expert */
 
-/* Bytes of workspace ep_layout needs for these sizes (a pure host function). */
+/* Bytes of workspace for these sizes: the layout's own part plus the
+ * 512-byte-per-token scale staging area (a pure host function). */
 size_t ep_workspace_bytes(int num_tokens, int num_topk, int num_experts, int expert_alignment);
 
 /* Worst-case receive rows: T*K + E*(A-1); a capacity of this many rows can
@@ -293,6 +300,13 @@ int ep_ll_layout(const int64_t* topk_idx, const float* topk_weights, int num_tok
  *                [capacity, H/128] for FP8 input, else ep_scale_bytes(capacity,
  *                H, scale_format) bytes in that format; ignored for bf16 output
  * Rows that no pair selects and that are not padding are left untouched.
+ * One kernel, except for column-major per-block scales (EP_SF_COL_MAJOR
+ * without EP_SF_PER_ROW) on an ep_layout / ep_layout_no_alloc handle whose
+ * workspace holds the staging area: the cast kernel then stages each token's
+ * scale row once, and a second kernel writes the column-major array receive
+ * row by receive row, so that neighbouring threads store neighbouring rows.
+ * Otherwise each of the K * H/128 scales of a token is one store.  Both write
+ * the same bytes.
  */
 int ep_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, const float* x_scales,
                 int hidden, int cast_to_fp8, int scale_format, int do_zero_padding, void* recv_x,
@@ -432,10 +446,11 @@ int ep_combine_regions(const ep_layout_t* layout, const int64_t* topk_idx, const
  * ep_combine and ep_get_status work on the handle as usual.  The caller still
  * provides every input and output array.  It calls no cudaMalloc or cudaFree.
  *
- *   - Sizes whose workspace (ep_workspace_bytes) exceeds 4 MiB are rejected
- *     with EP_ERR_UNSUPPORTED, and every other argument error is returned as
- *     ep_layout returns it; a rejected call enqueues nothing and leaves the
- *     array as it was.
+ *   - Sizes whose layout part (ep_workspace_bytes - 512 * T) exceeds 4 MiB
+ *     are rejected with EP_ERR_UNSUPPORTED, and every other argument error is
+ *     returned as ep_layout returns it; a rejected call enqueues nothing and
+ *     leaves the array as it was.  The scale staging area is used only when
+ *     the whole of ep_workspace_bytes fits in the array.
  *   - Every GPU that loads the library holds the 4 MiB until the process exits.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents (each accepted call clears the words that must start at zero).

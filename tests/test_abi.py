@@ -52,6 +52,8 @@ def test_pure_host_functions(lib):
     ws = lib.ep_workspace_bytes(4096, 8, 256, 128)
     assert ws % 256 == 0 and ws >= 256 + 128 * 256 * 4 + 257 * 4 + 256 * 127 * 4
     assert lib.ep_workspace_bytes(-1, 8, 256, 1) == 0
+    # 512 bytes per token of scale staging for column-major FP8 dispatch
+    assert lib.ep_workspace_bytes(4096, 8, 256, 128) - lib.ep_workspace_bytes(0, 8, 256, 128) == 4096 * 512
     assert lib.ep_status_string(0) == b"ok"
     assert lib.ep_status_string(4) == b"bounded wait ran out"
 
@@ -114,7 +116,10 @@ def test_rank_layout_host_checks(lib, T, K, E, R, A, expect):
 def test_rank_layout_workspace_and_pointers(lib):
     p = ctypes.c_void_p(0x10000)
     ws = lib.ep_rank_workspace_bytes(4096, 8, 256)
-    assert ws % 256 == 0 and ws >= lib.ep_workspace_bytes(4096, 8, 8, 1) + 4096 * 8 * 8 + 256 * 4
+    # the expand part without its scale staging area (512 bytes per token: per-rank
+    # handles store column-major scales one by one), then the per-rank scratch
+    expand = lib.ep_workspace_bytes(4096, 8, 8, 1) - 4096 * 512
+    assert ws % 256 == 0 and ws >= expand + 4096 * 8 * 8 + 256 * 4
     assert lib.ep_rank_workspace_bytes(-1, 8, 256) == 0
     s = _handle(ws_bytes=ws - 256)
     assert lib.ep_rank_layout(p, None, 4096, 8, 256, 8, 1, None, None, None, None, None, ctypes.byref(s), None) == 1

@@ -136,3 +136,72 @@ def test_full_size_fp8_dispatch(ep, fmt):
     rq, rs = oracle.cast_fp8(inp["x"], per_row=bool(fmt & SF_PER_ROW), round_scale=bool(fmt & SF_POW2))
     assert np.array_equal(fp8_bits(q[:Np]), oracle.dispatch_rows(rq, ref, True)[:Np])
     _check_scales(fmt, s[:Np], oracle.dispatch_rows(_expected_scales(fmt, rs), ref, True)[:Np])
+
+
+COL_FORMATS = [f for f in FORMATS if f & SF_COL_MAJOR]
+
+
+@pytest.mark.parametrize("zero_pad", [True, False])
+@pytest.mark.parametrize("fmt", COL_FORMATS)
+def test_column_major_staged_and_direct(ep, fmt, zero_pad):
+    """Column-major scales leave through the workspace's staging area (a
+    handle sized by ep_workspace_bytes) or, when the workspace holds only the
+    layout's part, one store per scale from the cast kernel.  Both write the
+    same bytes everywhere: the oracle's scales on real rows, zeros on padding
+    rows with zero padding, and nothing else (a sentinel fill survives on
+    padding rows without zero padding and past the rows in use)."""
+    R, A = 8, 128
+    idx, w, x = _routing(fmt + 91)
+    ref = oracle.layout(idx, w, E, R, A)
+    Np = int(ref["off"][-1])
+    full = ep.workspace_bytes(T, K, E, A)
+    outs = []
+    for nbytes in (full, full - T * 512):
+        lay = ep.Layout(T, K, E, R, A, torch.device("cuda:0"), workspace_nbytes=nbytes)
+        ep.layout(to_dev(idx), to_dev(w), E, R, A, out=lay)
+        s = ep.scale_tensor(lay.capacity, H, fmt, lay.device)
+        raw = torch.as_strided(s, (s.shape[1], s.stride(1)), (s.stride(1), 1))
+        raw.view(torch.uint8).fill_(0x5A)
+        q, s = ep.dispatch(lay, to_dev_bf16(x), cast_to_fp8=True, do_zero_padding=zero_pad, scale_fmt=fmt,
+                           out_scales=s)
+        torch.cuda.synchronize()
+        assert ep.get_status(lay) == (ep.EP_OK, 0)
+        outs.append((fp8_bits(q[:Np]), raw.cpu().numpy().view(np.uint8).copy()))
+    (q0, r0), (q1, r1) = outs
+    assert np.array_equal(q0, q1)
+    assert np.array_equal(r0, r1)
+    rq, rs = oracle.cast_fp8(x, per_row=bool(fmt & SF_PER_ROW), round_scale=bool(fmt & SF_POW2))
+    exp_s = _expected_scales(fmt, rs)
+    raw = r0.view(np.uint32) if exp_s.dtype == np.float32 else r0
+    real = ref["recv_src"][:Np] >= 0
+    got = raw[:, :Np].T
+    assert np.array_equal(_bits(got[real]), _bits(exp_s[ref["recv_src"][:Np][real]]))
+    sentinel = 0x5A5A5A5A if exp_s.dtype == np.float32 else 0x5A
+    if zero_pad:
+        assert (got[~real] == 0).all()
+    else:
+        assert (got[~real] == sentinel).all()
+    assert (raw[:, Np:] == sentinel).all()
+
+
+def test_column_major_no_alloc_handle(ep):
+    """A no-alloc handle takes the staging area from its fixed array when the
+    array has room for it; the scales are the oracle's either way."""
+    from combine_ep_layout_11_b200 import _lib
+    import ctypes
+    lib = _lib.load()
+    fmt = SF_COL_MAJOR
+    R, A = 8, 128
+    idx, w, x = _routing(7)
+    ref = oracle.layout(idx, w, E, R, A)
+    Np = int(ref["off"][-1])
+    lay = ep.Layout(T, K, E, R, A, torch.device("cuda:0"), workspace_nbytes=256)   # replaced by the array
+    d_idx, d_w = to_dev(idx), to_dev(w)
+    rc = lib.ep_layout_no_alloc(ctypes.c_void_p(d_idx.data_ptr()), ctypes.c_void_p(d_w.data_ptr()), T, K, E, R, A,
+                                0, lay.ref(), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    q, s = ep.dispatch(lay, to_dev_bf16(x), cast_to_fp8=True, do_zero_padding=True, scale_fmt=fmt)
+    torch.cuda.synchronize()
+    rq, rs = oracle.cast_fp8(x)
+    assert np.array_equal(fp8_bits(q[:Np]), oracle.dispatch_rows(rq, ref, True)[:Np])
+    _check_scales(fmt, s[:Np], oracle.dispatch_rows(rs, ref, True)[:Np])
