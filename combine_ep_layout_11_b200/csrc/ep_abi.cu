@@ -76,6 +76,7 @@ int prepare_layout(const int64_t* topk_idx, const float* topk_weights, int T, in
     a->recv_lexp = layout->recv_local_expert;
     a->hdr = reinterpret_cast<ep::WsHeader*>(wsb);
     a->table = reinterpret_cast<int32_t*>(wsb + ws.table_off);
+    a->sup = reinterpret_cast<int32_t*>(wsb + ws.sup_off);
     a->padpre = reinterpret_cast<int32_t*>(wsb + ws.padpre_off);
     a->pad_rows = reinterpret_cast<int32_t*>(wsb + ws.padrows_off);
     a->stats = layout->cumulative_local_expert_recv_stats;
@@ -270,6 +271,7 @@ int ep_rank_layout(const int64_t* topk_idx, const float* topk_weights, int num_t
     la.recv_lexp = reinterpret_cast<int32_t*>(wsb + ws.scratch_lexp_off);
     la.hdr = header(layout);
     la.table = reinterpret_cast<int32_t*>(wsb + ws.expand.table_off);
+    la.sup = reinterpret_cast<int32_t*>(wsb + ws.expand.sup_off);
     la.padpre = reinterpret_cast<int32_t*>(wsb + ws.expand.padpre_off);
     la.pad_rows = reinterpret_cast<int32_t*>(wsb + ws.expand.padrows_off);
     la.stats = nullptr;

@@ -50,6 +50,11 @@ static_assert(sizeof(WsHeader) <= 256, "the header fits its 256 bytes");
 
 // Most chunks (CTAs of the layout kernel) a layout uses.
 constexpr int kMaxChunks = 256;
+// Chunks per super-chunk: the layout also sums the chunk counts of every run
+// of kSupChunks chunks, so that a chunk's scan reads at most
+// kMaxChunks / kSupChunks super-chunk rows and kSupChunks - 1 chunk rows.
+constexpr int kSupChunks = 16;
+constexpr int kSupRows = kMaxChunks / kSupChunks;
 
 struct Chunking {
     int num_chunks;       // C: CTAs of the counting / slot kernels
@@ -78,6 +83,8 @@ constexpr size_t kStageRowBytes = 512;
 
 struct WsLayout {
     size_t table_off;    // int32 [kMaxChunks][round4(E)]: per-chunk expert counts
+    size_t sup_off;      // int32 [2][kSupRows][round4(E)]: per-super-chunk sums, two
+                         // buffers used by alternate calls (grid-barrier generation parity)
     size_t padpre_off;   // int32 [E+1]: exclusive prefix of padding rows per expert
     size_t padrows_off;  // int32 [E*(A-1)]: receive row of every padding row
     size_t base_total;   // what the layout itself needs
@@ -91,7 +98,8 @@ inline WsLayout ws_layout(int T, int K, int E, int A) {
     (void)K;
     WsLayout w;
     w.table_off = 256;
-    w.padpre_off = round_up(w.table_off + (size_t)kMaxChunks * round4(E) * 4, 256);
+    w.sup_off = round_up(w.table_off + (size_t)kMaxChunks * round4(E) * 4, 256);
+    w.padpre_off = round_up(w.sup_off + 2 * (size_t)kSupRows * round4(E) * 4, 256);
     w.padrows_off = round_up(w.padpre_off + ((size_t)E + 1) * 4, 256);
     w.base_total = round_up(w.padrows_off + (size_t)E * (size_t)(A > 1 ? A - 1 : 0) * 4 + 4, 256);
     w.stage_off = w.base_total;

@@ -22,6 +22,7 @@ struct LayoutArgs {
     int32_t* recv_lexp;
     WsHeader* hdr;
     int32_t* table;
+    int32_t* sup;               // [2][kSupRows][round4(E)], zero before the first call
     int32_t* padpre;
     int32_t* pad_rows;
     int32_t* stats;             // [E] running receive counts, nullable

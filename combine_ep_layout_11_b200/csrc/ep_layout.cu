@@ -7,12 +7,15 @@
 // resident at once):
 //   1. count: the chunk's per-expert histogram with warp-aggregated shared
 //      atomics (__match_any_sync groups lanes holding the same expert; one
-//      leader adds the group size), published as row c of table[C][E];
+//      leader adds the group size), published as row c of table[C][E] and
+//      added into the sum of its super-chunk (16 consecutive chunks);
 //   2. one grid barrier (bounded wait);
 //   3. scan, redundantly in every CTA: for each expert the total over all
-//      chunks and the sum over chunks before c (16-byte loads of the table, four
-//      thread groups over the chunk range); off[e] = sum_{e'<e} align(cnt, A)
-//      and the padding prefix by block scans;
+//      chunks (the super-chunk sums) and the sum over chunks before c (the
+//      super-chunk sums before c's, then the rows of c's own super-chunk
+//      before c): at most 8 + 15 rows of 16-byte loads at 128 chunks, over
+//      eight thread groups; off[e] = sum_{e'<e} align(cnt, A) and the padding
+//      prefix by block scans;
 //   4. assign: each warp owns a contiguous run of the chunk's pairs; a first
 //      pass counts per (warp, expert), a scan across warps gives each warp its
 //      starting row, a second pass ranks lanes of the same expert with

@@ -240,10 +240,13 @@ __device__ __forceinline__ bool grid_barrier(WsHeader* hdr, uint32_t n, uint32_t
 //           the group's lowest lane adds the group size to the warp's row
 //           wh[w][e]; the expert ids stay in registers for the assign;
 //   publish the chunk histogram (sum over warps, which also turns wh into
-//           per-warp starting offsets) is row c of table[C][Ep];
+//           per-warp starting offsets) is row c of table[C][Ep], and is added
+//           (red) into row c / kSupChunks of this call's super-chunk sums;
 //   barrier one bounded grid barrier;
-//   scan    thread groups sum table columns over disjoint chunk ranges with
-//           16-byte loads: the total per expert and the sum over chunks < c;
+//   scan    thread groups sum, with 16-byte loads, the super-chunk rows (all
+//           of them: the total per expert; those before c's own: part of the
+//           prefix) and the chunk rows of c's super-chunk before c (the rest
+//           of the prefix): at most kSupRows + kSupChunks - 1 rows;
 //           one packed 64-bit block scan gives off[e] and the padding prefix;
 //   assign  rank = popc(peers & lanemask_lt) within the round, plus the warp's
 //           running offset, plus the chunk base: the stable token-major,
@@ -321,6 +324,18 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     __syncthreads();
     for (int e4 = tid; e4 < Ep / 4; e4 += NT)
         reinterpret_cast<int4*>(a.table + (size_t)c * Ep)[e4] = reinterpret_cast<const int4*>(L.cnt)[e4];
+    // the counts are also added into the super-chunk's row of this call's sum
+    // buffer (generation parity); the other buffer, which the previous call
+    // used, is zeroed for the next one
+    {
+        int32_t* sup_now = a.sup + (size_t)(s_gen0 & 1u) * kSupRows * Ep + (size_t)(c / kSupChunks) * Ep;
+        for (int e = tid; e < E; e += NT) {
+            const int v = L.cnt[e];
+            if (v) atomicAdd(&sup_now[e], v);
+        }
+        int4* sup_next = reinterpret_cast<int4*>(a.sup + (size_t)((s_gen0 + 1u) & 1u) * kSupRows * Ep);
+        for (int i = c * NT + tid; i < kSupRows * Ep / 4; i += C * NT) sup_next[i] = make_int4(0, 0, 0, 0);
+    }
 
     // ---- barrier ----
     if (!grid_barrier(a.hdr, (uint32_t)C, s_gen0)) {
@@ -340,25 +355,37 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
         // is no longer needed once published); several: partials, then a sum
         int32_t* dst_tot = groups == 1 ? L.cnt : part_tot;
         int32_t* dst_pre = groups == 1 ? L.base : part_pre;
+        // the rows a chunk sums: the G super-chunk rows of this call (all of
+        // them for the totals, those before its own super-chunk sg for its
+        // prefix), then the chunk rows c0 .. c-1 of its own super-chunk
+        const int sg = c / kSupChunks, c0 = sg * kSupChunks;
+        const int G = (C + kSupChunks - 1) / kSupChunks;
+        const int nv = G + (c - c0);
+        const int4* sup_now = reinterpret_cast<const int4*>(a.sup + (size_t)(s_gen0 & 1u) * kSupRows * Ep);
+        const int4* tab = reinterpret_cast<const int4*>(a.table);
         const int g = tid / cols;
         if (g < groups) {
-            const int c_lo = (int)((int64_t)C * g / groups), c_hi = (int)((int64_t)C * (g + 1) / groups);
+            const int v_lo = nv * g / groups, v_hi = nv * (g + 1) / groups;
             for (int q = tid % cols; q < cols; q += (cols < NT ? cols : NT)) {
                 int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
-                const int4* col = reinterpret_cast<const int4*>(a.table) + q;
-                // up to 16 rows in flight at once (a group's whole range when
-                // C <= 128 and E <= 256), then summed
-                for (int r0 = c_lo; r0 < c_hi; r0 += 16) {
-                    // sixteen unconditional loads (rows past the range re-read
-                    // the last row and are dropped), issued back to back
-                    int4 v[16];
+                for (int r0 = v_lo; r0 < v_hi; r0 += 8) {
+                    // eight unconditional loads (rows past the range re-read the
+                    // last row and are dropped), issued back to back
+                    int4 v[8];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = ld_cg_v4(col + (size_t)min(r0 + i, c_hi - 1) * cols);
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = min(r0 + i, v_hi - 1);
+                        v[i] = ld_cg_v4((r < G ? sup_now + (size_t)r * cols : tab + (size_t)(c0 + r - G) * cols) + q);
+                    }
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        if (r0 + i >= c_hi) continue;
-                        tot.x += v[i].x; tot.y += v[i].y; tot.z += v[i].z; tot.w += v[i].w;
-                        if (r0 + i < c) { pre.x += v[i].x; pre.y += v[i].y; pre.z += v[i].z; pre.w += v[i].w; }
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = r0 + i;
+                        if (r >= v_hi) continue;
+                        if (r < G) {
+                            tot.x += v[i].x; tot.y += v[i].y; tot.z += v[i].z; tot.w += v[i].w;
+                            if (r >= sg) continue;
+                        }
+                        pre.x += v[i].x; pre.y += v[i].y; pre.z += v[i].z; pre.w += v[i].w;
                     }
                 }
                 reinterpret_cast<int4*>(dst_tot + g * Ep)[q] = tot;
