@@ -139,6 +139,12 @@ int prepare_dispatch(const ep_layout_t* layout, const void* x, int x_dtype, cons
     a->capacity = layout->capacity;
     a->nb = fp8_out ? H / 128 : 0;
     a->zero_pad = do_zero_padding ? 1 : 0;
+    // padding rows: E*(A-1) at most for the expand form, the whole slab of an
+    // expert for the fixed-slab form, none for the per-rank form
+    if (layout->kind == EP_LAYOUT_LL_SLAB)
+        a->max_pad_rows = (int64_t)layout->num_experts * layout->num_ranks * layout->num_max_tokens_per_rank;
+    else if (layout->kind == EP_LAYOUT_EXPAND)
+        a->max_pad_rows = (int64_t)layout->num_experts * (layout->expert_alignment - 1);
     if (!ep::set_scale_format(a, scale_format, layout->capacity)) return EP_ERR_INVALID_ARG;
     // column-major per-block scales go through the staging area when the
     // handle's workspace holds it (per-row scales are K words per token: one

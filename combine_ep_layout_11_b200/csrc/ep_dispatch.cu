@@ -20,6 +20,7 @@ namespace {
 using namespace dispatch_dev;
 
 constexpr uint32_t kMaxSegBytes = 16384;   // one bulk copy per row segment
+constexpr uint32_t kTailSegBytes = 4096;   // segments of the last tokens
 
 // ---------------------------------------------------------------------------
 // Copy kernel.  Work is handed out by tickets (atomic counters in the layout's
@@ -49,9 +50,36 @@ __device__ __forceinline__ uint8_t* region_row(const DispatchArgs& a, int64_t e,
     return a.regions[e / a.El] + row * row_bytes;
 }
 
+// Items: tokens [0, t_full) in nseg segments of seg_bytes, then the last
+// tokens [t_full, T) in nseg2 smaller segments of seg2_bytes, so the work
+// drawn last is small and the SMs finish together.
+struct CopyItems {
+    uint32_t row_bytes, seg_bytes, seg2_bytes;
+    int nseg, nseg2;
+    uint32_t t_full;
+    __device__ __forceinline__ uint32_t count(uint32_t T) const {
+        return t_full * (uint32_t)nseg + (T - t_full) * (uint32_t)nseg2;
+    }
+    // token, byte offset and length of item i
+    __device__ __forceinline__ void locate(uint32_t i, int64_t& t, uint32_t& off, uint32_t& bytes) const {
+        const uint32_t nf = t_full * (uint32_t)nseg;
+        uint32_t seg;
+        if (i < nf) {
+            t = i / nseg;
+            off = (i % nseg) * seg_bytes;
+            seg = seg_bytes;
+        } else {
+            t = t_full + (i - nf) / nseg2;
+            off = ((i - nf) % nseg2) * seg2_bytes;
+            seg = seg2_bytes;
+        }
+        bytes = min(seg, row_bytes - off);
+    }
+};
+
 template <bool kRegions>
-__global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArgs a, uint32_t row_bytes,
-                                                                     uint32_t seg_bytes, int nseg, int stages) {
+__global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArgs a, CopyItems it, int stages) {
+    const uint32_t row_bytes = it.row_bytes, seg_bytes = it.seg_bytes;
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t stride = round_up_u32(seg_bytes, 128);
     uint8_t* ring = smem;
@@ -73,11 +101,11 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
 
     // token rows: one ticket per (token, segment) item; the row of a stage is
     // loaded by load_row, its destinations by load_slots
-    const uint32_t items = (uint32_t)a.T * (uint32_t)nseg;
+    const uint32_t items = it.count((uint32_t)a.T);
     auto load_row = [&](int s, uint32_t item) {
-        const int64_t t = item / nseg;
-        const uint32_t off = (uint32_t)(item % nseg) * seg_bytes;
-        const uint32_t bytes = min(seg_bytes, row_bytes - off);
+        int64_t t;
+        uint32_t off, bytes;
+        it.locate(item, t, off, bytes);
         if (lane == 0) {
             stage_item[s] = item;
             mbar_arrive_expect_tx(&full[s], bytes);
@@ -85,7 +113,9 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
         }
     };
     auto load_slots = [&](int s, uint32_t item) {
-        const int64_t t = item / nseg;
+        int64_t t;
+        uint32_t off, bytes;
+        it.locate(item, t, off, bytes);
         if (lane < K) {
             const int32_t slot = a.pair_slot[t * K + lane];
             if (kRegions) dsts[s * 32 + lane] = region_row<kRegions>(a, a.topk_idx[t * K + lane], slot, row_bytes);
@@ -178,10 +208,9 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
         }
         __syncwarp();
         const uint32_t item = stage_item[s];
-        const int64_t t = item / nseg;
-        const int sg = (int)(item % nseg);
-        const uint32_t off = (uint32_t)sg * seg_bytes;
-        const uint32_t bytes = min(seg_bytes, row_bytes - off);
+        int64_t t;
+        uint32_t off, bytes;
+        it.locate(item, t, off, bytes);
         if (lane < K && kRegions) {
             uint8_t* dst = dsts[s * 32 + lane];
             if (dst != nullptr) bulk_store(dst + off, ring + (size_t)s * stride, bytes);
@@ -190,7 +219,7 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
             if (slot >= 0 && (int64_t)slot < a.capacity)
                 bulk_store(a.recv + (int64_t)slot * row_bytes + off, ring + (size_t)s * stride, bytes);
         }
-        if (!kRegions && a.x_scales != nullptr && sg == 0) {
+        if (!kRegions && a.x_scales != nullptr && off == 0) {
             // e4m3 input: carry the token's scale row to every destination
             for (int k = 0; k < K; ++k) {
                 const int32_t slot = slots[s * 32 + k];
@@ -221,10 +250,14 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
 }  // namespace
 
 cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStream_t s, bool regions) {
-    const uint32_t row_bytes = (uint32_t)a.H * (uint32_t)elem_bytes;
-    const int nseg = (int)((row_bytes + kMaxSegBytes - 1) / kMaxSegBytes);
-    const uint32_t seg_bytes = round_up_u32((row_bytes + nseg - 1) / nseg, 16);
-    const uint32_t stride = round_up_u32(seg_bytes, 128);
+    CopyItems it{};
+    it.row_bytes = (uint32_t)a.H * (uint32_t)elem_bytes;
+    it.nseg = (int)((it.row_bytes + kMaxSegBytes - 1) / kMaxSegBytes);
+    it.seg_bytes = round_up_u32((it.row_bytes + it.nseg - 1) / it.nseg, 16);
+    it.nseg2 = (int)((it.row_bytes + kTailSegBytes - 1) / kTailSegBytes);
+    if (it.nseg2 < it.nseg) it.nseg2 = it.nseg;
+    it.seg2_bytes = round_up_u32((it.row_bytes + it.nseg2 - 1) / it.nseg2, 16);
+    const uint32_t stride = round_up_u32(it.seg_bytes, 128);
     // three row stages of at most 16 KB, up to four CTAs per SM: a sweep of
     // 2-4 stages, 3-4 CTAs per SM and 2-4 KB zero buffers on the prefill,
     // large-prefill and decode workloads put every setting within 2 %
@@ -240,7 +273,18 @@ cudaError_t launch_dispatch_copy(const DispatchArgs& a, int elem_bytes, cudaStre
     if (ctas_per_sm > 4) ctas_per_sm = 4;
     if (ctas_per_sm < 1) ctas_per_sm = 1;
     const int grid = a.sms * ctas_per_sm;
-    return launch_pdl(kernel, dim3(grid), dim3(kCopyThreads), smem, s, false, a, row_bytes, seg_bytes, nseg, stages);
+    // The last 2 * grid tokens go in segments of at most 4 KB, so the SMs run
+    // out of work together (decode: 82-83 against 86 us; large prefill: 381
+    // against 386-389 us; 3 or 4 * grid measured the same, 2 KB segments and
+    // a tail of grid / 2 or grid tokens less well).  Not where padding may
+    // exceed a fifth of the rows: its 2 KB pieces already keep the SMs busy
+    // to the end, and the small segments cost more than they save (prefill:
+    // 137.7 against 134.6 us).
+    const int64_t pads = a.zero_pad ? (regions ? a.num_pad_list : a.max_pad_rows) : 0;
+    const bool split = pads * 4 <= (int64_t)a.T * a.K;
+    const int64_t tail = 2 * (int64_t)grid;
+    it.t_full = !split ? (uint32_t)a.T : a.T > tail ? (uint32_t)(a.T - tail) : 0u;
+    return launch_pdl(kernel, dim3(grid), dim3(kCopyThreads), smem, s, false, a, it, stages);
 }
 
 }  // namespace ep

@@ -65,6 +65,7 @@ struct DispatchArgs {
     int64_t capacity;
     int nb;                    // 128-column blocks per row (H/128) when FP8 is involved
     int zero_pad;
+    int64_t max_pad_rows;      // a bound on the padding rows, known on the host
     int sms;
     // scale output of the cast (EP_SF_* bits): ng scales per row (nb, or 1 per
     // row), sf_elem bytes each (4: fp32, 1: UE8M0); scale (row, g) at byte
