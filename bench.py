@@ -463,6 +463,7 @@ def run_ours(args, rank, world, local_rank):
         e2e = run_e2e(args, ep, torch, dev, st.inp, cfg, st.lay, st.y, st.fp8, st.recv, st.recv_s, flush,
                       st.do_layout, st.per_rank)
         e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dist, dev)
+        e2e["copy_ms_per_step"] = max_over_ranks(e2e["copy_ms_per_step"], dist, dev)
 
     if rank != 0:
         if dist:
@@ -525,7 +526,14 @@ def run_ours(args, rank, world, local_rank):
                               "outputs (the combine input) stay resident on the device, as a GPU expert layer "
                               "produces them there; uploads, calls and downloads pipelined over three streams, "
                               "timed from the first upload to the last download; no L2 flush (each step moves "
-                              "more than L2 holds)" % e2e["steps"]}
+                              "more than L2 holds)" % e2e["steps"],
+                       "copy_bound": {"ms_per_step": round(e2e["copy_ms_per_step"], 4),
+                                      "frac": round(e2e["copy_ms_per_step"] / e2e["ms_per_step"], 4),
+                                      "gbs_per_direction": round(max(e2e["h2d"], e2e["d2h"]) /
+                                                                 (e2e["copy_ms_per_step"] * 1e6), 1),
+                                      "how": "the same uploads and downloads alone (no calls), both "
+                                             "directions at once: the PCIe ceiling of this leg; frac = "
+                                             "that time over the leg's"}}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, st.inp, args.layout)
     if world == 1 and args.per_workload and args.tokens is None:
@@ -610,9 +618,32 @@ def run_e2e(args, ep, torch, dev, inp, cfg, lay, y, fp8, recv, recv_s, flush, do
     e1.synchronize()
     torch.cuda.synchronize(dev)
     assert torch.equal(h_out[(steps - 1) % 2], d_out[(steps - 1) % 2].view(torch.int16).cpu())
+    e2e_ms = e0.elapsed_time(e1) / steps
+
+    # the ceiling of this leg: the same uploads and downloads with no calls,
+    # both directions at once on their streams
+    def copies(n):
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_up):
+                d_idx[b].copy_(h_idx, non_blocking=True)
+                d_w[b].copy_(h_w, non_blocking=True)
+                d_x[b].copy_(h_x, non_blocking=True)
+            with torch.cuda.stream(s_down):
+                h_out[b].copy_(d_out[b].view(torch.int16), non_blocking=True)
+
+    copies(2)
+    torch.cuda.synchronize(dev)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(s_up)
+    s_down.wait_event(c0)
+    copies(steps)
+    s_down.wait_stream(s_up)
+    c1.record(s_down)
+    c1.synchronize()
     h2d = h_idx.numel() * 8 + h_w.numel() * 4 + h_x.numel() * 2
-    return {"ms_per_step": e0.elapsed_time(e1) / steps, "h2d": int(h2d), "d2h": int(h_out[0].numel() * 2),
-            "steps": steps}
+    return {"ms_per_step": e2e_ms, "h2d": int(h2d), "d2h": int(h_out[0].numel() * 2),
+            "steps": steps, "copy_ms_per_step": c0.elapsed_time(c1) / steps}
 
 
 # --------------------------------------------------------------------------
