@@ -350,3 +350,38 @@ def test_fused_layout_dispatch_many_rounds(ep):
     assert ep.get_status(lay) == (ep.EP_OK, 0)
     Np = check_layout(lay, ref)
     assert np.array_equal(bf16_bits(recv[:Np]), oracle.dispatch_rows(x, ref, True)[:Np])
+
+
+def _copy_grid():
+    """CTAs of the copy kernel: four per SM (its three 16 KB stages fit four times)."""
+    return 4 * torch.cuda.get_device_properties(0).multi_processor_count
+
+
+@pytest.mark.parametrize("dT", [-3, 0, 5])
+@pytest.mark.parametrize("H", [16384, 7168], ids=["row32KB", "row14KB"])
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_tail_segments_around_the_split(ep, dT, H, fused):
+    """Without padding that could fill the tail (A = 1) the copy kernel hands
+    out the last 2 x grid tokens as segments of at most 4 KB.  Batches just
+    below, at and above that many tokens (all tokens small, none but a few
+    large) with rows of one and two 16 KB segments: bit-exact rows and
+    combine."""
+    T = 2 * _copy_grid() + dT
+    T -= T % 4
+    idx, w, x = _rand(T, 6, 64, H, seed=T + H, drop=0.05)
+    _full(ep, idx, w, x, 64, 4, 1, fused=fused)
+
+
+def test_tail_segments_fp8_input(ep):
+    """e4m3 rows (7 KB: one segment, two in the tail) with their scale rows,
+    carried once per token from the first segment."""
+    T, K, E, R, A, H = 2 * _copy_grid() + 8, 8, 64, 4, 1, 7168
+    idx, w, x = _rand(T, K, E, H, seed=3)
+    q, s = oracle.cast_fp8(x)
+    ref = oracle.layout(idx, w, E, R, A)
+    lay = ep.layout(to_dev(idx), to_dev(w), E, R, A)
+    rq, rs = ep.dispatch(lay, to_dev(q).view(torch.float8_e4m3fn), x_scales=to_dev(s), do_zero_padding=True)
+    torch.cuda.synchronize()
+    Np = int(ref["off"][-1])
+    assert np.array_equal(fp8_bits(rq[:Np]), oracle.dispatch_rows(q, ref, True)[:Np])
+    assert np.array_equal(f32_bits(rs[:Np]), oracle.dispatch_rows(s, ref, True)[:Np].view(np.uint32))
