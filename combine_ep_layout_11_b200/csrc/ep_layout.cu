@@ -57,7 +57,9 @@ cudaError_t launch_layout_nt(LayoutArgs a, int sms, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     int max_chunks = sms * (per_sm > 0 ? per_sm : 1);
     if (max_chunks > kLayoutChunks) max_chunks = kLayoutChunks;
-    Chunking ch = chunking(a.T, a.K, max_chunks, NT);
+    // the fixed-slab form lists up to E * slab padding rows, far more than its
+    // pairs: as many chunks as the tokens allow, so every SM shares that work
+    Chunking ch = chunking(a.T, a.K, max_chunks, a.slab > 0 ? 1 : NT);
     if (ch.num_chunks == 0) {   // no tokens (the fixed-slab form still has its padding rows to list)
         ch.num_chunks = 1;
         ch.chunk_tokens = 0;
