@@ -62,9 +62,13 @@ __device__ __forceinline__ int pair_key(const LayoutArgs& a, int64_t i, bool& ba
         return key;
     }
     const int R = a.K;
-    const int64_t t = i / R;
-    const int r = (int)(i - t * R);
+    // pair indices stay below 2^31 (T * R <= INT_MAX is checked on the host):
+    // 32-bit division
+    const int64_t t = (int)i / R;
+    const int r = (int)i - (int)t * R;
+    // rank r holds the experts [lo, lo + El): a range test, no 64-bit division
     const int El = a.src_E / R;
+    const int64_t lo = (int64_t)r * El, hi = lo + El;
     const int64_t* row = a.src_idx + t * a.src_K;
     int key = -1;
     for (int k0 = 0; k0 < a.src_K; k0 += 8) {
@@ -74,13 +78,11 @@ __device__ __forceinline__ int pair_key(const LayoutArgs& a, int64_t i, bool& ba
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int64_t e = ev[j];
-            if (e >= 0 && e < a.src_E) {
-                if (e / El == r) {
-                    key = r;
-                    // each selected (t, k) is local to exactly one rank: counted once
-                    if (hist) atomicAdd(&hist[e], 1);
-                }
-            } else if (e != -1) {
+            if (e >= lo && e < hi) {
+                key = r;
+                // each selected (t, k) is local to exactly one rank: counted once
+                if (hist) atomicAdd(&hist[e], 1);
+            } else if (e != -1 && (e < 0 || e >= a.src_E)) {
                 bad = true;
             }
         }
@@ -122,9 +124,10 @@ __device__ __forceinline__ uint32_t atom_add_release_u32(uint32_t* p, uint32_t v
 __device__ __forceinline__ void write_rank_row(const LayoutArgs& a, int64_t i, int slot) {
     if (!a.rank_topk_idx && !a.rank_topk_w) return;
     const int R = a.K, K = a.src_K;
-    const int64_t t = i / R;
-    const int r = (int)(i - t * R);
+    const int64_t t = (int)i / R;   // 32-bit: T * R <= INT_MAX
+    const int r = (int)i - (int)t * R;
     const int El = a.src_E / R;
+    const int64_t lo = (int64_t)r * El, hi = lo + El;   // rank r's experts
     const int64_t* row = a.src_idx + t * K;
     int64_t* oi = a.rank_topk_idx ? a.rank_topk_idx + (int64_t)slot * K : nullptr;
     float* ow = a.rank_topk_w ? a.rank_topk_w + (int64_t)slot * K : nullptr;
@@ -148,8 +151,8 @@ __device__ __forceinline__ void write_rank_row(const LayoutArgs& a, int64_t i, i
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int64_t e = ev[j + q];
-                const bool local = k + q < K && e >= 0 && e < a.src_E && e / El == r;
-                o[q] = local ? e - (int64_t)r * El : -1;
+                const bool local = k + q < K && e >= lo && e < hi;
+                o[q] = local ? e - lo : -1;
                 w4[q] = local ? wv[j + q] : 0.0f;
             }
             if (vec) {
