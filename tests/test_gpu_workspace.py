@@ -125,3 +125,29 @@ def test_fused_call_advances_the_generation(ep):
                                      out_layout=lay, out=recv)
     assert _words(lay)[8] == 2 and (_words(lay)[2:8] == 0).all()
     assert np.array_equal(bf16_bits(recv2[:Np]), oracle.dispatch_rows(x, ref, True)[:Np])
+
+
+def test_one_handle_across_batch_sizes(ep):
+    """One workspace through layouts of different batch sizes, so the number of
+    chunks (CTAs) changes from call to call while the two super-chunk sum
+    buffers alternate with the generation: every call bit-exact."""
+    from combine_ep_layout_11_b200 import _lib
+    lib = _lib.load()
+    Tmax, K, E, R, A = 8192, 8, 256, 8, 128
+    lay = ep.Layout(Tmax, K, E, R, A, DEV)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for call, T in enumerate((8192, 640, 4096, 96, 8192, 1024, 2048), start=1):
+        idx, w, _ = _rand(T, K, E, 8, 100 + call)
+        d_idx, d_w = to_dev(idx), to_dev(w)
+        rc = lib.ep_layout(ctypes.c_void_p(d_idx.data_ptr()), ctypes.c_void_p(d_w.data_ptr()), T, K, E, R, A, 0,
+                           lay.ref(), stream)
+        assert rc == 0
+        torch.cuda.synchronize()
+        ref = oracle.layout(idx, w, E, R, A)
+        assert np.array_equal(lay.num_recv_tokens_per_expert.cpu().numpy(), ref["cnt"]), "call %d" % call
+        assert np.array_equal(lay.expert_offset.cpu().numpy(), ref["off"]), "call %d" % call
+        assert np.array_equal(lay._pair_slot_buf[:T * K].cpu().numpy(), ref["pair_slot"].reshape(-1))
+        Np = int(ref["off"][-1])
+        assert np.array_equal(lay.recv_src_token[:Np].cpu().numpy(), ref["recv_src"][:Np])
+        assert _words(lay)[8] == call
+    assert ep.get_status(lay) == (ep.EP_OK, 0)
