@@ -205,3 +205,31 @@ def test_column_major_no_alloc_handle(ep):
     rq, rs = oracle.cast_fp8(x)
     assert np.array_equal(fp8_bits(q[:Np]), oracle.dispatch_rows(rq, ref, True)[:Np])
     _check_scales(fmt, s[:Np], oracle.dispatch_rows(rs, ref, True)[:Np])
+
+
+@pytest.mark.parametrize("fmt", [SF_COL_MAJOR, SF_COL_MAJOR | SF_POW2 | SF_UE8M0])
+def test_column_major_capacity_overflow(ep, fmt):
+    """A receive buffer smaller than the layout: both column-major routes write
+    exactly the rows below the capacity (the oracle's scales there) and report
+    EP_ERR_CAPACITY."""
+    R, A, cap = 8, 128, 1000
+    idx, w, x = _routing(fmt + 5)
+    ref = oracle.layout(idx, w, E, R, A)
+    assert int(ref["off"][-1]) > cap
+    full = ep.workspace_bytes(T, K, E, A)
+    raws = []
+    for nbytes in (full, full - T * 512):
+        lay = ep.Layout(T, K, E, R, A, torch.device("cuda:0"), capacity=cap, workspace_nbytes=nbytes)
+        ep.layout(to_dev(idx), to_dev(w), E, R, A, out=lay)
+        s = ep.scale_tensor(cap, H, fmt, lay.device)
+        raw = torch.as_strided(s, (s.shape[1], s.stride(1)), (s.stride(1), 1))
+        raw.view(torch.uint8).fill_(0x5A)
+        q, s = ep.dispatch(lay, to_dev_bf16(x), cast_to_fp8=True, do_zero_padding=True, scale_fmt=fmt, out_scales=s)
+        code, _ = ep.get_status(lay)
+        assert code == ep.EP_ERR_CAPACITY
+        raws.append(raw.cpu().numpy().view(np.uint8).copy())
+    assert np.array_equal(raws[0], raws[1])
+    rq, rs = oracle.cast_fp8(x, round_scale=bool(fmt & SF_POW2))
+    exp_s = oracle.dispatch_rows(_expected_scales(fmt, rs), ref, True)[:cap]
+    got = (raws[0].view(np.uint32) if exp_s.dtype == np.float32 else raws[0])[:, :cap].T
+    assert np.array_equal(_bits(got), _bits(exp_s))
