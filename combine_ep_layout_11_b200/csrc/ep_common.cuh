@@ -41,9 +41,9 @@ struct WsHeader {
     uint32_t tok_ticket;  // dispatch: next token-row ticket
     uint32_t pad_ticket;  // dispatch: next padding ticket
     uint32_t done;        // dispatch: CTAs finished (the last one resets the tickets)
-    uint32_t bar_count;   // layout grid barrier: CTAs arrived in the current generation
-    uint32_t reserved;
-    uint32_t bar_gen;     // layout grid barrier generation (any value will do)
+    uint32_t bar_count;       // layout grid barrier: CTAs arrived, even generations
+    uint32_t bar_count_odd;   // the same for odd generations
+    uint32_t bar_gen;         // layout grid barrier generation (any value will do)
 };
 constexpr size_t kHeaderClearBytes = offsetof(WsHeader, bar_gen);
 static_assert(sizeof(WsHeader) <= 256, "the header fits its 256 bytes");

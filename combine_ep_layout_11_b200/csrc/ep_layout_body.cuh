@@ -109,10 +109,8 @@ __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ uint32_t atom_add_release_u32(uint32_t* p, uint32_t v) {
-    uint32_t old;
-    asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
+__device__ __forceinline__ void red_add_release_u32(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // Exclusive scan of one 64-bit value per thread across a CTA of NT threads;
@@ -201,36 +199,41 @@ __device__ __forceinline__ long long block_exclusive_scan64(long long v, long lo
     return prefix;
 }
 
-// Grid-wide barrier over `n` co-resident CTAs by generation counting (no reset
-// between calls).  `gen0` is the generation read before this CTA's arrival
-// (every arrival of this generation happens after that read, so the value
-// cannot have moved on yet).  The CTA's writes are ordered before thread 0's
-// release arrival by __syncthreads; the last arriver publishes the new
-// generation with a release store; the others acquire it.  Bounded: false if
-// the other CTAs have not all arrived within kWaitLimitNs.
+// One bounded grid barrier over the n co-resident CTAs of this launch.  Two
+// arrival counters alternate with the parity of the generation gen0, which
+// every CTA read before arriving: each CTA's thread 0 adds one to its counter
+// with a release reduction (no round trip to wait for) and polls it with
+// acquire loads until all n have arrived; the CTA's writes are ordered before
+// that reduction by __syncthreads.  After the barrier CTA 0 zeroes the other
+// counter (the previous call used it, the next one will) and advances the
+// generation.  The counter of this call keeps the value n until the next call
+// zeroes it: a CTA still polling must not see it fall.  Bounded: false if the
+// other CTAs have not all arrived within kWaitLimitNs (the workspace must then
+// be zeroed again before the next call).
 __device__ __forceinline__ bool grid_barrier(WsHeader* hdr, uint32_t n, uint32_t gen0) {
     __shared__ int s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
+        uint32_t* cnt = (gen0 & 1u) ? &hdr->bar_count_odd : &hdr->bar_count;
         __threadfence();
-        const uint32_t arrived = atom_add_release_u32(&hdr->bar_count, 1u);
+        red_add_release_u32(cnt, 1u);
         int ok = 1;
-        if (arrived == n - 1) {
-            hdr->bar_count = 0;
-            st_release_u32(&hdr->bar_gen, gen0 + 1);
-        } else {
-            const uint64_t t0 = globaltimer_ns();
-            while (ld_acquire_u32(&hdr->bar_gen) == gen0) {
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                    ok = 0;
-                    break;
-                }
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_u32(cnt) < n) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                ok = 0;
+                break;
             }
         }
         s_ok = ok;
     }
     __syncthreads();
-    return s_ok != 0;
+    const bool ok = s_ok != 0;
+    if (ok && blockIdx.x == 0 && threadIdx.x == 0) {
+        *((gen0 & 1u) ? &hdr->bar_count : &hdr->bar_count_odd) = 0;
+        hdr->bar_gen = gen0 + 1;
+    }
+    return ok;
 }
 
 // The layout work of one CTA: chunk c = blockIdx.x of a.C co-resident CTAs of

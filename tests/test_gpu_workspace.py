@@ -1,15 +1,17 @@
 """The workspace's control words on the GPU, through the C ABI.
 
-The layout's grid barrier counts arrivals in `bar_count` and advances
-`bar_gen` once per call; the dispatch kernels hand out work by ticket and the
-last CTA sets the tickets back to zero.  These tests check the words
+The layout's grid barrier counts arrivals in one of two counters, chosen by
+the parity of `bar_gen`, and advances `bar_gen` once per call (zeroing the
+other counter for the next call); the dispatch kernels hand out work by ticket
+and the last CTA sets the tickets back to zero.  These tests check the words
 themselves and the property they exist for: a workspace reused across calls of
 different inputs - with a zero-token call, which skips the layout kernel and
 clears the header on the host, in between - gives results bit-identical to the
 oracle every time, and a second dispatch on a handle does all the work again.
 
 Header words (int32 index): status 0, num_pad 1, pending 2, tok_ticket 3,
-pad_ticket 4, done 5, bar_count 6, bar_gen 8.
+pad_ticket 4, done 5, bar_count 6 (even generations), bar_count_odd 7,
+bar_gen 8.
 """
 import ctypes
 
@@ -49,9 +51,10 @@ def _rand(T, K, E, H, seed):
 
 
 def test_reused_workspace_across_inputs_and_zero_token_calls(ep):
-    """bar_gen advances by one per layout kernel and every other control word
-    is back at zero after each call; a zero-token call in between (host-side
-    clear, no kernel) keeps the next layout bit-exact."""
+    """bar_gen advances by one per layout kernel; after each call the tickets
+    and flags are back at zero, the counter of the call's parity holds its
+    chunk count and the other is zero; a zero-token call in between
+    (host-side clear, no kernel) keeps the next layout bit-exact."""
     from combine_ep_layout_11_b200 import _lib
     lib = _lib.load()
     T, K, E, R, A, H = 4096, 8, 256, 8, 128, 256
@@ -65,7 +68,8 @@ def test_reused_workspace_across_inputs_and_zero_token_calls(ep):
         ref = oracle.layout(idx, w, E, R, A)
         check_layout(lay, ref)
         assert int(words[1]) == int(ref["off"][-1]) - int((idx >= 0).sum())   # num_pad
-        assert (words[2:8] == 0).all()                    # pending, tickets, barrier count
+        assert (words[2:6] == 0).all()                    # pending, tickets
+        assert words[6 + (call & 1)] == 0 and words[6 + ((call - 1) & 1)] > 0   # barrier counters
         # a call with no tokens on the same handle: counts and offsets zeroed, generation kept
         rc = lib.ep_layout(None, None, 0, K, E, R, A, 0, lay.ref(), stream)
         assert rc == 0
@@ -123,7 +127,7 @@ def test_fused_call_advances_the_generation(ep):
     assert np.array_equal(bf16_bits(recv[:Np]), oracle.dispatch_rows(x, ref, True)[:Np])
     lay2, recv2 = ep.layout_dispatch(to_dev(idx), to_dev(w), to_dev_bf16(x), E, R, A, do_zero_padding=True,
                                      out_layout=lay, out=recv)
-    assert _words(lay)[8] == 2 and (_words(lay)[2:8] == 0).all()
+    assert _words(lay)[8] == 2 and (_words(lay)[2:6] == 0).all()
     assert np.array_equal(bf16_bits(recv2[:Np]), oracle.dispatch_rows(x, ref, True)[:Np])
 
 
