@@ -219,9 +219,13 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
     // eight with one: the fastest of the (columns per lane, rows per batch)
     // pairs measured on the prefill and decode workloads, expand and per-rank
     // handles, once the selected entries are packed (2-8 rows per batch,
-    // 512 B - 4 KB per row and item)
-    auto kernel = a.regions ? (a.bias0 ? combine_kernel<2, 2, 8, true, true> : combine_kernel<2, 2, 2, false, true>)
-                            : (a.bias0 ? combine_kernel<2, 2, 8, true> : combine_kernel<2, 2, 2, false>);
+    // 512 B - 4 KB per row and item).  Without a bias the kernel is held to
+    // 64 registers so four CTAs (32 warps) share an SM instead of three:
+    // more loads in flight per SM, 328 against 337 us at large prefill
+    // (five or six CTAs spill; with a bias the 8-row batches need the
+    // registers).
+    auto kernel = a.regions ? (a.bias0 ? combine_kernel<2, 2, 8, true, true> : combine_kernel<2, 4, 2, false, true>)
+                            : (a.bias0 ? combine_kernel<2, 2, 8, true> : combine_kernel<2, 4, 2, false>);
     int blocks_per_sm = 0;
     cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kernel, kCombineThreads, 0);
     if (err != cudaSuccess) return err;
