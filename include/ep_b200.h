@@ -134,7 +134,9 @@ extern "C" {
  *                                             destination rank (e mod E/R), -1 on padding
  *   workspace                  ep_workspace_bytes() bytes, 256-byte aligned,
  *                              zero-filled by the caller before its first use
- *                              (every later ep_layout leaves it ready again);
+ *                              (every later ep_layout leaves it ready again;
+ *                              after a call reported EP_ERR_TIMEOUT, zero it
+ *                              again before the next one);
  *                              holds the device status word and scan scratch,
  *                              and last a staging area of 512 bytes per token
  *                              for ep_dispatch's column-major FP8 scales.  A
