@@ -83,8 +83,14 @@ def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    except (OSError, KeyError, ValueError):
+        v = d["hbm_gbs"]
+        if isinstance(v, dict):   # {"value": ...} or {"gbs": ...}
+            v = v.get("value", v.get("gbs"))
+        v = float(v)
+        if not v > 0:
+            raise ValueError("hbm_gbs")
+        return v, "measured"
+    except (OSError, KeyError, ValueError, TypeError):
         return 6650.0, "fallback"
 
 
