@@ -39,7 +39,7 @@ namespace {
 constexpr int kLayoutChunks = 128;
 
 template <int NT, bool kRankKeys>
-__global__ void __launch_bounds__(NT) layout_kernel(LayoutArgs a) {
+__global__ void __launch_bounds__(NT, 1) layout_kernel(LayoutArgs a) {
     extern __shared__ __align__(16) int32_t sm[];
     pdl_wait();
     pdl_launch_dependents();

@@ -195,8 +195,7 @@ __device__ __forceinline__ long long block_exclusive_scan64(long long v, long lo
     __syncthreads();
     const long long prefix = (wid > 0 ? scratch[wid - 1] : 0) + x - v;
     *total = scratch[kW - 1];
-    __syncthreads();
-    return prefix;
+    return prefix;   // `scratch` is read until here: a barrier must come before its next write
 }
 
 // One bounded grid barrier over the n co-resident CTAs of this launch.  Two
@@ -350,17 +349,17 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     }
 
     // ---- scan ----
+    const int cols = Ep / 4;
+    int groups = NT / cols;
+    if (groups > 8) groups = 8;
+    if (groups < 1) groups = 1;
+    int32_t* part_tot = L.part;              // [groups][Ep]
+    int32_t* part_pre = L.part + 4 * NT;     // [groups][Ep]   (groups * Ep <= 4 * NT)
+    // one group: sums go straight to cnt / base (the chunk histogram in cnt
+    // is no longer needed once published); several: partials, summed below
+    int32_t* dst_tot = groups == 1 ? L.cnt : part_tot;
+    int32_t* dst_pre = groups == 1 ? L.base : part_pre;
     {
-        const int cols = Ep / 4;
-        int groups = NT / cols;
-        if (groups > 8) groups = 8;
-        if (groups < 1) groups = 1;
-        int32_t* part_tot = L.part;              // [groups][Ep]
-        int32_t* part_pre = L.part + 4 * NT;     // [groups][Ep]   (groups * Ep <= 4 * NT)
-        // one group: sums go straight to cnt / base (the chunk histogram in cnt
-        // is no longer needed once published); several: partials, then a sum
-        int32_t* dst_tot = groups == 1 ? L.cnt : part_tot;
-        int32_t* dst_pre = groups == 1 ? L.base : part_pre;
         // the rows a chunk sums: the G super-chunk rows of this call (all of
         // them for the totals, those before its own super-chunk sg for its
         // prefix), then the chunk rows c0 .. c-1 of its own super-chunk
@@ -399,21 +398,12 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
             }
         }
         __syncthreads();
-        if (groups > 1) {
-            for (int e = tid; e < E; e += NT) {
-                int tot = 0, pre = 0;
-                for (int j = 0; j < groups; ++j) {
-                    tot += part_tot[j * Ep + e];
-                    pre += part_pre[j * Ep + e];
-                }
-                L.cnt[e] = tot;
-                L.base[e] = pre;
-            }
-            __syncthreads();
-        }
     }
-    // aligned offsets (high word) and padding prefix (low word) in one scan;
-    // each thread owns a run of consecutive experts
+    // Per expert, each thread owning a run of consecutive experts: its total and
+    // its sum over earlier chunks (the thread groups' partials added up), then
+    // the aligned offsets (high word) and padding prefix (low word) in one block
+    // scan.  Every per-expert value is written and read by its owner only until
+    // the barrier before the assign, so no other barrier is needed.
     const int ipt = (E + NT - 1) / NT;
     const int e0 = min(tid * ipt, E), e1 = min(e0 + ipt, E);
     long long loc = 0;
@@ -421,16 +411,31 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
     // rows: the rest (none when an expert overflows its slab)
     auto rows_of = [&](int e) { return a.slab > 0 ? a.slab : align_up_i(L.cnt[e], a.A); };
     for (int e = e0; e < e1; ++e) {
+        int tot = dst_tot[e], pre = dst_pre[e];
+        for (int j = 1; j < groups; ++j) {
+            tot += part_tot[j * Ep + e];
+            pre += part_pre[j * Ep + e];
+        }
+        L.cnt[e] = tot;
+        L.base[e] = pre;
         const int al = rows_of(e);
-        loc += ((long long)al << 32) + max(al - L.cnt[e], 0);
+        loc += ((long long)al << 32) + max(al - tot, 0);
     }
     long long total = 0;
     long long prefix = block_exclusive_scan64<NT>(loc, s_scratch, &total);
     for (int e = e0; e < e1; ++e) {
         const int al = rows_of(e);
-        L.off[e] = (int)(prefix >> 32);
-        L.padpre[e] = (int)(prefix & 0xffffffffll);
-        L.base[e] += (int)(prefix >> 32);
+        const int o = (int)(prefix >> 32), pp = (int)(prefix & 0xffffffffll);
+        L.off[e] = o;
+        L.padpre[e] = pp;
+        L.base[e] += o;
+        if (c == 0) {   // the per-expert outputs, written once
+            a.cnt[e] = L.cnt[e];
+            if (a.slab > 0 && L.cnt[e] > a.slab) s_over = 1;   // more pairs than the slab holds
+            if (a.stats) a.stats[e] += L.cnt[e];
+            a.off[e] = o;
+            a.padpre[e] = pp;
+        }
         prefix += ((long long)al << 32) + max(al - L.cnt[e], 0);
     }
     const int total_rows = (int)(total >> 32), total_pad = (int)(total & 0xffffffffll);
@@ -439,13 +444,6 @@ __device__ __forceinline__ bool layout_body(const LayoutArgs& a, int32_t* sm) {
         L.padpre[E] = total_pad;
     }
     if (c == 0) {
-        for (int e = tid; e < E; e += NT) {
-            a.cnt[e] = L.cnt[e];
-            if (a.slab > 0 && L.cnt[e] > a.slab) s_over = 1;   // more pairs than the slab holds
-            if (a.stats) a.stats[e] += L.cnt[e];
-            a.off[e] = L.off[e];
-            a.padpre[e] = L.padpre[e];
-        }
         if (tid == 0) {
             a.off[E] = total_rows;
             a.padpre[E] = total_pad;
