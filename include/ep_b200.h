@@ -25,6 +25,11 @@
  *                receive rows per expert.
  *   ep_layout_dispatch  ep_layout and ep_dispatch in one call (§2.1: V2's
  *                dispatch() derives its layout from topk_idx).
+ *   ep_source_offsets, ep_dispatch_regions, ep_combine_regions  several source
+ *                groups (the NVLink intranode path of §2.1 dispatch() seen
+ *                from one GPU): each group's write offsets in the layout of
+ *                the whole batch, and dispatch / combine over R receive
+ *                regions given as separate buffers.
  * The placement also matches the last stages of the Ascend full-mesh dispatch
  * on the "URMA" tag page (count reconciliation, prefix-sum placement, reorder).
  *
