@@ -147,3 +147,27 @@ def test_default_workload_is_the_largest_one_gpu_configuration(monkeypatch):
     cfg = bench.bench_config(args)
     assert max(workload.WORKLOADS, key=lambda n: workload.WORKLOADS[n]["T"]) == "large_prefill"
     assert (cfg["T"], cfg["H"], cfg["E"], cfg["K"], cfg["R"], cfg["A"]) == (16384, 7168, 256, 8, 64, 128)
+
+
+@pytest.mark.parametrize("body,expect", [
+    ('{"hbm_gbs": 6548.2}', (6548.2, "measured")),
+    ('{"hbm_gbs": {"value": 6500}}', (6500.0, "measured")),
+    ('{"hbm_gbs": {"gbs": 6400.5}}', (6400.5, "measured")),
+    ('{"bf16_tflops": 1590}', (6650.0, "fallback")),
+    ('{"hbm_gbs": null}', (6650.0, "fallback")),
+    ('{"hbm_gbs": -1}', (6650.0, "fallback")),
+    ('not json', (6650.0, "fallback")),
+])
+def test_measured_peaks_reader(tmp_path, monkeypatch, body, expect):
+    """The HBM denominator comes from MEASURED_PEAKS.json when it holds a
+    positive hbm_gbs (plain or under "value" / "gbs"), else the fallback."""
+    import bench
+    (tmp_path / "MEASURED_PEAKS.json").write_text(body)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_peaks() == expect
+
+
+def test_measured_peaks_absent(tmp_path, monkeypatch):
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_peaks() == (6650.0, "fallback")
